@@ -1,0 +1,447 @@
+"""Benchmark of the Gated DeltaNet mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--decode-workload NAME]
+
+Prints ONE JSON line (rank 0).  `value` is prefill tokens/s of one mixer layer
+over all ranks (each rank runs its own copy of the workload: the mixer is
+independent per sequence, so ranks share nothing and scaling is weak).  The
+decode half of the metric (one recurrent step for a batch of sequences on an
+fp32 state in HBM) is reported under "decode".
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; before every timed step a 256 MiB buffer is written
+to flush L2 (outside the events).  Max over ranks.  `roofline` reports the
+chunked-core kernel alone (CUDA events recorded by the library around that
+launch).  `e2e` repeats the prefill through the public API with the step's
+inputs copied from pinned host memory and the outputs copied back inside the
+timed region.  `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hybrid_linear_attention_05_b200.workloads import WORKLOADS, make_decode, make_prefill  # noqa: E402
+
+DEFAULT_PREFILL = "prefill_T4096_Hk16_Hv16_d128"
+DEFAULT_DECODE = "decode_B256_Hk16_Hv32_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------ work counts
+
+
+def prefill_counts(inp, chunk):
+    """Algorithmic bytes and FLOPs of one prefill (whole call) and of the
+    chunked-core kernel alone."""
+    w = inp.w
+    T, N, Hk, Hv, d = inp.T, inp.N, w.Hk, w.Hv, w.d
+    e = 2 if w.dtype == "bf16" else 4
+    state_in = 0 if inp.initial_state is None else N * Hv * d * d * 4
+    state_out = N * Hv * d * d * 4
+    # chunked core: normalised q, k, values, gates, z in; out and state out
+    core_bytes = (T * (2 * Hk * d * e + Hv * d * e + Hv * 8 + Hv * d * e + Hv * d * e)
+                  + state_in + state_out)
+    core_flops = T * Hv * (10 * chunk * d + 6 * d * d)
+    # whole call: mixed projection, a, b, z in, out, states, conv tail
+    call_bytes = (T * (w.Cc * e + 2 * Hv * e + Hv * d * e + Hv * d * e) + state_in + state_out
+                  + N * w.Cc * 3 * e)
+    return dict(core_bytes=core_bytes, core_flops=core_flops, call_bytes=call_bytes,
+                call_flops=core_flops)
+
+
+def decode_counts(inp):
+    w = inp.w
+    B, Hv, d = inp.mixed_qkv.shape[0], w.Hv, w.d
+    e = 2 if w.dtype == "bf16" else 4
+    state = 2 * B * Hv * d * d * 4
+    conv = 2 * B * w.Cc * 3 * e
+    io = B * (w.Cc * e + 2 * Hv * e + Hv * d * e + Hv * d * e)
+    return dict(bytes=state + conv + io, flops=B * Hv * 6 * d * d)
+
+
+# ------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------- CPU baseline
+
+
+def cpu_oracle_prefill_sample(inp, budget_s=12.0, max_threads=None):
+    """Time the fp64 oracle on the first `n` tokens of the first sequence
+    (all heads), growing n until the run takes about budget_s/4, then one
+    timed run at the size that fills the budget.  Returns (tokens/s, cores,
+    description)."""
+    import oracle
+    w = inp.w
+    threads = min(os.cpu_count() or 1, w.Hv * 1, max_threads or 1 << 30)
+    first = int(inp.cu_seqlens[1])
+
+    def run(n):
+        x0 = time.perf_counter()
+        oracle.prefill(w.Hk, w.Hv, w.d, w.d, [0, n], inp.mixed_qkv[:n], inp.conv_w, inp.a[:n],
+                       inp.b[:n], inp.A_log, inp.dt_bias, inp.z[:n], inp.norm_w,
+                       None if inp.initial_state is None else inp.initial_state[:1],
+                       None, scale=w.scale, nthreads=threads)
+        return time.perf_counter() - x0
+
+    n = min(32, first)
+    dt = run(n)
+    while dt < budget_s / 8 and n < first:
+        n = min(first, n * 2)
+        dt = run(n)
+    n_final = min(first, max(n, int(n * (budget_s / max(dt, 1e-6)))))
+    if n_final != n:
+        dt = run(n_final)
+        n = n_final
+    return n / dt, threads, "first %d tokens of one sequence, all %d value heads" % (n, w.Hv)
+
+
+def cpu_oracle_decode_sample(inp, budget_s=6.0):
+    import oracle
+    w = inp.w
+    threads = os.cpu_count() or 1
+    B_all = inp.mixed_qkv.shape[0]
+
+    def run(B):
+        x0 = time.perf_counter()
+        oracle.decode(w.Hk, w.Hv, w.d, w.d, inp.mixed_qkv[:B], inp.conv_w, inp.a[:B], inp.b[:B],
+                      inp.A_log, inp.dt_bias, inp.z[:B], inp.norm_w, inp.state[:B],
+                      inp.conv_state[:B], scale=w.scale, nthreads=threads)
+        return time.perf_counter() - x0
+
+    B = min(8, B_all)
+    dt = run(B)
+    while dt < budget_s / 4 and B < B_all:
+        B = min(B_all, B * 2)
+        dt = run(B)
+    return B / dt, threads, "%d of %d sequences, one token each" % (B, B_all)
+
+
+# ------------------------------------------------------------- GPU arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from hybrid_linear_attention_05_b200 import api, gdn
+    from hybrid_linear_attention_05_b200 import build as libbuild
+
+    libbuild.build()
+    gdn.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_kind = load_peaks()
+
+    wp = WORKLOADS[args.workload]
+    inp = make_prefill(wp)
+    dp = api.to_device(inp, device=dev, chunk=args.chunk)
+    bufs = api.PrefillBuffers(dp)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(core_ev=None):
+        api.prefill(dp, bufs=bufs, core_events=core_ev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    cevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for a, b in cevs:  # torch creates the CUDA event on first record; the library re-records it
+        a.record(stream)
+        b.record(stream)
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            step(core_ev=cevs[i])
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    core_ms = [a.elapsed_time(b) for a, b in cevs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = inp.T * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    cnt = prefill_counts(inp, dp.chunk)
+    core_avg_s = statistics.mean(core_ms) * 1e-3
+    hbm = peaks["hbm_gbs"]
+    roofline = {
+        "kernel": "gdn_chunk_tc" if dp.chunk == 64 else "gdn_chunk_simt",
+        "bound": "hbm",
+        "achieved": cnt["core_bytes"] / core_avg_s / 1e9,
+        "peak": hbm,
+        "unit": "GB/s",
+        "frac": cnt["core_bytes"] / core_avg_s / 1e9 / hbm,
+        "traffic": args.core_traffic,
+        "peak_source": peak_kind,
+        "algorithmic_bytes_per_launch": cnt["core_bytes"],
+        "algorithmic_flops_per_launch": cnt["core_flops"],
+        "kernel_us": core_avg_s * 1e6,
+        "tensor_tflops": cnt["core_flops"] / core_avg_s / 1e12,
+        "tensor_frac_of_burst": cnt["core_flops"] / core_avg_s / 1e12 / peaks["bf16_tflops"],
+        "whole_call_hbm_frac": cnt["call_bytes"] / (ms_per_step * 1e-3) / 1e9 / hbm,
+    }
+
+    # ---------------- e2e: pinned host inputs -> device -> prefill -> host
+    host = {k: torch.from_numpy(np.ascontiguousarray(getattr(inp, k))).to(dp.dtype).pin_memory()
+            for k in ("mixed_qkv", "a", "b", "z")}
+    h_cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).pin_memory()
+    h_S0 = None if inp.initial_state is None else torch.from_numpy(inp.initial_state).pin_memory()
+    h_out = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+    h_S = torch.empty(bufs.final_state.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + h_cu.numel() * 4 + (
+        0 if h_S0 is None else h_S0.numel() * 4)
+    d2h = h_out.numel() * h_out.element_size() + h_S.numel() * 4
+
+    def e2e_step():
+        for k, t in host.items():
+            getattr(dp, k).copy_(t, non_blocking=True)
+        dp.cu_seqlens.copy_(h_cu, non_blocking=True)
+        if h_S0 is not None:
+            dp.initial_state.copy_(h_S0, non_blocking=True)
+        api.prefill(dp, bufs=bufs)
+        h_out.copy_(bufs.out, non_blocking=True)
+        h_S.copy_(bufs.final_state, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e = {"value": tokens / (e2e_total / args.steps * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    del host, h_out, h_S
+
+    # ---------------- decode half of the metric
+    wd = WORKLOADS[args.decode_workload]
+    dinp = make_decode(wd)
+    dd = api.decode_to_device(dinp, device=dev)
+    dout = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dev)
+    for _ in range(args.warmup):
+        api.decode(dd, out=dout)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    dev_ms = []
+    for i in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        api.decode(dd, out=dout)
+        b.record(stream)
+        dev_ms.append((a, b))
+    torch.cuda.synchronize()
+    d_ms = [a.elapsed_time(b) for a, b in dev_ms]
+    d_total = sum(d_ms)
+    if world > 1:
+        t = torch.tensor([d_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        d_total = float(t.item())
+    dcnt = decode_counts(dinp)
+    d_step_s = d_total / args.steps * 1e-3
+    decode = {
+        "metric": "GDN decode tokens/s per layer", "unit": "tokens/s",
+        "value": dd.B * world / d_step_s, "ms_per_step": d_step_s * 1e3,
+        "workload": args.decode_workload,
+        "roofline": {"kernel": "gdn_decode", "bound": "hbm",
+                     "achieved": dcnt["bytes"] / d_step_s / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": dcnt["bytes"] / d_step_s / 1e9 / hbm, "traffic": args.decode_traffic,
+                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": dcnt["bytes"]},
+        "l2": "state (%d MiB) larger than L2" % (dd.state.numel() * 4 >> 20),
+    }
+    del dd
+
+    result = {
+        "metric": "GDN prefill tokens/s per layer (decode tokens/s under 'decode')",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wp.dtype, "data": "synthetic",
+        "config": {"workload": args.workload, "sequences": inp.N, "tokens": inp.T,
+                   "key_heads": wp.Hk, "value_heads": wp.Hv, "head_dim": wp.d,
+                   "chunk": dp.chunk, "parallelism": "replica per GPU (weak)",
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": roofline,
+        "decode": decode,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return result, inp, dinp
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_PREFILL)
+    ap.add_argument("--decode-workload", default=DEFAULT_DECODE)
+    ap.add_argument("--chunk", type=int, default=None, help="override the workload's chunk length")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--core-traffic", type=float, default=None,
+                    help="dram bytes per chunked-core launch from an ncu capture of this build")
+    ap.add_argument("--decode-traffic", type=float, default=None)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # The reference arm is the fp64 CPU oracle (no reference implementation
+        # exists to install); rank 0 runs it, other ranks exit without work.
+        if rank != 0:
+            return
+        wp = WORKLOADS[args.workload]
+        inp = make_prefill(wp)
+        vals = []
+        for i in range(args.warmup + args.steps):
+            v, cores, sample = cpu_oracle_prefill_sample(inp, budget_s=3.0)
+            if i >= args.warmup:
+                vals.append(v)
+        value = statistics.mean(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": "GDN prefill tokens/s per layer", "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": inp.T / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "tokens": inp.T},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    result, inp, dinp = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            v, cores, sample = cpu_oracle_prefill_sample(inp)
+            result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
+                                      "kind": "oracle", "sample": sample}
+            dv, dcores, dsample = cpu_oracle_decode_sample(dinp)
+            result["decode"]["cpu_baseline"] = {"value": dv, "unit": "tokens/s", "cores": dcores,
+                                                "kind": "oracle", "sample": dsample}
+        print(json.dumps(result))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

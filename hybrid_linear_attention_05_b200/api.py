@@ -1,0 +1,148 @@
+"""Tensor-level convenience calls over the C ABI.
+
+``prefill`` and ``decode`` take torch CUDA tensors, allocate the outputs and
+the workspace with torch, and call ``gdn_prefill`` / ``gdn_decode`` on the
+current stream.  ``to_device`` moves a seeded workload (numpy arrays from
+``workloads``) onto the GPU in the workload's dtype.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import gdn
+from .workloads import DecodeInputs, PrefillInputs
+
+
+def _torch_dtype(name: str):
+    return torch.bfloat16 if name == "bf16" else torch.float32
+
+
+@dataclass
+class DevicePrefill:
+    Hk: int
+    Hv: int
+    d: int
+    chunk: int
+    scale: float
+    N: int
+    T: int
+    cu_seqlens: torch.Tensor
+    mixed_qkv: torch.Tensor
+    conv_w: torch.Tensor
+    a: torch.Tensor
+    b: torch.Tensor
+    A_log: torch.Tensor
+    dt_bias: torch.Tensor
+    z: torch.Tensor
+    norm_w: torch.Tensor
+    initial_state: Optional[torch.Tensor]
+    conv_state_in: Optional[torch.Tensor]
+
+    @property
+    def dtype(self):
+        return self.mixed_qkv.dtype
+
+    @property
+    def Cc(self):
+        return 2 * self.Hk * self.d + self.Hv * self.d
+
+
+def to_device(inp: PrefillInputs, device="cuda", chunk: Optional[int] = None) -> DevicePrefill:
+    w = inp.w
+    dt = _torch_dtype(w.dtype)
+
+    def t(x, dtype=dt):
+        return None if x is None else torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dtype)
+
+    return DevicePrefill(
+        Hk=w.Hk, Hv=w.Hv, d=w.d, chunk=chunk or w.chunk, scale=w.scale, N=inp.N, T=inp.T,
+        cu_seqlens=t(inp.cu_seqlens, torch.int32), mixed_qkv=t(inp.mixed_qkv), conv_w=t(inp.conv_w),
+        a=t(inp.a), b=t(inp.b), A_log=t(inp.A_log, torch.float32),
+        dt_bias=t(inp.dt_bias, torch.float32), z=t(inp.z), norm_w=t(inp.norm_w),
+        initial_state=t(inp.initial_state, torch.float32), conv_state_in=t(inp.conv_state_in))
+
+
+@dataclass
+class PrefillOut:
+    out: torch.Tensor            # [T, Hv, d]
+    final_state: torch.Tensor    # [N, Hv, d, d] fp32
+    conv_state_out: torch.Tensor  # [N, Cc, 3]
+
+
+class PrefillBuffers:
+    """Outputs and workspace for repeated prefill calls on one shape."""
+
+    def __init__(self, dp: DevicePrefill):
+        dev = dp.mixed_qkv.device
+        self.dims = gdn.make_dims(dp.Hk, dp.Hv, dp.d, scale=dp.scale)
+        self.dtype_code = gdn.dtype_code(dp.mixed_qkv)
+        self.out = torch.empty((dp.T, dp.Hv, dp.d), dtype=dp.dtype, device=dev)
+        self.final_state = torch.empty((dp.N, dp.Hv, dp.d, dp.d), dtype=torch.float32, device=dev)
+        self.conv_state_out = torch.empty((dp.N, dp.Cc, 3), dtype=dp.dtype, device=dev)
+        self.ws_bytes = gdn.gdn_prefill_workspace_size(self.dims, dp.T, self.dtype_code)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+
+def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[PrefillBuffers] = None,
+            core_events=None) -> PrefillOut:
+    bufs = bufs or PrefillBuffers(dp)
+    ev0, ev1 = (None, None) if core_events is None else (core_events[0].cuda_event,
+                                                         core_events[1].cuda_event)
+    gdn.gdn_prefill(
+        bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b, A_log=dp.A_log,
+        dt_bias=dp.dt_bias, z=dp.z, norm_w=dp.norm_w, cu_seqlens=dp.cu_seqlens, N=dp.N,
+        T_tot=dp.T, chunk=dp.chunk, dtype=bufs.dtype_code, out=bufs.out,
+        workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
+        initial_state=dp.initial_state, final_state=bufs.final_state,
+        conv_state_in=dp.conv_state_in, conv_state_out=bufs.conv_state_out, impl=impl,
+        core_event_begin=ev0, core_event_end=ev1)
+    return PrefillOut(bufs.out, bufs.final_state, bufs.conv_state_out)
+
+
+@dataclass
+class DeviceDecode:
+    Hk: int
+    Hv: int
+    d: int
+    scale: float
+    B: int
+    mixed_qkv: torch.Tensor
+    conv_w: torch.Tensor
+    a: torch.Tensor
+    b: torch.Tensor
+    A_log: torch.Tensor
+    dt_bias: torch.Tensor
+    z: torch.Tensor
+    norm_w: torch.Tensor
+    state: torch.Tensor
+    conv_state: torch.Tensor
+
+
+def decode_to_device(inp: DecodeInputs, device="cuda") -> DeviceDecode:
+    w = inp.w
+    dt = _torch_dtype(w.dtype)
+
+    def t(x, dtype=dt):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dtype)
+
+    return DeviceDecode(
+        Hk=w.Hk, Hv=w.Hv, d=w.d, scale=w.scale, B=inp.mixed_qkv.shape[0],
+        mixed_qkv=t(inp.mixed_qkv), conv_w=t(inp.conv_w), a=t(inp.a), b=t(inp.b),
+        A_log=t(inp.A_log, torch.float32), dt_bias=t(inp.dt_bias, torch.float32), z=t(inp.z),
+        norm_w=t(inp.norm_w), state=t(inp.state, torch.float32), conv_state=t(inp.conv_state))
+
+
+def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One step; dd.state and dd.conv_state are updated in place."""
+    if out is None:
+        out = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dd.mixed_qkv.device)
+    dims = gdn.make_dims(dd.Hk, dd.Hv, dd.d, scale=dd.scale)
+    gdn.gdn_decode(dims, mixed_qkv=dd.mixed_qkv, conv_w=dd.conv_w, a=dd.a, b=dd.b,
+                   A_log=dd.A_log, dt_bias=dd.dt_bias, z=dd.z, norm_w=dd.norm_w, state=dd.state,
+                   conv_state=dd.conv_state, out=out, B=dd.B,
+                   dtype=gdn.dtype_code(dd.mixed_qkv))
+    return out

@@ -1,0 +1,177 @@
+// One decode step of the Gated DeltaNet mixer for a batch of sequences.
+//
+// One CTA per (sequence, key head) owns the G = Hv/Hk value heads that read
+// that key head, so the conv-cache channels it updates in place (its q and k
+// head, and its G value heads) belong to no other CTA.
+//   1. conv over (cache[0..2], new input) + SiLU for those channels, cache
+//      shifted left with the new raw input appended;
+//   2. L2 norm of q and k, gates alpha = exp(-exp(A_log) softplus(a+dt_bias)),
+//      beta = sigmoid(b);
+//   3. each state row S[r, :] (dk floats) is read once from HBM and written
+//      once: u = S k, p = S q, delta = beta (v - alpha u),
+//      S' = alpha S + delta k^T, o = alpha p + (k.q) delta   (= S' q);
+//   4. gated RMSNorm of o with z.
+// The state rows are spread over the warps with each lane holding a float4 of
+// a row; row dot products are shuffle reductions over the lanes of the row.
+// HBM traffic is dominated by the fp32 state: 2 * Hv * dk * dv * 4 bytes per
+// token ("Qwen3.5", HF model doc, Usage tips: the single-token recurrence is
+// memory-bandwidth-bound).
+#include "gdn_internal.h"
+
+namespace gdn {
+
+namespace {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
+  constexpr int NT = 256, NW = NT / 32;
+  constexpr int LPR = D / 4;            // lanes per state row
+  constexpr int RPW = 32 / LPR;         // rows per warp per pass
+  constexpr int ROWS_PER_WARP = D / NW; // rows of one head handled by a warp
+  constexpr int PASSES = ROWS_PER_WARP / RPW;
+  static_assert(PASSES >= 1, "decode layout");
+
+  extern __shared__ float sm[];
+  const int G = p.Hv / p.Hk;
+  float* ys = sm;                 // [(2 + G) * D] q | k | v of this CTA
+  float* os = ys + (2 + G) * D;   // [G * D] core outputs
+  float* misc = os + G * D;       // [4 + 2G]: rq, rk, kq, -, alpha[G], beta[G]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x / p.Hk, kh = blockIdx.x % p.Hk;
+  const int Cc = p.Cc;
+  const int NC = (2 + G) * D;
+  const T* xrow = static_cast<const T*>(p.x) + (size_t)b * Cc;
+  T* cs = static_cast<T*>(p.conv_state) + (size_t)b * Cc * 3;
+  const T* cw = static_cast<const T*>(p.conv_w);
+
+  // 1. conv + SiLU, cache update in place (each channel read then written by one thread)
+  for (int idx = tid; idx < NC; idx += NT) {
+    int c;
+    if (idx < D) c = kh * D + idx;
+    else if (idx < 2 * D) c = p.Hk * D + kh * D + (idx - D);
+    else c = 2 * p.Hk * D + kh * G * D + (idx - 2 * D);
+    const float xn = ld_f(xrow + c);
+    const float h0 = ld_f(cs + (size_t)c * 3 + 0);
+    const float h1 = ld_f(cs + (size_t)c * 3 + 1);
+    const float h2 = ld_f(cs + (size_t)c * 3 + 2);
+    float y = ld_f(cw + (size_t)c * 4 + 0) * h0;
+    y = fmaf(ld_f(cw + (size_t)c * 4 + 1), h1, y);
+    y = fmaf(ld_f(cw + (size_t)c * 4 + 2), h2, y);
+    y = fmaf(ld_f(cw + (size_t)c * 4 + 3), xn, y);
+    ys[idx] = silu_f(y);
+    st_f(cs + (size_t)c * 3 + 0, h1);
+    st_f(cs + (size_t)c * 3 + 1, h2);
+    st_f(cs + (size_t)c * 3 + 2, xn);
+  }
+  __syncthreads();
+  // 2. norms and gates
+  if (warp < 2) {
+    float ss = 0.f;
+    for (int i = lane; i < D; i += 32) { const float v = ys[warp * D + i]; ss = fmaf(v, v, ss); }
+    ss = warp_sum(ss);
+    if (lane == 0) misc[warp] = rsqrtf(ss + p.eps_l2) * (warp == 0 ? p.scale : 1.0f);
+  } else if (warp == 2) {
+    for (int gi = lane; gi < G; gi += 32) {
+      const int h = kh * G + gi;
+      const float av = ld_f(static_cast<const T*>(p.a) + (size_t)b * p.Hv + h);
+      const float bv = ld_f(static_cast<const T*>(p.b) + (size_t)b * p.Hv + h);
+      const float gg = -expf(__ldg(p.A_log + h)) * softplus_f(av + __ldg(p.dt_bias + h));
+      misc[4 + gi] = expf(gg);
+      misc[4 + G + gi] = sigmoid_f(bv);
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < 2 * D; i += NT) ys[i] *= misc[i < D ? 0 : 1];
+  __syncthreads();
+  if (warp == 0) {
+    float kq = 0.f;
+    for (int i = lane; i < D; i += 32) kq = fmaf(ys[i], ys[D + i], kq);
+    kq = warp_sum(kq);
+    if (lane == 0) misc[2] = kq;
+  }
+  __syncthreads();
+
+  // 3. state stream
+  const float* qv = ys;
+  const float* kv = ys + D;
+  const int col = (lane % LPR) * 4;
+  const float4 k4 = make_float4(kv[col], kv[col + 1], kv[col + 2], kv[col + 3]);
+  const float4 q4 = make_float4(qv[col], qv[col + 1], qv[col + 2], qv[col + 3]);
+  const float kq = misc[2];
+  for (int gi = 0; gi < G; ++gi) {
+    const int h = kh * G + gi;
+    const float alpha = misc[4 + gi], beta = misc[4 + G + gi];
+    float* Sh = p.state + ((size_t)b * p.Hv + h) * D * D;
+    const float* vv = ys + (2 + gi) * D;
+    float4 Sv[PASSES];
+#pragma unroll
+    for (int s = 0; s < PASSES; ++s) {
+      const int r = warp * ROWS_PER_WARP + s * RPW + lane / LPR;
+      Sv[s] = *reinterpret_cast<const float4*>(Sh + (size_t)r * D + col);
+    }
+#pragma unroll
+    for (int s = 0; s < PASSES; ++s) {
+      const int r = warp * ROWS_PER_WARP + s * RPW + lane / LPR;
+      float u = Sv[s].x * k4.x + Sv[s].y * k4.y + Sv[s].z * k4.z + Sv[s].w * k4.w;
+      float pp = Sv[s].x * q4.x + Sv[s].y * q4.y + Sv[s].z * q4.z + Sv[s].w * q4.w;
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) {
+        u += __shfl_xor_sync(0xffffffffu, u, o, 32);
+        pp += __shfl_xor_sync(0xffffffffu, pp, o, 32);
+      }
+      const float delta = beta * (vv[r] - alpha * u);
+      float4 sn;
+      sn.x = fmaf(alpha, Sv[s].x, delta * k4.x);
+      sn.y = fmaf(alpha, Sv[s].y, delta * k4.y);
+      sn.z = fmaf(alpha, Sv[s].z, delta * k4.z);
+      sn.w = fmaf(alpha, Sv[s].w, delta * k4.w);
+      *reinterpret_cast<float4*>(Sh + (size_t)r * D + col) = sn;
+      if ((lane % LPR) == 0) os[gi * D + r] = fmaf(alpha, pp, kq * delta);
+    }
+  }
+  __syncthreads();
+
+  // 4. gated RMSNorm, one warp per value head
+  for (int gi = warp; gi < G; gi += NW) {
+    const int h = kh * G + gi;
+    float ss = 0.f;
+    for (int r = lane; r < D; r += 32) { const float o = os[gi * D + r]; ss = fmaf(o, o, ss); }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / D + p.eps_norm);
+    const T* zz = static_cast<const T*>(p.z) + ((size_t)b * p.Hv + h) * D;
+    T* oo = static_cast<T*>(p.out) + ((size_t)b * p.Hv + h) * D;
+    const T* ww = static_cast<const T*>(p.norm_w);
+    for (int r = lane; r < D; r += 32)
+      st_f(oo + r, os[gi * D + r] * inv * ld_f(ww + r) * silu_f(ld_f(zz + r)));
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
+  const int G = p.Hv / p.Hk;
+  const size_t smem = ((size_t)(2 + G) * D + (size_t)G * D + 4 + 2 * G) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_kernel<T, D><<<p.B * p.Hk, 256, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, int d, gdn_dtype dt, cudaStream_t st) {
+  if (p.B == 0) return cudaSuccess;
+  if (dt == GDN_BF16) {
+    if (d == 128) return launch_t<__nv_bfloat16, 128>(p, st);
+    if (d == 64) return launch_t<__nv_bfloat16, 64>(p, st);
+    return launch_t<__nv_bfloat16, 32>(p, st);
+  }
+  if (d == 128) return launch_t<float, 128>(p, st);
+  if (d == 64) return launch_t<float, 64>(p, st);
+  return launch_t<float, 32>(p, st);
+}
+
+}  // namespace gdn

@@ -1,0 +1,210 @@
+// C ABI of the library: host-side validation, workspace carving and kernel
+// dispatch.  See include/gdn.h for the contract of every entry point.
+#include <stdint.h>
+#include <string.h>
+
+#include "gdn_internal.h"
+
+using namespace gdn;
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+size_t esize(gdn_dtype dt) { return dt == GDN_BF16 ? 2 : 4; }
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+gdn_status check_dims(const gdn_dims* d) {
+  if (!d) return GDN_ERR_NULL;
+  if (d->Hk < 1 || d->Hv < 1 || d->Hv % d->Hk != 0 || d->dk < 1 || d->dv < 1 || d->conv_k < 1)
+    return GDN_ERR_DIMS;
+  if (!(d->eps_l2 >= 0.f) || !(d->eps_norm >= 0.f) || !(d->scale == d->scale)) return GDN_ERR_DIMS;
+  if (d->dk != d->dv || d->conv_k != 4) return GDN_ERR_UNSUPPORTED;
+  if (d->dk != 32 && d->dk != 64 && d->dk != 128) return GDN_ERR_UNSUPPORTED;
+  // keep every packed row index below 2^31 elements
+  if ((int64_t)(2 * d->Hk + d->Hv) * d->dk > (1 << 24)) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+bool dtype_ok(gdn_dtype dt) { return dt == GDN_F32 || dt == GDN_BF16; }
+bool core_dtype_ok(gdn_dtype dt) { return dt == GDN_F32 || dt == GDN_BF16 || dt == GDN_F16; }
+// Type of the normalised q, k and v between the kernels of gdn_prefill.
+gdn_dtype mid_dtype(gdn_dtype in) { return in == GDN_BF16 ? GDN_F16 : GDN_F32; }
+
+struct Workspace {
+  void* q; void* k; void* v; float* g; float* beta;
+  size_t bytes;
+};
+
+Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base) {
+  Workspace w{};
+  const size_t e = esize(dt);
+  const size_t nq = align_up((size_t)T * d->Hk * d->dk * e, 256);
+  const size_t nv = align_up((size_t)T * d->Hv * d->dv * e, 256);
+  const size_t ng = align_up((size_t)T * d->Hv * sizeof(float), 256);
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  w.q = p ? p + off : nullptr; off += nq;
+  w.k = p ? p + off : nullptr; off += nq;
+  w.v = p ? p + off : nullptr; off += nv;
+  w.g = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
+  w.beta = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
+  w.bytes = off;
+  return w;
+}
+
+enum class Path { None, Simt, Tc };
+
+Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid) {
+  const bool tc = chunk_tc_supported(d, chunk, dt_mid);
+  const bool simt = chunk_simt_supported(d, chunk);
+  switch (impl) {
+    case GDN_IMPL_TC: return tc ? Path::Tc : Path::None;
+    case GDN_IMPL_SIMT: return simt ? Path::Simt : Path::None;
+    case GDN_IMPL_AUTO: return tc ? Path::Tc : (simt ? Path::Simt : Path::None);
+  }
+  return Path::None;
+}
+
+gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dtype) {
+  if (check_dims(dims) != GDN_OK || T_tot < 0 || !dtype_ok(dtype)) return 0;
+  return carve(dims, T_tot, dtype, nullptr).bytes;
+}
+
+gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (!a) return GDN_ERR_NULL;
+  if (a->N < 0 || a->T_tot < 0) return GDN_ERR_DIMS;
+  if (!dtype_ok(a->dtype)) return GDN_ERR_DIMS;
+  if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
+  const int d = dims->dk;
+  const int Cc = 2 * dims->Hk * d + dims->Hv * d;
+  const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype));
+  if (path == Path::None) return GDN_ERR_UNSUPPORTED;
+  if (!a->cu_seqlens || !a->conv_w || !a->A_log || !a->dt_bias || !a->norm_w) return GDN_ERR_NULL;
+  if (a->T_tot > 0 && (!a->mixed_qkv || !a->a || !a->b || !a->z || !a->out || !a->workspace))
+    return GDN_ERR_NULL;
+  const void* ptrs[] = {a->mixed_qkv, a->conv_w, a->a, a->b, a->A_log, a->dt_bias, a->z,
+                        a->norm_w, a->cu_seqlens, a->initial_state, a->final_state,
+                        a->conv_state_in, a->conv_state_out, a->out, a->workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const Workspace need = carve(dims, a->T_tot, a->dtype, nullptr);
+  if (a->T_tot > 0 && a->workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
+  const size_t cs_bytes = (size_t)a->N * Cc * 3 * esize(a->dtype);
+  if (overlap(a->conv_state_in, cs_bytes, a->conv_state_out, cs_bytes)) return GDN_ERR_ALIAS;
+  const size_t st_bytes = (size_t)a->N * dims->Hv * d * d * sizeof(float);
+  if (a->initial_state != a->final_state && overlap(a->initial_state, st_bytes, a->final_state, st_bytes))
+    return GDN_ERR_ALIAS;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Workspace ws = carve(dims, a->T_tot, a->dtype, a->workspace);
+
+  ConvPrepParams cp{};
+  cp.x = a->mixed_qkv; cp.conv_w = a->conv_w; cp.a = a->a; cp.b = a->b;
+  cp.A_log = a->A_log; cp.dt_bias = a->dt_bias; cp.cu_seqlens = a->cu_seqlens;
+  cp.conv_state_in = a->conv_state_in; cp.conv_state_out = a->conv_state_out;
+  cp.q = ws.q; cp.k = ws.k; cp.v = ws.v; cp.g = ws.g; cp.beta = ws.beta;
+  cp.T = a->T_tot; cp.N = a->N; cp.Hk = dims->Hk; cp.Hv = dims->Hv; cp.Cc = Cc;
+  cp.scale = dims->scale; cp.eps_l2 = dims->eps_l2;
+  s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
+  if (s != GDN_OK) return s;
+
+  ChunkParams ch{};
+  ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
+  ch.cu_seqlens = a->cu_seqlens; ch.S0 = a->initial_state; ch.S_out = a->final_state;
+  ch.z = a->z; ch.norm_w = a->norm_w; ch.out = a->out; ch.o_raw = nullptr;
+  ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
+  ch.eps_norm = dims->eps_norm;
+  if (a->core_event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_begin), st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  s = from_cuda(path == Path::Tc ? launch_chunk_tc(ch, st)
+                                 : launch_chunk_simt(ch, d, a->dtype, mid_dtype(a->dtype), st));
+  if (s != GDN_OK) return s;
+  if (a->core_event_end && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_end), st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return GDN_OK;
+}
+
+gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* a, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (!a) return GDN_ERR_NULL;
+  if (a->B < 0 || !dtype_ok(a->dtype)) return GDN_ERR_DIMS;
+  if (a->B == 0) return GDN_OK;
+  if (!a->mixed_qkv || !a->conv_w || !a->a || !a->b || !a->A_log || !a->dt_bias || !a->z ||
+      !a->norm_w || !a->state || !a->conv_state || !a->out)
+    return GDN_ERR_NULL;
+  const void* ptrs[] = {a->mixed_qkv, a->conv_w, a->a, a->b, a->A_log, a->dt_bias, a->z,
+                        a->norm_w, a->state, a->conv_state, a->out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const int d = dims->dk;
+  DecodeParams p{};
+  p.x = a->mixed_qkv; p.conv_w = a->conv_w; p.a = a->a; p.b = a->b;
+  p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.z = a->z; p.norm_w = a->norm_w;
+  p.state = a->state; p.conv_state = a->conv_state; p.out = a->out;
+  p.B = a->B; p.Hk = dims->Hk; p.Hv = dims->Hv; p.Cc = 2 * dims->Hk * d + dims->Hv * d;
+  p.scale = dims->scale; p.eps_l2 = dims->eps_l2; p.eps_norm = dims->eps_norm;
+  return from_cuda(launch_decode(p, d, a->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (!a) return GDN_ERR_NULL;
+  if (a->N < 0 || a->T_tot < 0 || !core_dtype_ok(a->dtype)) return GDN_ERR_DIMS;
+  if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
+  const int d = dims->dk;
+  const Path path = pick_path(a->impl, d, a->chunk, a->dtype);
+  if (path == Path::None) return GDN_ERR_UNSUPPORTED;
+  if (!a->cu_seqlens) return GDN_ERR_NULL;
+  if (a->T_tot > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o)) return GDN_ERR_NULL;
+  const void* ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
+                        a->final_state, a->o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const size_t st_bytes = (size_t)a->N * dims->Hv * d * d * sizeof(float);
+  if (a->initial_state != a->final_state && overlap(a->initial_state, st_bytes, a->final_state, st_bytes))
+    return GDN_ERR_ALIAS;
+  ChunkParams ch{};
+  ch.q = a->q; ch.k = a->k; ch.v = a->v; ch.g = a->g; ch.beta = a->beta;
+  ch.cu_seqlens = a->cu_seqlens; ch.S0 = a->initial_state; ch.S_out = a->final_state;
+  ch.z = nullptr; ch.norm_w = nullptr; ch.out = nullptr; ch.o_raw = a->o;
+  ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
+  ch.eps_norm = dims->eps_norm;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return from_cuda(path == Path::Tc ? launch_chunk_tc(ch, st)
+                                    : launch_chunk_simt(ch, d, GDN_F32, a->dtype, st));
+}
+
+const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_NULL: return "a required pointer is NULL";
+    case GDN_ERR_DIMS: return "inconsistent or out-of-range sizes";
+    case GDN_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case GDN_ERR_UNSUPPORTED: return "shape or option not supported by this build";
+    case GDN_ERR_CUDA: return "a CUDA call failed";
+    case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDN_ERR_ALIAS: return "buffers that must not overlap overlap";
+  }
+  return "unknown status";
+}
+
+const char* gdn_version(void) { return "gdn-b200 0.1"; }
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Internal launch interfaces between the C-ABI layer (gdn_api.cu) and the
+// kernels.  Nothing here is exported from the shared library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+// conv_prep.cu
+struct ConvPrepParams {
+  const void* x;              // [T, Cc]
+  const void* conv_w;         // [Cc, 4]
+  const void* a;              // [T, Hv]
+  const void* b;              // [T, Hv]
+  const float* A_log;         // [Hv]
+  const float* dt_bias;       // [Hv]
+  const int32_t* cu_seqlens;  // [N+1]
+  const void* conv_state_in;  // [N, Cc, 3] or null
+  void* conv_state_out;       // [N, Cc, 3] or null
+  void* q;                    // [T, Hk, d]  fp16 (bf16 inputs) or fp32
+  void* k;                    // [T, Hk, d]
+  void* v;                    // [T, Hv, d]
+  float* g;                   // [Hv, T]
+  float* beta;                // [Hv, T]
+  int T, N, Hk, Hv, Cc;
+  float scale, eps_l2;
+  int tok_blocks;             // set by the launcher
+};
+cudaError_t launch_conv_prep(const ConvPrepParams& p, int d, gdn_dtype dt, cudaStream_t st);
+
+// Parameters of the chunked core (both implementations).
+struct ChunkParams {
+  const void* q;              // [T, Hk, d]
+  const void* k;              // [T, Hk, d]
+  const void* v;              // [T, Hv, d]
+  const float* g;             // [Hv, T]
+  const float* beta;          // [Hv, T]
+  const int32_t* cu_seqlens;  // [N+1]
+  const float* S0;            // [N, Hv, d, d] or null
+  float* S_out;               // [N, Hv, d, d] or null
+  // gated-norm epilogue (when out != null)
+  const void* z;              // [T, Hv*d]
+  const void* norm_w;         // [d]
+  void* out;                  // [T, Hv, d]
+  float* o_raw;               // [T, Hv, d] fp32 core output (when out == null)
+  int T, N, Hk, Hv, chunk;
+  float eps_norm;
+};
+
+// chunk_simt.cu: fp32 CUDA-core chunked core.  Supported (d, chunk) pairs:
+// d in {32, 64} with chunk in {16, 32, 64}; d = 128 with chunk in {16, 32}.
+bool chunk_simt_supported(int d, int chunk);
+// dt_out: dtype of z / norm_w / out; dt_mid: dtype of q, k, v.
+cudaError_t launch_chunk_simt(const ChunkParams& p, int d, gdn_dtype dt_out, gdn_dtype dt_mid,
+                              cudaStream_t st);
+
+// chunk_tc.cu: tcgen05 chunked core, fp16 operands (q, k, v of dtype
+// dt_mid = GDN_F16), d = 128, chunk = 64.
+bool chunk_tc_supported(int d, int chunk, gdn_dtype dt_mid);
+cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st);
+
+// decode.cu
+struct DecodeParams {
+  const void* x;              // [B, Cc]
+  const void* conv_w;         // [Cc, 4]
+  const void* a;              // [B, Hv]
+  const void* b;              // [B, Hv]
+  const float* A_log;
+  const float* dt_bias;
+  const void* z;              // [B, Hv*d]
+  const void* norm_w;         // [d]
+  float* state;               // [B, Hv, d, d]
+  void* conv_state;           // [B, Cc, 3]
+  void* out;                  // [B, Hv, d]
+  int B, Hk, Hv, Cc;
+  float scale, eps_l2, eps_norm;
+};
+cudaError_t launch_decode(const DecodeParams& p, int d, gdn_dtype dt, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,188 @@
+"""Thin ctypes binding of the C ABI in ``include/gdn.h``.
+
+Argument marshalling only: every step of the mixer runs in the CUDA library.
+torch tensors are accepted for convenience (their device pointers and the
+current CUDA stream are passed through); plain integer device pointers work
+too.  The library is loaded from this package directory; if it is missing
+the import of the binding fails loudly -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgdn_b200.so")
+
+GDN_OK = 0
+GDN_ERR_NULL = -1
+GDN_ERR_DIMS = -2
+GDN_ERR_ALIGN = -3
+GDN_ERR_UNSUPPORTED = -4
+GDN_ERR_CUDA = -5
+GDN_ERR_WORKSPACE = -6
+GDN_ERR_ALIAS = -7
+
+GDN_F32 = 0
+GDN_BF16 = 1
+GDN_F16 = 2
+
+GDN_IMPL_AUTO = 0
+GDN_IMPL_SIMT = 1
+GDN_IMPL_TC = 2
+
+EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_chunk_core",
+            "gdn_status_string", "gdn_version"]
+
+
+class gdn_dims(ctypes.Structure):
+    _fields_ = [("Hk", ctypes.c_int), ("Hv", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("conv_k", ctypes.c_int), ("scale", ctypes.c_float),
+                ("eps_l2", ctypes.c_float), ("eps_norm", ctypes.c_float)]
+
+
+_vp = ctypes.c_void_p
+
+
+class gdn_prefill_args(ctypes.Structure):
+    _fields_ = [("mixed_qkv", _vp), ("conv_w", _vp), ("a", _vp), ("b", _vp), ("A_log", _vp),
+                ("dt_bias", _vp), ("z", _vp), ("norm_w", _vp), ("cu_seqlens", _vp),
+                ("N", ctypes.c_int), ("T_tot", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("impl", ctypes.c_int),
+                ("initial_state", _vp), ("final_state", _vp), ("conv_state_in", _vp),
+                ("conv_state_out", _vp), ("out", _vp), ("workspace", _vp),
+                ("workspace_bytes", ctypes.c_size_t), ("core_event_begin", _vp),
+                ("core_event_end", _vp)]
+
+
+class gdn_decode_args(ctypes.Structure):
+    _fields_ = [("mixed_qkv", _vp), ("conv_w", _vp), ("a", _vp), ("b", _vp), ("A_log", _vp),
+                ("dt_bias", _vp), ("z", _vp), ("norm_w", _vp), ("state", _vp),
+                ("conv_state", _vp), ("out", _vp), ("B", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class gdn_core_args(ctypes.Structure):
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp),
+                ("cu_seqlens", _vp), ("N", ctypes.c_int), ("T_tot", ctypes.c_int),
+                ("chunk", ctypes.c_int), ("dtype", ctypes.c_int), ("impl", ctypes.c_int),
+                ("initial_state", _vp), ("final_state", _vp), ("o", _vp)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libgdn_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libgdn_b200.so is missing; build it with "
+                "`python -m hybrid_linear_attention_05_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.gdn_prefill_workspace_size.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
+        L.gdn_prefill_workspace_size.restype = ctypes.c_size_t
+        L.gdn_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args), _vp]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_decode_args), _vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_chunk_core.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_core_args), _vp]
+        L.gdn_chunk_core.restype = ctypes.c_int
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (%d)" % (where, status_string(status), status))
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def make_dims(Hk, Hv, dk, dv=None, scale=None, eps_l2=1e-6, eps_norm=1e-6, conv_k=4) -> gdn_dims:
+    dv = dk if dv is None else dv
+    return gdn_dims(int(Hk), int(Hv), int(dk), int(dv), int(conv_k),
+                    float(dk ** -0.5 if scale is None else scale), float(eps_l2), float(eps_norm))
+
+
+def ptr(x) -> Optional[int]:
+    """Device pointer of a tensor (or pass-through int / None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.float16:
+        return GDN_F16
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+def current_stream_handle() -> int:
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(status, where, raise_on_error):
+    if raise_on_error and status != GDN_OK:
+        raise GdnError(status, where)
+    return status
+
+
+def gdn_prefill_workspace_size(dims: gdn_dims, T_tot: int, dtype: int) -> int:
+    return int(lib().gdn_prefill_workspace_size(ctypes.byref(dims), int(T_tot), int(dtype)))
+
+
+def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,
+                cu_seqlens, N, T_tot, chunk, dtype, out, workspace, workspace_bytes,
+                initial_state=None, final_state=None, conv_state_in=None, conv_state_out=None,
+                impl=GDN_IMPL_AUTO, core_event_begin=None, core_event_end=None, stream=None,
+                raise_on_error=True) -> int:
+    args = gdn_prefill_args(
+        ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
+        ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
+        ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
+        ptr(workspace), int(workspace_bytes), core_event_begin, core_event_end)
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_prefill(ctypes.byref(dims), ctypes.byref(args), s), "gdn_prefill",
+                  raise_on_error)
+
+
+def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w, state,
+               conv_state, out, B, dtype, stream=None, raise_on_error=True) -> int:
+    args = gdn_decode_args(ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log),
+                           ptr(dt_bias), ptr(z), ptr(norm_w), ptr(state), ptr(conv_state),
+                           ptr(out), int(B), int(dtype))
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_decode(ctypes.byref(dims), ctypes.byref(args), s), "gdn_decode",
+                  raise_on_error)
+
+
+def gdn_chunk_core(dims: gdn_dims, *, q, k, v, g, beta, cu_seqlens, N, T_tot, chunk, dtype, o,
+                   initial_state=None, final_state=None, impl=GDN_IMPL_AUTO, stream=None,
+                   raise_on_error=True) -> int:
+    args = gdn_core_args(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(cu_seqlens), int(N),
+                         int(T_tot), int(chunk), int(dtype), int(impl), ptr(initial_state),
+                         ptr(final_state), ptr(o))
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_chunk_core(ctypes.byref(dims), ctypes.byref(args), s),
+                  "gdn_chunk_core", raise_on_error)
+
+
+def gdn_version() -> str:
+    return lib().gdn_version().decode()

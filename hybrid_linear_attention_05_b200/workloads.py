@@ -25,7 +25,7 @@ the values the GPU consumes.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 from typing import Optional
 
 import numpy as np
@@ -48,6 +48,7 @@ class Workload:
     s0_std: float = 0.0       # 0 -> zero initial state
     varlen_total: int = 0     # >0: lengths drawn at random summing to this
     varlen_n: int = 0
+    q_scale: Optional[float] = None  # factor on the normalised q; None -> d ** -0.5
 
     @property
     def Cc(self) -> int:
@@ -55,7 +56,7 @@ class Workload:
 
     @property
     def scale(self) -> float:
-        return self.d ** -0.5
+        return self.d ** -0.5 if self.q_scale is None else float(self.q_scale)
 
 
 WORKLOADS = {

@@ -1,0 +1,210 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet token mixer.
+ *
+ * The mixer is the linear-attention layer that fills three of every four
+ * layers of the Qwen3.5 / Qwen3-Next hybrid stack ("Qwen3.5", HF transformers
+ * model doc, Usage tips: layer_types alternate three Gated DeltaNet layers
+ * with one full-attention layer).  For each token it computes
+ *
+ *   1. y = causal depthwise conv1d (kernel 4, no bias) of the mixed q|k|v
+ *      projection, then SiLU                 ("Qwen3.5 (Qwen3-Next)", API
+ *      table: linear_conv_kernel_dim 4; "Qwen/Qwen3.5-9B", module tree:
+ *      conv1d 8192x1x4, 32.8K parameters);
+ *   2. q, k = per-head L2-normalised slices of y (q also times `scale`),
+ *      v = the value slice;
+ *   3. per value head: g = -exp(A_log) * softplus(a + dt_bias),
+ *      alpha = exp(g), beta = sigmoid(b)     ("Qwen/Qwen3.5-9B", module tree:
+ *      in_proj_a / in_proj_b 4096->32 and the direct parameters "32, 32");
+ *   4. the gated delta rule, value head h reading key head h / (Hv/Hk):
+ *         S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *         o_t = S_t q_t,     S in R^{dv x dk}
+ *      ("Qwen (text & vision-language)", Architecture notes and Generation:
+ *      conv1d + delta rule, with a conv state and a recurrent state carried
+ *      per layer);
+ *   5. out = o / sqrt(mean(o^2) + eps_norm) * norm_w * silu(z), one dv-wide
+ *      norm_w shared by all heads    ("Qwen/Qwen3.5-9B", module tree: norm
+ *      Qwen3_5RMSNormGated with 128 parameters).
+ *
+ * gdn_prefill runs steps 1-5 over variable-length packed sequences with the
+ * chunked (WY / UT transform) form of step 4, which is algebraically equal to
+ * the recurrence ("Qwen (text & vision-language)", Verified parity).
+ * gdn_decode runs one token per sequence with the recurrent form on an fp32
+ * state held in HBM and updated in place ("Qwen3.5", HF model doc, Usage
+ * tips: the single-token recurrence is memory-bandwidth-bound).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named "device" must point to device memory of the current
+ *     CUDA device; the caller owns all memory.  The library allocates nothing
+ *     and keeps no state between calls; calls on different streams are
+ *     independent.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream).  A call returns after launching.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns a negative gdn_status and launches nothing.
+ *     Contents of device arrays (e.g. cu_seqlens) cannot be checked on the
+ *     host; out-of-range offsets are clamped by the kernels so that no access
+ *     leaves the buffers, but the results are then unspecified.
+ *   - Layouts are row-major (C order).  "dtype" below is gdn_dtype `dtype`
+ *     of the call: bf16 (GDN_BF16) or fp32 (GDN_F32).  States are always fp32.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Channel order of the mixed projection: [q heads | k heads | v heads],
+ *     head-major within each block (q head i occupies channels i*dk ..
+ *     i*dk+dk-1).  Value head h reads key head h / (Hv/Hk).
+ *   - Conv taps: conv_w[c][3] multiplies the current token, conv_w[c][0] the
+ *     token three steps back.  A conv history [.., Cc, 3] holds the last
+ *     three raw (pre-conv) inputs per channel, oldest first.
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_NULL = -1,        /* a required pointer is NULL                       */
+  GDN_ERR_DIMS = -2,        /* inconsistent or out-of-range sizes               */
+  GDN_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned                 */
+  GDN_ERR_UNSUPPORTED = -4, /* valid, but not a shape this build supports       */
+  GDN_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed (launch, ...)  */
+  GDN_ERR_WORKSPACE = -6,   /* workspace missing or smaller than required       */
+  GDN_ERR_ALIAS = -7        /* buffers that must not overlap do overlap         */
+} gdn_status;
+
+/* Element types.  gdn_prefill / gdn_decode take GDN_F32 or GDN_BF16 inputs;
+ * GDN_F16 is accepted only for the q, k, v of gdn_chunk_core (it is the type
+ * gdn_prefill itself uses between its kernels for bf16 inputs). */
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype;
+
+/* Implementation selector for the chunked core of gdn_prefill. */
+typedef enum {
+  GDN_IMPL_AUTO = 0,   /* tensor cores when supported, else CUDA cores        */
+  GDN_IMPL_SIMT = 1,   /* fp32 CUDA-core chunked kernel                       */
+  GDN_IMPL_TC = 2      /* tcgen05 tensor-core chunked kernel (bf16 inputs,
+                          fp16 operands, d = 128, chunk 64);
+                          GDN_ERR_UNSUPPORTED otherwise                       */
+} gdn_impl;
+
+/* Layer shape.  Supported: dk == dv in {32, 64, 128}; Hv % Hk == 0;
+ * conv_k == 4.  scale multiplies q after its L2 norm (dk^-1/2 is usual);
+ * eps_l2 is added to sum(x^2) inside the q/k L2 norm; eps_norm to mean(o^2)
+ * inside the gated RMSNorm (1e-6 for the Qwen3.5 family). */
+typedef struct {
+  int Hk, Hv, dk, dv;
+  int conv_k;
+  float scale;
+  float eps_l2;
+  float eps_norm;
+} gdn_dims;
+
+/* ------------------------------------------------------------------ prefill
+ * Packed varlen prefill: N sequences, sequence n occupying tokens
+ * cu_seqlens[n] .. cu_seqlens[n+1]-1 of the packed token axis (T_tot tokens).
+ * Cc = 2*Hk*dk + Hv*dv.
+ */
+typedef struct {
+  const void* mixed_qkv;       /* device [T_tot, Cc]      dtype                     */
+  const void* conv_w;          /* device [Cc, 4]          dtype                     */
+  const void* a;               /* device [T_tot, Hv]      dtype                     */
+  const void* b;               /* device [T_tot, Hv]      dtype                     */
+  const float* A_log;          /* device [Hv]             fp32                      */
+  const float* dt_bias;        /* device [Hv]             fp32                      */
+  const void* z;               /* device [T_tot, Hv*dv]   dtype                     */
+  const void* norm_w;          /* device [dv]             dtype                     */
+  const int32_t* cu_seqlens;   /* device [N+1] int32, cu[0]=0, non-decreasing,
+                                  cu[N]=T_tot; empty sequences are allowed        */
+  int N;                       /* number of sequences (>= 1)                      */
+  int T_tot;                   /* packed tokens (>= 0)                            */
+  int chunk;                   /* chunk length: 16, 32 or 64                      */
+  gdn_dtype dtype;
+  gdn_impl impl;
+  const float* initial_state;  /* device [N, Hv, dv, dk] fp32, or NULL for zeros  */
+  float* final_state;          /* device [N, Hv, dv, dk] fp32, or NULL; may be the
+                                  same pointer as initial_state (updated in place) */
+  const void* conv_state_in;   /* device [N, Cc, 3] dtype, or NULL for zeros      */
+  void* conv_state_out;        /* device [N, Cc, 3] dtype, or NULL; must not
+                                  overlap conv_state_in                           */
+  void* out;                   /* device [T_tot, Hv, dv] dtype                    */
+  void* workspace;             /* device scratch, >= gdn_prefill_workspace_size  */
+  size_t workspace_bytes;
+  void* core_event_begin;      /* optional cudaEvent_t recorded on `stream` just
+                                  before / after the chunked-core kernel (timing
+                                  of that kernel alone); NULL to skip           */
+  void* core_event_end;
+} gdn_prefill_args;
+
+/* Bytes of device workspace gdn_prefill needs for these sizes (0 when the
+ * sizes are invalid).  The workspace holds the normalised q, k, the values v
+ * (fp16 for bf16 inputs, fp32 for fp32 inputs) and the gates of every token
+ * between the two kernels of the call. */
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dtype);
+
+/* Steps 1-5 over packed sequences.  Writes out, and final_state /
+ * conv_state_out when given.  The workspace is overwritten. */
+gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* args, void* stream);
+
+/* ------------------------------------------------------------------- decode
+ * One token for each of B independent sequences.  state and conv_state are
+ * read and overwritten in place with the values after this token.
+ */
+typedef struct {
+  const void* mixed_qkv;       /* device [B, Cc]          dtype                     */
+  const void* conv_w;          /* device [Cc, 4]          dtype                     */
+  const void* a;               /* device [B, Hv]          dtype                     */
+  const void* b;               /* device [B, Hv]          dtype                     */
+  const float* A_log;          /* device [Hv]             fp32                      */
+  const float* dt_bias;        /* device [Hv]             fp32                      */
+  const void* z;               /* device [B, Hv*dv]       dtype                     */
+  const void* norm_w;          /* device [dv]             dtype                     */
+  float* state;                /* device [B, Hv, dv, dk]  fp32, in place            */
+  void* conv_state;            /* device [B, Cc, 3]       dtype, in place           */
+  void* out;                   /* device [B, Hv, dv]      dtype                     */
+  int B;                       /* batch (>= 0)                                      */
+  gdn_dtype dtype;
+} gdn_decode_args;
+
+gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* args, void* stream);
+
+/* --------------------------------------------------------------- core only
+ * Step 4 alone, chunked form, on given q, k (already normalised/scaled), v,
+ * log-decay g and beta.  It exists so that the exact invariants of the delta
+ * rule can be checked on the GPU without the conv, L2 norm and gated norm.
+ *   q, k  device [T_tot, Hk, dk] dtype;  v device [T_tot, Hv, dv] dtype
+ *         (dtype GDN_F32, GDN_BF16 or GDN_F16; the tensor-core kernel takes
+ *         GDN_F16)
+ *   g, beta device [Hv, T_tot] fp32 (head-major)
+ *   o     device [T_tot, Hv, dv] fp32 (the core output before the gated norm)
+ *   initial_state / final_state as in gdn_prefill_args.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  const int32_t* cu_seqlens;
+  int N, T_tot, chunk;
+  gdn_dtype dtype;
+  gdn_impl impl;
+  const float* initial_state;
+  float* final_state;
+  float* o;
+} gdn_core_args;
+
+gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* args, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* gdn_status_string(gdn_status status);
+
+/* Library version string, e.g. "gdn-b200 0.1". */
+const char* gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H */

@@ -1,0 +1,142 @@
+"""CPU-side checks of the C ABI: the library builds for sm_100a, loads
+without a GPU, exports every function gdn.h declares, sizes its workspace
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_linear_attention_05_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(gdn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "gdn_prefill" in names and "gdn_decode" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(gdn.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings(L):
+    assert gdn.gdn_version().startswith("gdn-b200")
+    for code in range(-7, 1):
+        assert gdn.status_string(code) not in ("", "unknown status")
+    assert gdn.status_string(-99) == "unknown status"
+
+
+def test_workspace_size():
+    dims = gdn.make_dims(16, 32, 128)
+    T = 1000
+    n = gdn.gdn_prefill_workspace_size(dims, T, gdn.GDN_BF16)
+    raw = T * (2 * 16 * 128 * 2 + 32 * 128 * 2 + 2 * 32 * 4)
+    assert raw <= n <= raw + 5 * 256
+    assert gdn.gdn_prefill_workspace_size(dims, T, gdn.GDN_F32) > n
+    assert gdn.gdn_prefill_workspace_size(gdn.make_dims(3, 4, 128), T, gdn.GDN_BF16) == 0
+    assert gdn.gdn_prefill_workspace_size(dims, -1, gdn.GDN_BF16) == 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned, never dereferenced "device" address
+
+
+def prefill_kwargs(**over):
+    kw = dict(mixed_qkv=FAKE, conv_w=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, z=FAKE,
+              norm_w=FAKE, cu_seqlens=FAKE, N=1, T_tot=16, chunk=32, dtype=gdn.GDN_BF16,
+              out=FAKE, workspace=FAKE, workspace_bytes=1 << 30, impl=gdn.GDN_IMPL_SIMT,
+              stream=0, raise_on_error=False)
+    kw.update(over)
+    return kw
+
+
+@pytest.mark.parametrize("dims,status", [
+    (gdn.make_dims(3, 4, 128), gdn.GDN_ERR_DIMS),        # Hv % Hk != 0
+    (gdn.make_dims(0, 4, 128), gdn.GDN_ERR_DIMS),
+    (gdn.make_dims(2, 4, 128, dv=64), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 96), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128, conv_k=3), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128, eps_norm=-1.0), gdn.GDN_ERR_DIMS),
+])
+def test_prefill_rejects_bad_dims(L, dims, status):
+    assert gdn.gdn_prefill(dims, **prefill_kwargs()) == status
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(mixed_qkv=None), gdn.GDN_ERR_NULL),
+    (dict(cu_seqlens=None), gdn.GDN_ERR_NULL),
+    (dict(workspace=None), gdn.GDN_ERR_NULL),
+    (dict(out=None), gdn.GDN_ERR_NULL),
+    (dict(z=FAKE + 8), gdn.GDN_ERR_ALIGN),
+    (dict(final_state=FAKE + 4), gdn.GDN_ERR_ALIGN),
+    (dict(workspace_bytes=1000), gdn.GDN_ERR_WORKSPACE),
+    (dict(chunk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(N=-1), gdn.GDN_ERR_DIMS),
+    (dict(T_tot=-5), gdn.GDN_ERR_DIMS),
+    (dict(N=0, T_tot=3), gdn.GDN_ERR_DIMS),
+    (dict(dtype=7), gdn.GDN_ERR_DIMS),
+    (dict(chunk=64, impl=gdn.GDN_IMPL_SIMT), gdn.GDN_ERR_UNSUPPORTED),  # d=128 needs chunk <= 32 on CUDA cores
+    (dict(conv_state_in=FAKE, conv_state_out=FAKE + 1024), gdn.GDN_ERR_ALIAS),
+    (dict(initial_state=FAKE, final_state=FAKE + 4096), gdn.GDN_ERR_ALIAS),
+    (dict(chunk=16, impl=gdn.GDN_IMPL_TC), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_prefill_rejects_bad_args(L, over, status):
+    dims = gdn.make_dims(2, 4, 128)
+    assert gdn.gdn_prefill(dims, **prefill_kwargs(**over)) == status
+
+
+def test_prefill_empty_batch_is_noop(L):
+    dims = gdn.make_dims(2, 4, 128)
+    assert gdn.gdn_prefill(dims, **prefill_kwargs(N=0, T_tot=0)) == gdn.GDN_OK
+
+
+def test_null_struct_pointers(L):
+    assert L.gdn_prefill(None, None, None) == gdn.GDN_ERR_NULL
+    dims = gdn.make_dims(2, 4, 128)
+    assert L.gdn_prefill(ctypes.byref(dims), None, None) == gdn.GDN_ERR_NULL
+    assert L.gdn_decode(ctypes.byref(dims), None, None) == gdn.GDN_ERR_NULL
+    assert L.gdn_chunk_core(ctypes.byref(dims), None, None) == gdn.GDN_ERR_NULL
+
+
+def decode_kwargs(**over):
+    kw = dict(mixed_qkv=FAKE, conv_w=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, z=FAKE,
+              norm_w=FAKE, state=FAKE, conv_state=FAKE, out=FAKE, B=4, dtype=gdn.GDN_BF16,
+              stream=0, raise_on_error=False)
+    kw.update(over)
+    return kw
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(state=None), gdn.GDN_ERR_NULL),
+    (dict(conv_state=None), gdn.GDN_ERR_NULL),
+    (dict(out=FAKE + 2), gdn.GDN_ERR_ALIGN),
+    (dict(B=-1), gdn.GDN_ERR_DIMS),
+    (dict(B=0), gdn.GDN_OK),
+])
+def test_decode_rejects_bad_args(L, over, status):
+    assert gdn.gdn_decode(gdn.make_dims(2, 4, 128), **decode_kwargs(**over)) == status
+
+
+def test_core_rejects_bad_args(L):
+    dims = gdn.make_dims(1, 1, 32)
+    kw = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu_seqlens=FAKE, N=1, T_tot=8, chunk=16,
+              dtype=gdn.GDN_F32, o=FAKE, stream=0, raise_on_error=False)
+    assert gdn.gdn_chunk_core(dims, **{**kw, "o": None}) == gdn.GDN_ERR_NULL
+    assert gdn.gdn_chunk_core(dims, **{**kw, "beta": FAKE + 4}) == gdn.GDN_ERR_ALIGN
+    assert gdn.gdn_chunk_core(dims, **{**kw, "chunk": 8}) == gdn.GDN_ERR_UNSUPPORTED

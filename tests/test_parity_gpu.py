@@ -1,0 +1,353 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle
+on the same seeded inputs.
+
+Bars (max|gpu - ref| / max|ref|): 5e-3 for prefill (bf16 tensor-core
+operands; the fp32 CUDA-core kernel is held to the same bar and reports its
+much smaller error), 1e-4 for the fp32 decode step (state exactly; bf16
+outputs after allowing their own rounding).
+"""
+import numpy as np
+import pytest
+
+from gdn_testlib import (DECODE_TOL, PREFILL_TOL, oracle_prefill, oracle_subproblem, relerr,
+                         relerr_beyond_bf16)
+import oracle
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from hybrid_linear_attention_05_b200 import api, build, gdn  # noqa: E402
+from hybrid_linear_attention_05_b200.workloads import (WORKLOADS, make_decode, make_prefill,  # noqa: E402
+                                                       resized)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    gdn.lib()
+
+
+TINY = WORKLOADS["prefill_T64_Hk2_Hv2_d32_c16_f32"]
+P08 = WORKLOADS["prefill_T4096_Hk16_Hv16_d128"]
+P9B = WORKLOADS["prefill_4x8192_Hk16_Hv32_d128"]
+D9B = WORKLOADS["decode_B256_Hk16_Hv32_d128"]
+P397 = WORKLOADS["prefill_varlen8_T65536_Hk16_Hv64_d128"]
+
+IMPLS = {"simt": (gdn.GDN_IMPL_SIMT, 32), "tc": (gdn.GDN_IMPL_TC, 64)}
+
+
+def np64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_prefill(inp, impl, chunk, guard=True):
+    dp = api.to_device(inp, chunk=chunk)
+    bufs = api.PrefillBuffers(dp)
+    if guard:  # canaries on both sides of every output
+        for name in ("out", "final_state", "conv_state_out"):
+            t = getattr(bufs, name)
+            big = torch.full((t.numel() + 2 * 64,), float("nan"), dtype=t.dtype, device=t.device)
+            setattr(bufs, name, big[64:64 + t.numel()].view(t.shape))
+            setattr(bufs, name + "_guard", big)
+    status = gdn.gdn_prefill(
+        bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b, A_log=dp.A_log,
+        dt_bias=dp.dt_bias, z=dp.z, norm_w=dp.norm_w, cu_seqlens=dp.cu_seqlens, N=dp.N,
+        T_tot=dp.T, chunk=dp.chunk, dtype=bufs.dtype_code, out=bufs.out, workspace=bufs.workspace,
+        workspace_bytes=bufs.ws_bytes, initial_state=dp.initial_state,
+        final_state=bufs.final_state, conv_state_in=dp.conv_state_in,
+        conv_state_out=bufs.conv_state_out, impl=impl, raise_on_error=False)
+    if status == gdn.GDN_ERR_UNSUPPORTED:
+        pytest.skip("implementation not available for this shape")
+    assert status == gdn.GDN_OK, gdn.status_string(status)
+    torch.cuda.synchronize()
+    if guard:
+        for name in ("out", "final_state", "conv_state_out"):
+            big = getattr(bufs, name + "_guard")
+            n = getattr(bufs, name).numel()
+            assert torch.isnan(big[:64].float()).all() and torch.isnan(big[64 + n:].float()).all(), \
+                "write outside " + name
+    return bufs
+
+
+def check_full(inp, bufs, tol=PREFILL_TOL):
+    ref = oracle_prefill(inp)
+    e_out = relerr(np64(bufs.out), ref.out)
+    e_S = relerr(np64(bufs.final_state), ref.final_state)
+    assert e_out <= tol, e_out
+    assert e_S <= tol, e_S
+    # the conv tail is a copy of raw inputs: exact
+    np.testing.assert_array_equal(np64(bufs.conv_state_out), ref.conv_state_out)
+    return e_out, e_S
+
+
+# ------------------------------------------------------------------ prefill
+
+
+def test_tiny_fp32_workload():
+    """The tiny fp32 workload (T=64, 2/2 heads of width 32, chunk 16) in full."""
+    inp = make_prefill(TINY)
+    bufs = run_prefill(inp, gdn.GDN_IMPL_AUTO, 16)
+    e_out, e_S = check_full(inp, bufs)
+    assert e_out < 1e-4 and e_S < 1e-4  # fp32 CUDA-core path: far inside the bar
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("d", [32, 64])
+def test_simt_small_heads(chunk, d):
+    w = resized(TINY, Hk=2, Hv=4, d=d, dtype="bf16", s0_std=0.02, seed=21)
+    inp = make_prefill(w, seqlens=(chunk * 3 + 7, 1, 2, chunk - 1, 0, chunk), with_conv_state=True)
+    bufs = run_prefill(inp, gdn.GDN_IMPL_SIMT, chunk)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("impl", ["simt", "tc"])
+def test_qwen08b_shapes_ragged(impl):
+    """16/16 heads of width 128 over several chunks with a ragged tail."""
+    code, chunk = IMPLS[impl]
+    inp = make_prefill(P08, seqlens=(333,))
+    bufs = run_prefill(inp, code, chunk)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("impl", ["simt", "tc"])
+def test_9b_shapes_gqa_varlen(impl):
+    """16 key / 32 value heads, nonzero initial states, conv history,
+    sequences of lengths 1, 2, 3, 64 and one spanning several chunks."""
+    code, chunk = IMPLS[impl]
+    inp = make_prefill(P9B, seqlens=(200, 1, 2, 3, 64, 0, 129), with_conv_state=True)
+    bufs = run_prefill(inp, code, chunk)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("impl", ["simt", "tc"])
+def test_397b_shapes_varlen(impl):
+    code, chunk = IMPLS[impl]
+    inp = make_prefill(P397, seqlens=(65, 130, 7, 64))
+    bufs = run_prefill(inp, code, chunk)
+    check_full(inp, bufs)
+
+
+def test_in_place_state_update():
+    """final_state may be the initial_state buffer itself."""
+    w = resized(P9B, Hk=2, Hv=4, seed=31)
+    inp = make_prefill(w, seqlens=(70, 5))
+    dp = api.to_device(inp, chunk=32)
+    bufs = api.PrefillBuffers(dp)
+    S = dp.initial_state.clone()
+    gdn.gdn_prefill(bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b,
+                    A_log=dp.A_log, dt_bias=dp.dt_bias, z=dp.z, norm_w=dp.norm_w,
+                    cu_seqlens=dp.cu_seqlens, N=dp.N, T_tot=dp.T, chunk=32,
+                    dtype=bufs.dtype_code, out=bufs.out, workspace=bufs.workspace,
+                    workspace_bytes=bufs.ws_bytes, initial_state=S, final_state=S,
+                    impl=gdn.GDN_IMPL_AUTO)
+    torch.cuda.synchronize()
+    ref = oracle_prefill(inp)
+    assert relerr(np64(S), ref.final_state) <= PREFILL_TOL
+    assert relerr(np64(bufs.out), ref.out) <= PREFILL_TOL
+
+
+# ------------------------------------------------------- full-size workloads
+
+
+def sampled_check(inp, bufs, pairs):
+    worst = 0.0
+    for n, h in pairs:
+        ref, s, cols = oracle_subproblem(inp, n, h)
+        e1 = relerr(np64(bufs.out[s, h]), ref.out[:, 0])
+        e2 = relerr(np64(bufs.final_state[n, h]), ref.final_state[0, 0])
+        np.testing.assert_array_equal(np64(bufs.conv_state_out[n][cols]), ref.conv_state_out[0])
+        assert e1 <= PREFILL_TOL and e2 <= PREFILL_TOL, (n, h, e1, e2)
+        worst = max(worst, e1, e2)
+    return worst
+
+
+@pytest.mark.parametrize("name,pairs", [
+    ("prefill_T4096_Hk16_Hv16_d128", [(0, 0), (0, 7), (0, 15)]),
+    ("prefill_4x8192_Hk16_Hv32_d128", [(0, 0), (1, 13), (3, 31)]),
+    ("prefill_varlen8_T65536_Hk16_Hv64_d128", [(0, 0), (3, 21), (7, 63)]),
+])
+def test_full_size_sampled(name, pairs):
+    """Full benchmark sizes in the benchmark's launch configuration; the
+    oracle recomputes a few (sequence, value head) pairs on their own."""
+    w = WORKLOADS[name]
+    inp = make_prefill(w)
+    bufs = run_prefill(inp, gdn.GDN_IMPL_AUTO, w.chunk, guard=False)
+    sampled_check(inp, bufs, pairs)
+    assert torch.isfinite(bufs.out.float()).all()
+
+
+# ------------------------------------------------------------------- decode
+
+
+def run_decode(inp):
+    dd = api.decode_to_device(inp)
+    out = api.decode(dd)
+    torch.cuda.synchronize()
+    return dd, out
+
+
+def oracle_decode(inp):
+    w = inp.w
+    return oracle.decode(w.Hk, w.Hv, w.d, w.d, inp.mixed_qkv, inp.conv_w, inp.a, inp.b, inp.A_log,
+                         inp.dt_bias, inp.z, inp.norm_w, inp.state, inp.conv_state, scale=w.scale)
+
+
+def test_decode_full_batch():
+    """The full decode workload: batch 256, 16/32 heads, 512 MiB fp32 state."""
+    inp = make_decode(D9B)
+    dd, out = run_decode(inp)
+    ref_out, ref_S, ref_cs = oracle_decode(inp)
+    assert relerr(np64(dd.state), ref_S) <= DECODE_TOL
+    assert relerr_beyond_bf16(np64(out), ref_out) <= DECODE_TOL
+    np.testing.assert_array_equal(np64(dd.conv_state), ref_cs)
+
+
+@pytest.mark.parametrize("d,Hk,Hv", [(32, 2, 2), (64, 2, 8), (128, 4, 16)])
+def test_decode_fp32(d, Hk, Hv):
+    w = resized(D9B, Hk=Hk, Hv=Hv, d=d, dtype="f32", seed=40 + d)
+    inp = make_decode(w, batch=5)
+    dd, out = run_decode(inp)
+    ref_out, ref_S, ref_cs = oracle_decode(inp)
+    assert relerr(np64(dd.state), ref_S) <= DECODE_TOL
+    assert relerr(np64(out), ref_out) <= DECODE_TOL
+    np.testing.assert_array_equal(np64(dd.conv_state), ref_cs)
+
+
+def test_prefill_then_decode_composition():
+    """prefill of T tokens followed by a decode of token T+1 equals the
+    oracle's prefill of T+1 tokens (state and last output)."""
+    w = resized(P9B, Hk=2, Hv=4, seed=50)
+    T = 70
+    inp = make_prefill(w, seqlens=(T + 1, T + 1), with_conv_state=True)
+    cu = inp.cu_seqlens
+    first = np.concatenate([np.arange(cu[n], cu[n] + T) for n in range(2)])
+    last = cu[1:] - 1
+    import dataclasses
+    pre = dataclasses.replace(inp, cu_seqlens=np.array([0, T, 2 * T], np.int32),
+                              mixed_qkv=inp.mixed_qkv[first], a=inp.a[first], b=inp.b[first],
+                              z=inp.z[first])
+    bufs = run_prefill(pre, gdn.GDN_IMPL_AUTO, 32, guard=False)
+    dd = api.DeviceDecode(
+        Hk=w.Hk, Hv=w.Hv, d=w.d, scale=w.scale, B=2,
+        mixed_qkv=torch.from_numpy(inp.mixed_qkv[last]).cuda().bfloat16(),
+        conv_w=torch.from_numpy(inp.conv_w).cuda().bfloat16(),
+        a=torch.from_numpy(inp.a[last]).cuda().bfloat16(), b=torch.from_numpy(inp.b[last]).cuda().bfloat16(),
+        A_log=torch.from_numpy(inp.A_log).cuda(), dt_bias=torch.from_numpy(inp.dt_bias).cuda(),
+        z=torch.from_numpy(inp.z[last]).cuda().bfloat16(),
+        norm_w=torch.from_numpy(inp.norm_w).cuda().bfloat16(),
+        state=bufs.final_state.clone(), conv_state=bufs.conv_state_out.clone())
+    out = api.decode(dd)
+    torch.cuda.synchronize()
+    ref = oracle_prefill(inp)
+    assert relerr(np64(dd.state), ref.final_state) <= PREFILL_TOL
+    assert relerr(np64(out), ref.out[last]) <= PREFILL_TOL
+    np.testing.assert_array_equal(np64(dd.conv_state), ref.conv_state_out)
+
+
+# ------------------------------------------------------------- core only
+
+
+def rounded(x, dtype):
+    """x as float64 holding exactly the values of its `dtype` copy."""
+    if dtype == torch.float32:
+        return x.astype(np.float32).astype(np.float64)
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dtype).double().numpy()
+
+
+def run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, impl, S0=None, dtype=torch.float32):
+    dev = "cuda"
+    T = q.shape[0]
+    N = len(cu) - 1
+    t = lambda x, dt=dtype: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev, dt)
+    o = torch.empty((T, Hv, d), dtype=torch.float32, device=dev)
+    S = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    status = gdn.gdn_chunk_core(
+        gdn.make_dims(Hk, Hv, d, scale=1.0), q=t(q), k=t(k), v=t(v),
+        g=t(np.ascontiguousarray(g.T), torch.float32), beta=t(np.ascontiguousarray(beta.T), torch.float32),
+        cu_seqlens=torch.tensor(cu, dtype=torch.int32, device=dev), N=N, T_tot=T, chunk=chunk,
+        dtype=gdn.dtype_code(t(q)), o=o, initial_state=None if S0 is None else t(S0, torch.float32),
+        final_state=S, impl=impl, raise_on_error=False)
+    if status == gdn.GDN_ERR_UNSUPPORTED:
+        pytest.skip("implementation not available for this shape")
+    assert status == gdn.GDN_OK
+    torch.cuda.synchronize()
+    return np64(o), np64(S)
+
+
+@pytest.mark.parametrize("impl,d,chunk,dtype", [
+    ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.float32),
+    ("tc", 128, 64, torch.float16)])
+def test_core_orthonormal_overwrite(impl, d, chunk, dtype):
+    """alpha = 1, beta = 1, orthonormal keys: S k_i = v_i after writing, and
+    a rewritten key returns its new value (exact in real arithmetic)."""
+    code = IMPLS[impl][0]
+    rng = np.random.default_rng(60)
+    m = min(d, 40)
+    Qm, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    keys = Qm[:, :m].T
+    if dtype != torch.float32:  # keys exactly representable: use signed unit vectors
+        keys = np.eye(d)[rng.permutation(d)[:m]] * rng.choice([-1.0, 1.0], size=(m, 1))
+    vals = rng.standard_normal((m, d))
+    order = np.concatenate([np.arange(m), [0, 1]])
+    newv = rng.standard_normal((2, d))
+    kseq = keys[order]
+    vseq = np.concatenate([vals, newv])
+    vseq = rounded(vseq, dtype)
+    T = len(order)
+    k = kseq[:, None, :]
+    o, S = run_core(k, k, vseq[:, None, :], np.zeros((T, 1)), np.ones((T, 1)), [0, T], 1, 1, d,
+                    chunk, code, dtype=dtype)
+    tol = 1e-4 if dtype == torch.float32 else PREFILL_TOL
+    exp_vals = vseq[:m].copy()
+    exp_vals[0], exp_vals[1] = vseq[m], vseq[m + 1]
+    got = S[0, 0] @ keys.T  # column i = S k_i
+    assert relerr(got.T, exp_vals) <= tol
+    assert relerr(o[:m, 0], vseq[:m]) <= tol  # read-back right after each write
+
+
+@pytest.mark.parametrize("impl,d,chunk,dtype", [
+    ("simt", 64, 32, torch.float32), ("tc", 128, 64, torch.float16)])
+def test_core_beta_zero_only_decays(impl, d, chunk, dtype):
+    code = IMPLS[impl][0]
+    rng = np.random.default_rng(61)
+    T, Hv = 150, 2
+    q = rng.standard_normal((T, 1, d)); q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k = rng.standard_normal((T, 1, d)); k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, Hv, d))
+    g = -rng.uniform(0, 0.05, (T, Hv))
+    S0 = rng.standard_normal((1, Hv, d, d)) * 0.1
+    q, k, v = [rounded(x, dtype) for x in (q, k, v)]
+    o, S = run_core(q, k, v, g, np.zeros((T, Hv)), [0, T], 1, Hv, d, chunk, code, S0=S0, dtype=dtype)
+    cum = np.exp(np.cumsum(g, axis=0))
+    tol = 1e-4 if dtype == torch.float32 else PREFILL_TOL
+    for h in range(Hv):
+        assert relerr(S[0, h], cum[-1, h] * S0[0, h]) <= tol
+        assert relerr(o[:, h], cum[:, h:h + 1] * (q[:, 0] @ S0[0, h].T)) <= tol
+
+
+@pytest.mark.parametrize("impl,d,chunk,dtype", [
+    ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.bfloat16),
+    ("simt", 64, 64, torch.float16), ("tc", 128, 64, torch.float16)])
+def test_core_matches_oracle(impl, d, chunk, dtype):
+    code = IMPLS[impl][0]
+    rng = np.random.default_rng(62)
+    Hk, Hv = 2, 4
+    lens = [3 * chunk + 11, 1, chunk]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T = int(cu[-1])
+    q = rng.standard_normal((T, Hk, d)); q /= np.linalg.norm(q, axis=-1, keepdims=True) * np.sqrt(d)
+    k = rng.standard_normal((T, Hk, d)); k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, Hv, d))
+    g = -np.exp(rng.uniform(0, np.log(16), Hv))[None] * np.log1p(np.exp(rng.standard_normal((T, Hv))))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((T, Hv))))
+    S0 = rng.standard_normal((3, Hv, d, d)) * 0.02
+    q, k, v = [rounded(x, dtype) for x in (q, k, v)]
+    g = g.astype(np.float32).astype(np.float64)
+    beta = beta.astype(np.float32).astype(np.float64)
+    o, S = run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, code, S0=S0, dtype=dtype)
+    o_ref, S_ref = oracle.core(Hk, Hv, d, d, cu, q, k, v, g, beta, S0.astype(np.float32))
+    tol = 1e-4 if dtype == torch.float32 else PREFILL_TOL
+    assert relerr(o, o_ref) <= tol
+    assert relerr(S, S_ref) <= tol
