@@ -57,7 +57,6 @@ constexpr uint32_t OFF_MISC = OFF_RS + 3 * 256 * 4;  // gamma, e^gamma, beta, sc
 constexpr uint32_t OFF_BAR = OFF_MISC + 3 * 64 * 4 + 64;
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
-static_assert(OFF_TF + 64 * 65 * 4 >= OFF_AF + 64 * 128 * 4 - 64 * 65 * 4, "epilogue staging");
 static_assert(OFF_AF + 64 * 128 * 4 <= OFF_MISC, "epilogue staging overlaps misc");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 

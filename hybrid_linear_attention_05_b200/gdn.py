@@ -33,7 +33,7 @@ GDN_IMPL_SIMT = 1
 GDN_IMPL_TC = 2
 
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_chunk_core",
-            "gdn_status_string", "gdn_version"]
+            "gdn_device_error", "gdn_status_string", "gdn_version"]
 
 
 class gdn_dims(ctypes.Structure):
@@ -89,6 +89,8 @@ def lib():
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_chunk_core.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_core_args), _vp]
         L.gdn_chunk_core.restype = ctypes.c_int
+        L.gdn_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+        L.gdn_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_version.argtypes = []
@@ -182,6 +184,13 @@ def gdn_chunk_core(dims: gdn_dims, *, q, k, v, g, beta, cu_seqlens, N, T_tot, ch
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_chunk_core(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_chunk_core", raise_on_error)
+
+
+def gdn_device_error(clear: bool = True) -> int:
+    """Synchronise the device and return (and clear) the kernels' error word."""
+    code = ctypes.c_int(0)
+    _check(lib().gdn_device_error(ctypes.byref(code), int(clear)), "gdn_device_error", True)
+    return code.value
 
 
 def gdn_version() -> str:

@@ -197,6 +197,13 @@ typedef struct {
 
 gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* args, void* stream);
 
+/* Error word of the tensor-core kernels.  Their internal waits (on TMA and
+ * tensor-core completion) are bounded; one that gives up records a nonzero
+ * code here and the kernel returns instead of hanging.  This call
+ * synchronises the current device, stores the code in *code (0 = none) and
+ * clears it when clear != 0. */
+gdn_status gdn_device_error(int* code, int clear);
+
 /* Human-readable name of a status code (static storage). */
 const char* gdn_status_string(gdn_status status);
 
