@@ -32,13 +32,31 @@ namespace gdn {
 
 __device__ int g_tc_error = 0;  // nonzero: a bounded wait in a kernel gave up
 
+#ifdef GDN_PHASE_TIMING
+// Development aid (off by default): SM cycles spent by CTA thread 0 in each
+// phase of the chunk loop, summed over all CTAs.
+__device__ unsigned long long g_phase_cycles[16];
+#define GDN_PHASE(k)                                             \
+  do {                                                           \
+    if (tid == 0) {                                              \
+      const long long t_ = clock64();                            \
+      atomicAdd(&g_phase_cycles[k], (unsigned long long)(t_ - t_prev)); \
+      t_prev = t_;                                               \
+    }                                                            \
+  } while (0)
+#else
+#define GDN_PHASE(k) \
+  do {               \
+  } while (0)
+#endif
+
 namespace {
 
 using namespace ptx;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 128;
+constexpr int NT = 256;  // two warpgroups; each TMEM lane (row) is split by columns between them
 
 // shared memory layout, byte offsets from a 1024-aligned base
 constexpr uint32_t OFF_KQ0 = 0;       // [K;Q] tile, stage 0: two dk halves x 128 rows x 128 B
@@ -50,21 +68,22 @@ constexpr uint32_t OFF_P = 131072;    // P (fp16), 64 rows x 128 B
 constexpr uint32_t OFF_TB = 139264;   // T diag(beta); with OFF_TBE later holds Vn^T (16 KiB)
 constexpr uint32_t OFF_TBE = 147456;  // T diag(beta e^gamma)
 constexpr uint32_t OFF_VTS = 155648;  // Vn^T diag(e^{gamma_L - gamma}), 128 rows x 128 B
-constexpr uint32_t OFF_AF = 172032;   // fp32 A [64][65]; the epilogue reuses AF..TF as O [64][128]
-constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4;
-constexpr uint32_t OFF_RS = OFF_TF + 64 * 65 * 4;
-constexpr uint32_t OFF_MISC = OFF_RS + 3 * 256 * 4;  // gamma, e^gamma, beta, scan scratch
-constexpr uint32_t OFF_BAR = OFF_MISC + 3 * 64 * 4 + 64;
+constexpr uint32_t OFF_Z = 172032;    // z tile (bf16, two dv halves x 64 tokens x 128 B); then the output tile
+constexpr uint32_t OFF_AF = 188416;   // fp32 A [64][65]; the epilogue reuses AF..TF as O [64][128]
+constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4;     // fp32 T [64][65]; before it, the decay table E
+constexpr uint32_t OFF_RS = OFF_TF + 64 * 65 * 4;     // fp32 scratch of the inverse, 1024 floats
+constexpr uint32_t OFF_MISC = OFF_RS + 1024 * 4;      // gamma, e^gamma, beta, rms, e^{gamma_L - gamma}, scan
+constexpr uint32_t OFF_BAR = OFF_MISC + 5 * 64 * 4 + 64;
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
-static_assert(OFF_AF + 64 * 128 * 4 <= OFF_MISC, "epilogue staging overlaps misc");
+static_assert(OFF_AF + 64 * 128 * 4 <= OFF_RS, "epilogue staging overlaps the scratch");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // TMEM columns (fp32 accumulators, 128 lanes each)
 constexpr uint32_t TM_D1 = 0, TM_D2 = 64, TM_D3 = 128, TM_D4 = 192, TM_S = 256, TM_D5 = 384;
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t TILE_BYTES = 64 * 128;           // one 64 x 64 fp16 TMA box
+constexpr uint32_t TILE_BYTES = 64 * 128;           // one 64 x 64 16-bit TMA box
 constexpr uint32_t STAGE_TX = 6 * TILE_BYTES;       // K, Q (2 halves each), V (2 halves)
 
 __device__ __forceinline__ void st_half8(uint8_t* base, uint32_t off, const float* f) {
@@ -75,25 +94,32 @@ __device__ __forceinline__ void st_half8(uint8_t* base, uint32_t off, const floa
   *reinterpret_cast<uint4*>(base + off) = u;
 }
 
-// T = (I + A)^-1 for the strictly lower triangular 64 x 64 A (row stride 65).
-// Diagonal 16 x 16 blocks by forward substitution (one column per thread),
-// then block rows r = 1..3:  T_rc = -T_rr * sum_{k=c}^{r-1} A_rk T_kc.
-__device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, float* Rs, int tid) {
+// Tf := (I + A)^-1 for the strictly lower triangular 64 x 64 A (fp32, row
+// stride 65), by recursive doubling of the block size:
+//   16 x 16 diagonal blocks by forward substitution (one column per thread);
+//   32 x 32: T_{r,r-1} = -T_rr A_{r,r-1} T_{r-1,r-1} for the 16-blocks (1,0), (3,2);
+//   64 x 64: T_{LL}   = -T_bb A_{LL} T_tt for the lower-left 32-block.
+// Every product step gives each thread independent accumulators.
+__device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, float* X, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid < 64) {
     const int b = tid >> 4, m = tid & 15;
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float acc = (i == m) ? 1.f : 0.f;
+      float a0 = (i == m) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < i; ++j) acc = fmaf(-Af[(16 * b + i) * 65 + 16 * b + j], x[j], acc);
-      x[i] = acc;
+      for (int j = 0; j < i; j += 2) {
+        a0 = fmaf(-Af[(16 * b + i) * 65 + 16 * b + j], x[j], a0);
+        if (j + 1 < i) a1 = fmaf(-Af[(16 * b + i) * 65 + 16 * b + j + 1], x[j + 1], a1);
+      }
+      x[i] = a0 + a1;
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * 65 + 16 * b + m] = x[i];
   } else {
-    // blocks above the diagonal are zero
-    for (int e = tid - 64; e < 6 * 256; e += 64) {
+    // 16-blocks above the diagonal are zero
+    for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
       const int blk = e >> 8, w = e & 255, i = w >> 4, m = w & 15;
       const int r = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
       const int c = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
@@ -101,54 +127,98 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
     }
   }
   __syncthreads();
-  for (int r = 1; r < 4; ++r) {
-    for (int e = tid; e < r * 256; e += NT) {
-      const int c = e >> 8, i = (e >> 4) & 15, m = e & 15;
-      float acc = 0.f;
-      for (int k = c; k < r; ++k) {
+  // 32 x 32 diagonal blocks: element e = tid + 256 k -> 16-block (r, r-1), r = 1 or 3
+  {
+    float acc[2] = {0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          acc = fmaf(Af[(16 * r + i) * 65 + 16 * k + j], Tf[(16 * k + j) * 65 + 16 * c + m], acc);
+    for (int j = 0; j < 16; ++j) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
+        acc[k] = fmaf(Af[(16 * r + i) * 65 + 16 * (r - 1) + j],
+                      Tf[(16 * (r - 1) + j) * 65 + 16 * (r - 1) + m], acc[k]);
       }
-      Rs[e] = acc;
     }
-    __syncthreads();
-    for (int e = tid; e < r * 256; e += NT) {
-      const int c = e >> 8, i = (e >> 4) & 15, m = e & 15;
-      float acc = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        acc = fmaf(Tf[(16 * r + i) * 65 + 16 * r + j], Rs[c * 256 + j * 16 + m], acc);
-      Tf[(16 * r + i) * 65 + 16 * c + m] = -acc;
-    }
-    __syncthreads();
+    for (int k = 0; k < 2; ++k) X[tid + NT * k] = acc[k];
   }
+  __syncthreads();
+  {
+    float acc[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = tid + NT * k, blk = e >> 8, r = blk ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
+        acc[k] = fmaf(Tf[(16 * r + i) * 65 + 16 * r + j], X[blk * 256 + j * 16 + m], acc[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
+      Tf[(16 * r + i) * 65 + 16 * (r - 1) + m] = -acc[k];
+    }
+  }
+  __syncthreads();
+  // 64 x 64: rows 32 + warp + 8k of the lower-left block, column `lane`
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+      const float t = Tf[j * 65 + lane];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = fmaf(Af[(32 + warp + 8 * k) * 65 + j], t, acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) X[(warp + 8 * k) * 32 + lane] = acc[k];
+  }
+  __syncthreads();
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+      const float x = X[j * 32 + lane];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = fmaf(Tf[(32 + warp + 8 * k) * 65 + 32 + j], x, acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) Tf[(32 + warp + 8 * k) * 65 + lane] = -acc[k];
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, ChunkParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
+                    ChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   float* Af = reinterpret_cast<float*>(smem + OFF_AF);
   float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
-  float* Rs = reinterpret_cast<float*>(smem + OFF_RS);
+  float* Ef = Tf;  // decay table e^{gamma_i - gamma_j}, [64][65], alive before the inverse
+  float* Xs = reinterpret_cast<float*>(smem + OFF_RS);
   float* Os = reinterpret_cast<float*>(smem + OFF_AF);
+  __nv_bfloat16* Zs = reinterpret_cast<__nv_bfloat16*>(smem + OFF_Z);
   float* gam = reinterpret_cast<float*>(smem + OFF_MISC);
   float* eg = gam + 64;
   float* bet = eg + 64;
-  float* scan = bet + 64;
-  const uint32_t bar_load0 = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 16;
+  float* rms = bet + 64;
+  float* decL = rms + 64;
+  float* scan = decL + 64;
+  const uint32_t bar_load0 = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 16, bar_z = sb + OFF_BAR + 24;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 32);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wg = tid >> 7;     // warpgroup: which column half of a TMEM row this thread handles
+  const int tl = tid & 127;    // TMEM lane (row) of this thread
   const int h = blockIdx.x, n = blockIdx.y;
   const int hk = h / (p.Hv / p.Hk);
   const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
   const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
   const int nchunks = (eos - bos + C - 1) / C;
   const size_t sbase = ((size_t)n * p.Hv + h) * D * D;
+  const bool norm_out = p.out != nullptr;
 
   if (nchunks == 0) {  // empty sequence: the state passes through
     if (p.S_out)
@@ -160,6 +230,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(bar_load0, 1);
     mbar_init(bar_load0 + 8, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_z, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -170,7 +241,7 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lanes
 
   auto issue_loads = [&](int cc, int s) {
     const int row = bos + cc * C;
@@ -187,18 +258,30 @@ __global__ void __launch_bounds__(NT, 1)
   };
   if (tid == 0) issue_loads(0, 0);
 
-  // initial state -> TMEM (row v = tid)
+  // gates are fetched one chunk ahead (threads 0..63, one token each)
+  float g_next = 0.f, b_next = 0.f;
+  auto load_gates = [&](int cc) {
+    const int t0 = bos + cc * C;
+    const int Lc = min(C, eos - t0);
+    g_next = tid < Lc ? __ldg(p.g + (size_t)h * p.T + t0 + tid) : 0.f;
+    b_next = tid < Lc ? __ldg(p.beta + (size_t)h * p.T + t0 + tid) : 0.f;
+  };
+  if (tid < 64) load_gates(0);
+  const float w_norm = norm_out ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tl]) : 0.f;
+
+  // initial state -> TMEM (row tl, columns wg*64 .. wg*64+63)
   {
     float r[32];
 #pragma unroll
-    for (int piece = 0; piece < 4; ++piece) {
+    for (int piece = 0; piece < 2; ++piece) {
+      const int col = wg * 64 + piece * 32;
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
-        float4 f = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)tid * D + piece * 32 + j)
+        float4 f = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)tl * D + col + j)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
         r[j] = f.x; r[j + 1] = f.y; r[j + 2] = f.z; r[j + 3] = f.w;
       }
-      tmem_st32(lane_base + TM_S + piece * 32, r);
+      tmem_st32(lane_base + TM_S + col, r);
     }
     tmem_wait_st();
   }
@@ -206,6 +289,9 @@ __global__ void __launch_bounds__(NT, 1)
   uint32_t mma_phase = 0;
   bool ok = true;
   int c = 0;
+#ifdef GDN_PHASE_TIMING
+  long long t_prev = clock64();
+#endif
   for (; c < nchunks; ++c) {
     const int s = c & 1;
     const int c0 = bos + c * C;
@@ -214,15 +300,19 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t vv = sb + (s ? OFF_V1 : OFF_V0);
     uint8_t* wt_ptr = smem + (s ? OFF_V1 : OFF_V0);  // -W^T reuses the consumed V tile
 
-    if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1, s ^ 1);
+    if (tid == 0) {
+      if (c + 1 < nchunks) issue_loads(c + 1, s ^ 1);
+      if (norm_out) {
+        mbar_arrive_expect_tx(bar_z, 2 * TILE_BYTES);
+        tma_load_2d(sb + OFF_Z, &tm_z, h * D, c0, bar_z);
+        tma_load_2d(sb + OFF_Z + TILE_BYTES, &tm_z, h * D + 64, c0, bar_z);
+      }
+    }
 
     // ---- gates of the chunk: gamma = cumulative g, e^gamma, beta
-    float gv = 0.f, bv = 0.f;
+    float gv = g_next, bv = b_next;
     if (tid < 64) {
-      if (tid < L) {
-        gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
-        bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
-      }
+      if (c + 1 < nchunks) load_gates(c + 1);
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float t = __shfl_up_sync(0xffffffffu, gv, o);
@@ -241,6 +331,7 @@ __global__ void __launch_bounds__(NT, 1)
     // ---- D1 = [K; Q] K^T
     ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
     if (__syncthreads_or(!ok)) break;
+    GDN_PHASE(0);
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, false, false);
@@ -252,58 +343,68 @@ __global__ void __launch_bounds__(NT, 1)
       }
       mma_commit(bar_mma);
     }
+    // meanwhile: decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i, else 0) and e^{gamma_L - gamma_i}
+    {
+#pragma unroll 4
+      for (int e = tid; e < 64 * 64; e += NT) {
+        const int i = e >> 6, j = e & 63;
+        Ef[i * 65 + j] = j <= i ? __expf(gam[i] - gam[j]) : 0.f;
+      }
+      if (tid < 64) decL[tid] = __expf(gam[L - 1] - gam[tid]);
+    }
     ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_PHASE(1);
 
-    // ---- A (rows 0..63) and P (rows 64..127)
+    // ---- A (rows 0..63) and P (rows 64..127); this thread: columns wg*32 .. wg*32+31
     {
-      float x[64];
-      tmem_ld32(lane_base + TM_D1, x);
-      tmem_ld32(lane_base + TM_D1 + 32, x + 32);
-      if (tid < 64) {
-        const int i = tid;
-        const float gi = gam[i], bi = bet[i];
+      float x[32];
+      tmem_ld32(lane_base + TM_D1 + wg * 32, x);
+      if (tl < 64) {
+        const int i = tl;
+        const float bi = i < L ? bet[i] : 0.f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          Af[i * 65 + j] = (j < i && i < L) ? bi * __expf(gi - gam[j]) * x[j] : 0.f;
+        for (int e = 0; e < 32; ++e) {
+          const int j = wg * 32 + e;
+          Af[i * 65 + j] = j < i ? bi * Ef[i * 65 + j] * x[e] : 0.f;
+        }
       } else {
-        const int i = tid - 64;
-        const float gi = gam[i];
+        const int i = tl - 64;
+        const float keep = i < L ? 1.f : 0.f;
         uint8_t* P = smem + OFF_P;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = q * 8 + e;
-            f[e] = (j <= i && i < L) ? __expf(gi - gam[j]) * x[j] : 0.f;
-          }
-          st_half8(P, swz(i, q), f);
+          for (int e = 0; e < 8; ++e) f[e] = keep * Ef[i * 65 + wg * 32 + q * 8 + e] * x[q * 8 + e];
+          st_half8(P, swz(i, wg * 4 + q), f);
         }
       }
     }
     __syncthreads();
+    GDN_PHASE(2);
 
     // ---- T = (I + A)^-1, then the B operands T diag(beta) and T diag(beta e^gamma)
-    solve_unit_lower(Af, Tf, Rs, tid);
+    solve_unit_lower(Af, Tf, Xs, tid);
+    GDN_PHASE(3);
     {
-      const int i = tid >> 1, hf = tid & 1;
+      const int i = tid >> 2, qt = tid & 3;  // row i, 16 columns per thread
       uint8_t* Tb = smem + OFF_TB;
       uint8_t* Tbe = smem + OFF_TBE;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         float fb[8], fe[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int j = hf * 32 + q * 8 + e;
+          const int j = qt * 16 + q * 8 + e;
           const float t = Tf[i * 65 + j] * bet[j];
           fb[e] = t;
           fe[e] = t * eg[j];
         }
-        st_half8(Tb, swz(i, hf * 4 + q), fb);
-        st_half8(Tbe, swz(i, hf * 4 + q), fe);
+        st_half8(Tb, swz(i, qt * 2 + q), fb);
+        st_half8(Tbe, swz(i, qt * 2 + q), fe);
       }
     }
     fence_proxy_async();
@@ -327,20 +428,20 @@ __global__ void __launch_bounds__(NT, 1)
       mma_commit(bar_mma);
     }
 
-    // ---- meanwhile: S -> fp16 operand, and S *= e^{gamma_L} in TMEM
+    // ---- meanwhile: S -> fp16 operand (this thread: dk half wg), and S *= e^{gamma_L} in TMEM
     {
       const float egL = eg[L - 1];
-      uint8_t* Sb = smem + OFF_S;
+      uint8_t* half_base = smem + OFF_S + wg * 16384;
 #pragma unroll
-      for (int piece = 0; piece < 4; ++piece) {
+      for (int piece = 0; piece < 2; ++piece) {
+        const int col = wg * 64 + piece * 32;
         float r[32];
-        tmem_ld32(lane_base + TM_S + piece * 32, r);
-        uint8_t* half_base = Sb + (piece >> 1) * 16384;
+        tmem_ld32(lane_base + TM_S + col, r);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tid, (piece & 1) * 4 + q), r + q * 8);
+        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, piece * 4 + q), r + q * 8);
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] *= egL;
-        tmem_st32(lane_base + TM_S + piece * 32, r);
+        tmem_st32(lane_base + TM_S + col, r);
       }
       tmem_wait_st();
     }
@@ -349,16 +450,16 @@ __global__ void __launch_bounds__(NT, 1)
     mma_phase ^= 1;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_PHASE(4);
 
-    // ---- -W^T as the MN-major B operand (row l = tid, 64 tokens)
+    // ---- -W^T as the MN-major B operand (row l = tl, tokens wg*32 .. wg*32+31)
     {
-      float x[64];
-      tmem_ld32(lane_base + TM_D3, x);
-      tmem_ld32(lane_base + TM_D3 + 32, x + 32);
+      float x[32];
+      tmem_ld32(lane_base + TM_D3 + wg * 32, x);
 #pragma unroll
-      for (int j = 0; j < 64; ++j) x[j] = -x[j];
+      for (int j = 0; j < 32; ++j) x[j] = -x[j];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) st_half8(wt_ptr, swz(tid, q), x + q * 8);
+      for (int q = 0; q < 4; ++q) st_half8(wt_ptr, swz(tl, wg * 4 + q), x + q * 8);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -388,25 +489,24 @@ __global__ void __launch_bounds__(NT, 1)
     mma_phase ^= 1;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_PHASE(5);
 
     // ---- Vn^T rows: plain (A of D5) and decayed to the chunk end (A of the state update)
     {
-      float x[64];
-      tmem_ld32(lane_base + TM_D2, x);
-      tmem_ld32(lane_base + TM_D2 + 32, x + 32);
-      const float gL = gam[L - 1];
+      float x[32];
+      tmem_ld32(lane_base + TM_D2 + wg * 32, x);
       uint8_t* Vt = smem + OFF_TB;
       uint8_t* Vts = smem + OFF_VTS;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int i = q * 8 + e;
-          f[e] = i < L ? x[i] * __expf(gL - gam[i]) : 0.f;
+          const int i = wg * 32 + q * 8 + e;
+          f[e] = i < L ? x[q * 8 + e] * decL[i] : 0.f;
         }
-        st_half8(Vt, swz(tid, q), x + q * 8);
-        st_half8(Vts, swz(tid, q), f);
+        st_half8(Vt, swz(tl, wg * 4 + q), x + q * 8);
+        st_half8(Vts, swz(tl, wg * 4 + q), f);
       }
     }
     fence_proxy_async();
@@ -434,46 +534,71 @@ __global__ void __launch_bounds__(NT, 1)
     mma_phase ^= 1;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_PHASE(6);
 
-    // ---- epilogue: O^T = D4 diag(e^gamma) + D5, transposed through shared memory
+    // ---- epilogue: O^T = D4 diag(e^gamma) + D5, staged as O [token][v]; tokens wg*32 .. +31
     {
       float a4[32], a5[32];
+      tmem_ld32(lane_base + TM_D4 + wg * 32, a4);
+      tmem_ld32(lane_base + TM_D5 + wg * 32, a5);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(lane_base + TM_D4 + half * 32, a4);
-        tmem_ld32(lane_base + TM_D5 + half * 32, a5);
+      for (int j = 0; j < 32; ++j) {
+        const int i = wg * 32 + j;
+        Os[i * D + tl] = fmaf(eg[i], a4[j], a5[j]);
+      }
+    }
+    if (norm_out) ok = mbar_wait(bar_z, (uint32_t)c & 1u);
+    if (__syncthreads_or(!ok)) break;
+    GDN_PHASE(7);
+    if (norm_out) {
+      // 1 / rms per token: warp w reduces tokens 8w .. 8w+7
+      float ss[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = half * 32 + j;
-          Os[i * D + tid] = fmaf(eg[i], a4[j], a5[j]);
+      for (int t = 0; t < 8; ++t) {
+        const float* row = Os + (8 * warp + t) * D;
+        const float o0 = row[lane], o1 = row[lane + 32], o2 = row[lane + 64], o3 = row[lane + 96];
+        ss[t] = o0 * o0 + o1 * o1 + o2 * o2 + o3 * o3;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) ss[t] = warp_sum(ss[t]);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (lane == t) rms[8 * warp + t] = rsqrtf(ss[t] * (1.0f / D) + p.eps_norm);
+      __syncthreads();
+      // gated output, written over the z tile (each element read, then written, by one thread)
+      __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int i = wg * 32 + j;
+        const float o = Os[i * D + tl];
+        const float zf = __bfloat162float(zcol[i * 64]);
+        zcol[i * 64] = __float2bfloat16_rn(o * rms[i] * w_norm * silu_f(zf));
+      }
+      __syncthreads();
+      // rows 0..L-1 of the tile -> out, 16 bytes per thread and pass
+      uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv + h) * D * 2;
+      const size_t ostride = (size_t)p.Hv * D * 2;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = tid + NT * k, row = e >> 4, c16 = e & 15;
+        if (row < L) {
+          const uint4 val = *reinterpret_cast<const uint4*>(smem + OFF_Z + (c16 >> 3) * TILE_BYTES +
+                                                           row * 128 + (c16 & 7) * 16);
+          *reinterpret_cast<uint4*>(obase + row * ostride + c16 * 16) = val;
         }
+      }
+      fence_proxy_async();  // the next chunk's z tile lands here through TMA
+    } else {
+      float* ocol = p.o_raw + ((size_t)c0 * p.Hv + h) * D + tl;
+      const size_t ostride = (size_t)p.Hv * D;
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int i = wg * 32 + j;
+        if (i < L) ocol[i * ostride] = Os[i * D + tl];
       }
     }
     __syncthreads();
-    for (int i = warp; i < L; i += NT / 32) {
-      const size_t ob = ((size_t)(c0 + i) * p.Hv + h) * D;
-      float o[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) o[u] = Os[i * D + lane + 32 * u];
-      if (p.out) {
-        float ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
-        ss = warp_sum(ss);
-        const float inv = rsqrtf(ss * (1.0f / D) + p.eps_norm);
-        const __nv_bfloat16* zz = static_cast<const __nv_bfloat16*>(p.z) + ob;
-        const __nv_bfloat16* ww = static_cast<const __nv_bfloat16*>(p.norm_w);
-        __nv_bfloat16* oo = static_cast<__nv_bfloat16*>(p.out) + ob;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = lane + 32 * u;
-          oo[v] = __float2bfloat16_rn(o[u] * inv * __bfloat162float(ww[v]) *
-                                      silu_f(__bfloat162float(zz[v])));
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) p.o_raw[ob + lane + 32 * u] = o[u];
-      }
-    }
-    __syncthreads();
+    GDN_PHASE(8);
   }
 
   if (!ok) {
@@ -482,16 +607,19 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) {
       atomicExch(&g_tc_error, 1);
       mbar_wait(bar_load0 + 8 * (c & 1), (uint32_t)(c >> 1) & 1u, 100000000ull);
-      if (c + 1 < nchunks) mbar_wait(bar_load0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, 100000000ull);
+      if (c + 1 < nchunks)
+        mbar_wait(bar_load0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, 100000000ull);
+      if (norm_out) mbar_wait(bar_z, (uint32_t)c & 1u, 100000000ull);
     }
   } else if (p.S_out) {
     float r[32];
 #pragma unroll
-    for (int piece = 0; piece < 4; ++piece) {
-      tmem_ld32(lane_base + TM_S + piece * 32, r);
+    for (int piece = 0; piece < 2; ++piece) {
+      const int col = wg * 64 + piece * 32;
+      tmem_ld32(lane_base + TM_S + col, r);
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(p.S_out + sbase + (size_t)tid * D + piece * 32 + j) =
+        *reinterpret_cast<float4*>(p.S_out + sbase + (size_t)tl * D + col + j) =
             make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
     }
   }
@@ -521,18 +649,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map over a row-major fp16 [rows, cols] array, 64 x 64 boxes,
-// 128-byte swizzle; rows past the end read as zeros.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+// Tensor map over a row-major 16-bit [rows, cols] array with 64 x 64 boxes;
+// rows past the end read as zeros.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              CUtensorMapDataType dt, CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, 64};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -543,25 +671,43 @@ bool chunk_tc_supported(int d, int chunk, gdn_dtype dt_mid) {
 
 cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st) {
   if (p.N == 0 || p.Hv == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mz;
   memset(&mq, 0, sizeof(mq));
   memset(&mk, 0, sizeof(mk));
   memset(&mv, 0, sizeof(mv));
+  memset(&mz, 0, sizeof(mz));
   if (p.T > 0) {
-    if (!make_map(&mq, p.q, (uint64_t)p.T, (uint64_t)p.Hk * D) ||
-        !make_map(&mk, p.k, (uint64_t)p.T, (uint64_t)p.Hk * D) ||
-        !make_map(&mv, p.v, (uint64_t)p.T, (uint64_t)p.Hv * D))
+    const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map(&mq, p.q, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
+        !make_map(&mk, p.k, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
+        !make_map(&mv, p.v, (uint64_t)p.T, (uint64_t)p.Hv * D, f16, sw))
+      return cudaErrorInvalidValue;
+    if (p.out && !make_map(&mz, p.z, (uint64_t)p.T, (uint64_t)p.Hv * D,
+                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.Hv, p.N);
-  chunk_tc_kernel<<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, p);
+  chunk_tc_kernel<<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mz, p);
   return cudaGetLastError();
 }
 
 }  // namespace gdn
+
+#ifdef GDN_PHASE_TIMING
+extern "C" int gdn_debug_phase_cycles(unsigned long long* out, int clear) {
+  cudaDeviceSynchronize();
+  if (cudaMemcpyFromSymbol(out, gdn::g_phase_cycles, sizeof(unsigned long long) * 16) != cudaSuccess) return -1;
+  if (clear) {
+    unsigned long long z[16] = {0};
+    cudaMemcpyToSymbol(gdn::g_phase_cycles, z, sizeof(z));
+  }
+  return 0;
+}
+#endif
 
 extern "C" gdn_status gdn_device_error(int* code, int clear) {
   if (!code) return GDN_ERR_NULL;
