@@ -32,8 +32,11 @@ GDN_IMPL_AUTO = 0
 GDN_IMPL_SIMT = 1
 GDN_IMPL_TC = 2
 
-EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_chunk_core",
-            "gdn_device_error", "gdn_status_string", "gdn_version"]
+EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_noalloc", "gdn_decode",
+            "gdn_chunk_core", "gdn_device_error", "gdn_status_string", "gdn_version"]
+
+# Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
+GDN_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class gdn_dims(ctypes.Structure):
@@ -85,6 +88,9 @@ def lib():
         L.gdn_prefill_workspace_size.restype = ctypes.c_size_t
         L.gdn_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args), _vp]
         L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill_noalloc.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
+                                          _vp]
+        L.gdn_prefill_noalloc.restype = ctypes.c_int
         L.gdn_decode.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_decode_args), _vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_chunk_core.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_core_args), _vp]
@@ -163,6 +169,23 @@ def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, n
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill(ctypes.byref(dims), ctypes.byref(args), s), "gdn_prefill",
                   raise_on_error)
+
+
+def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,
+                        cu_seqlens, N, T_tot, chunk, dtype, out, initial_state=None,
+                        final_state=None, conv_state_in=None, conv_state_out=None,
+                        impl=GDN_IMPL_AUTO, stream=None, raise_on_error=True) -> int:
+    """gdn_prefill on the library's own scratch: for callers that have no way
+    to allocate a workspace (see gdn.h).  Calls that overlap on the GPU race
+    on the shared scratch."""
+    args = gdn_prefill_args(
+        ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
+        ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
+        ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
+        None, 0, None, None)
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_prefill_noalloc(ctypes.byref(dims), ctypes.byref(args), s),
+                  "gdn_prefill_noalloc", raise_on_error)
 
 
 def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w, state,

@@ -147,6 +147,37 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dty
  * conv_state_out when given.  The workspace is overwritten. */
 gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* args, void* stream);
 
+/* ------------------------------------------------ prefill without workspace
+ * No counterpart on the pages: this is an addition of this library for
+ * callers that cannot hand gdn_prefill a workspace -- e.g. an operator plugin
+ * that receives only its input and output tensors and has no allocator to
+ * ask for temporary device memory, or a runtime that has carved up all device
+ * memory up front and allows no cudaMalloc (nor its implicit device
+ * synchronisation) while serving.
+ *
+ * gdn_prefill_noalloc runs gdn_prefill with its workspace taken from one
+ * fixed scratch array inside the library (GDN_NOALLOC_SCRATCH_BYTES of device
+ * memory, held on every device that loads the library until the process
+ * exits).  It allocates nothing.
+ *   - args->workspace and args->workspace_bytes are ignored; every other
+ *     argument means what it means for gdn_prefill, with the same checks.
+ *   - Returns GDN_ERR_WORKSPACE, launching nothing, when the workspace these
+ *     sizes need (gdn_prefill_workspace_size) exceeds
+ *     GDN_NOALLOC_SCRATCH_BYTES -- about 5400 tokens at 16 key / 16 value
+ *     heads of width 128, bf16.
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call outside any
+ *     CUDA stream capture.  GDN_ERR_CUDA if the lookup fails.
+ *   - All calls share the one scratch array, which keeps the previous call's
+ *     contents (nothing in it needs to start at zero).  Calls whose work may
+ *     overlap on the GPU -- on different streams, or from host threads that
+ *     do not order their streams -- race on it and corrupt each other's
+ *     results: issue them on one stream, or order them.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+gdn_status gdn_prefill_noalloc(const gdn_dims* dims, const gdn_prefill_args* args, void* stream);
+
 /* ------------------------------------------------------------------- decode
  * One token for each of B independent sequences.  state and conv_state are
  * read and overwritten in place with the values after this token.
