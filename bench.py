@@ -20,6 +20,7 @@ timed region.  `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -47,6 +48,50 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------- multi-rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------ profiled traffic
+
+PROFILES = os.path.join(ROOT, "profiles", "ncu_traffic.tsv")
+CSRC = os.path.join(ROOT, "hybrid_linear_attention_05_b200", "csrc")
+
+
+def source_digest(name: str) -> str:
+    with open(os.path.join(CSRC, name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(source: str, workload: str):
+    """DRAM bytes per launch recorded by an ncu capture of `source` on
+    `workload`, or None when there is none or the source changed since."""
+    if not os.path.exists(PROFILES):
+        return None
+    digest = source_digest(source)
+    for line in open(PROFILES):
+        parts = line.rstrip("\n").split("\t")
+        if len(parts) >= 4 and not line.startswith("#"):
+            if parts[0] == source and parts[1] == digest and parts[2] == workload:
+                return float(parts[3])
+    return None
 
 
 # ------------------------------------------------------------ work counts
@@ -249,14 +294,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     core_ms = [a.elapsed_time(b) for a, b in cevs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     tokens = inp.T * world
-    value = tokens / (ms_per_step * 1e-3)
+    value = job_throughput(inp.T, world, ms_per_step * 1e-3)
 
     cnt = prefill_counts(inp, dp.chunk)
     core_avg_s = statistics.mean(core_ms) * 1e-3
@@ -268,7 +309,8 @@ def run_ours(args, rank, world, local_rank):
         "peak": hbm,
         "unit": "GB/s",
         "frac": cnt["core_bytes"] / core_avg_s / 1e9 / hbm,
-        "traffic": args.core_traffic,
+        "traffic": args.core_traffic if args.core_traffic is not None else
+                   profiled_traffic("chunk_tc.cu" if dp.chunk == 64 else "chunk_simt.cu", args.workload),
         "peak_source": peak_kind,
         "algorithmic_bytes_per_launch": cnt["core_bytes"],
         "algorithmic_flops_per_launch": cnt["core_flops"],
@@ -311,12 +353,8 @@ def run_ours(args, rank, world, local_rank):
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e = {"value": tokens / (e2e_total / args.steps * 1e-3), "unit": "tokens/s",
+    e2e_total = max_over_ranks(sum(e2e_ms), dev)
+    e2e = {"value": job_throughput(inp.T, world, e2e_total / args.steps * 1e-3), "unit": "tokens/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     del host, h_out, h_S
 
@@ -339,20 +377,18 @@ def run_ours(args, rank, world, local_rank):
         dev_ms.append((a, b))
     torch.cuda.synchronize()
     d_ms = [a.elapsed_time(b) for a, b in dev_ms]
-    d_total = sum(d_ms)
-    if world > 1:
-        t = torch.tensor([d_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        d_total = float(t.item())
+    d_total = max_over_ranks(sum(d_ms), dev)
     dcnt = decode_counts(dinp)
     d_step_s = d_total / args.steps * 1e-3
     decode = {
         "metric": "GDN decode tokens/s per layer", "unit": "tokens/s",
-        "value": dd.B * world / d_step_s, "ms_per_step": d_step_s * 1e3,
+        "value": job_throughput(dd.B, world, d_step_s), "ms_per_step": d_step_s * 1e3,
         "workload": args.decode_workload,
         "roofline": {"kernel": "gdn_decode", "bound": "hbm",
                      "achieved": dcnt["bytes"] / d_step_s / 1e9, "peak": hbm, "unit": "GB/s",
-                     "frac": dcnt["bytes"] / d_step_s / 1e9 / hbm, "traffic": args.decode_traffic,
+                     "frac": dcnt["bytes"] / d_step_s / 1e9 / hbm,
+                     "traffic": args.decode_traffic if args.decode_traffic is not None else
+                                profiled_traffic("decode.cu", args.decode_workload),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": dcnt["bytes"]},
         "l2": "state (%d MiB) larger than L2" % (dd.state.numel() * 4 >> 20),
     }
