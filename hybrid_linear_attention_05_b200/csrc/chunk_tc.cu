@@ -69,9 +69,11 @@ constexpr uint32_t OFF_TB = 139264;   // T diag(beta); with OFF_TBE later holds 
 constexpr uint32_t OFF_TBE = 147456;  // T diag(beta e^gamma)
 constexpr uint32_t OFF_VTS = 155648;  // Vn^T diag(e^{gamma_L - gamma}), 128 rows x 128 B
 constexpr uint32_t OFF_Z = 172032;    // z tile (bf16, two dv halves x 64 tokens x 128 B); then the output tile
-constexpr uint32_t OFF_AF = 188416;   // fp32 A [64][65]; the epilogue reuses AF..TF as O [64][128]
-constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4;     // fp32 T [64][65]; before it, the decay table E
-constexpr uint32_t OFF_RS = OFF_TF + 64 * 65 * 4;     // fp32 scratch of the inverse, 1024 floats
+constexpr int AS = 68;                // row stride (floats) of A and T: 16-byte aligned rows
+constexpr int ES = 65;                // row stride of the decay table E (conflict-free row walks)
+constexpr uint32_t OFF_AF = 188416;   // fp32 A [64][AS]; the epilogue reuses AF..TF as O [64][128]
+constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;     // fp32 T [64][AS]; before it, the decay table E
+constexpr uint32_t OFF_RS = OFF_TF + 64 * AS * 4;     // fp32 scratch of the inverse, 1024 floats
 constexpr uint32_t OFF_MISC = OFF_RS + 1024 * 4;      // gamma, e^gamma, beta, rms, e^{gamma_L - gamma}, scan
 constexpr uint32_t OFF_BAR = OFF_MISC + 5 * 64 * 4 + 64;
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
@@ -95,7 +97,7 @@ __device__ __forceinline__ void st_half8(uint8_t* base, uint32_t off, const floa
 }
 
 // Tf := (I + A)^-1 for the strictly lower triangular 64 x 64 A (fp32, row
-// stride 65), by recursive doubling of the block size:
+// stride AS), by recursive doubling of the block size:
 //   16 x 16 diagonal blocks by forward substitution (one column per thread);
 //   32 x 32: T_{r,r-1} = -T_rr A_{r,r-1} T_{r-1,r-1} for the 16-blocks (1,0), (3,2);
 //   64 x 64: T_{LL}   = -T_bb A_{LL} T_tt for the lower-left 32-block.
@@ -110,20 +112,20 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
       float a0 = (i == m) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
       for (int j = 0; j < i; j += 2) {
-        a0 = fmaf(-Af[(16 * b + i) * 65 + 16 * b + j], x[j], a0);
-        if (j + 1 < i) a1 = fmaf(-Af[(16 * b + i) * 65 + 16 * b + j + 1], x[j + 1], a1);
+        a0 = fmaf(-Af[(16 * b + i) * AS + 16 * b + j], x[j], a0);
+        if (j + 1 < i) a1 = fmaf(-Af[(16 * b + i) * AS + 16 * b + j + 1], x[j + 1], a1);
       }
       x[i] = a0 + a1;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * 65 + 16 * b + m] = x[i];
+    for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AS + 16 * b + m] = x[i];
   } else {
     // 16-blocks above the diagonal are zero
     for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
       const int blk = e >> 8, w = e & 255, i = w >> 4, m = w & 15;
       const int r = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
       const int c = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-      Tf[(16 * r + i) * 65 + 16 * c + m] = 0.f;
+      Tf[(16 * r + i) * AS + 16 * c + m] = 0.f;
     }
   }
   __syncthreads();
@@ -135,8 +137,8 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
-        acc[k] = fmaf(Af[(16 * r + i) * 65 + 16 * (r - 1) + j],
-                      Tf[(16 * (r - 1) + j) * 65 + 16 * (r - 1) + m], acc[k]);
+        acc[k] = fmaf(Af[(16 * r + i) * AS + 16 * (r - 1) + j],
+                      Tf[(16 * (r - 1) + j) * AS + 16 * (r - 1) + m], acc[k]);
       }
     }
 #pragma unroll
@@ -150,24 +152,29 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int e = tid + NT * k, blk = e >> 8, r = blk ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
-        acc[k] = fmaf(Tf[(16 * r + i) * 65 + 16 * r + j], X[blk * 256 + j * 16 + m], acc[k]);
+        acc[k] = fmaf(Tf[(16 * r + i) * AS + 16 * r + j], X[blk * 256 + j * 16 + m], acc[k]);
       }
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
-      Tf[(16 * r + i) * 65 + 16 * (r - 1) + m] = -acc[k];
+      Tf[(16 * r + i) * AS + 16 * (r - 1) + m] = -acc[k];
     }
   }
   __syncthreads();
   // 64 x 64: rows 32 + warp + 8k of the lower-left block, column `lane`
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
-      const float t = Tf[j * 65 + lane];
+#pragma unroll 2
+    for (int j = 0; j < 32; j += 4) {
+      float t[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = fmaf(Af[(32 + warp + 8 * k) * 65 + j], t, acc[k]);
+      for (int q = 0; q < 4; ++q) t[q] = Tf[(j + q) * AS + lane];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 a4 = *reinterpret_cast<const float4*>(Af + (32 + warp + 8 * k) * AS + j);
+        acc[k] = fmaf(a4.x, t[0], fmaf(a4.y, t[1], fmaf(a4.z, t[2], fmaf(a4.w, t[3], acc[k]))));
+      }
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) X[(warp + 8 * k) * 32 + lane] = acc[k];
@@ -175,14 +182,19 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
   __syncthreads();
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
-      const float x = X[j * 32 + lane];
+#pragma unroll 2
+    for (int j = 0; j < 32; j += 4) {
+      float x[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = fmaf(Tf[(32 + warp + 8 * k) * 65 + 32 + j], x, acc[k]);
+      for (int q = 0; q < 4; ++q) x[q] = X[(j + q) * 32 + lane];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (32 + warp + 8 * k) * AS + 32 + j);
+        acc[k] = fmaf(t4.x, x[0], fmaf(t4.y, x[1], fmaf(t4.z, x[2], fmaf(t4.w, x[3], acc[k]))));
+      }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) Tf[(32 + warp + 8 * k) * 65 + lane] = -acc[k];
+    for (int k = 0; k < 4; ++k) Tf[(32 + warp + 8 * k) * AS + lane] = -acc[k];
   }
   __syncthreads();
 }
@@ -196,7 +208,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sb = smem_u32(smem);
   float* Af = reinterpret_cast<float*>(smem + OFF_AF);
   float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
-  float* Ef = Tf;  // decay table e^{gamma_i - gamma_j}, [64][65], alive before the inverse
+  float* Ef = Tf;  // decay table e^{gamma_i - gamma_j}, [64][ES], alive before the inverse
   float* Xs = reinterpret_cast<float*>(smem + OFF_RS);
   float* Os = reinterpret_cast<float*>(smem + OFF_AF);
   __nv_bfloat16* Zs = reinterpret_cast<__nv_bfloat16*>(smem + OFF_Z);
@@ -206,8 +218,11 @@ __global__ void __launch_bounds__(NT, 1)
   float* rms = bet + 64;
   float* decL = rms + 64;
   float* scan = decL + 64;
-  const uint32_t bar_load0 = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 16, bar_z = sb + OFF_BAR + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 32);
+  // mbarriers: TMA stages 0/1, z tile, and one per tensor-core commit point
+  const uint32_t bar_load0 = sb + OFF_BAR, bar_z = sb + OFF_BAR + 16;
+  const uint32_t bar_m1 = sb + OFF_BAR + 24, bar_w = sb + OFF_BAR + 32, bar_v = sb + OFF_BAR + 40,
+                 bar_o = sb + OFF_BAR + 48;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 56);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7;     // warpgroup: which column half of a TMEM row this thread handles
@@ -229,8 +244,11 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0) {
     mbar_init(bar_load0, 1);
     mbar_init(bar_load0 + 8, 1);
-    mbar_init(bar_mma, 1);
     mbar_init(bar_z, 1);
+    mbar_init(bar_m1, 1);
+    mbar_init(bar_w, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_o, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -286,7 +304,6 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_wait_st();
   }
 
-  uint32_t mma_phase = 0;
   bool ok = true;
   int c = 0;
 #ifdef GDN_PHASE_TIMING
@@ -332,6 +349,7 @@ __global__ void __launch_bounds__(NT, 1)
     ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
     if (__syncthreads_or(!ok)) break;
     GDN_PHASE(0);
+    const uint32_t par = (uint32_t)c & 1u;  // phase parity of the once-per-chunk barriers
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, false, false);
@@ -341,19 +359,34 @@ __global__ void __launch_bounds__(NT, 1)
         mma_f16(tmem + TM_D1, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
                 kk > 0);
       }
-      mma_commit(bar_mma);
+      mma_commit(bar_m1);
     }
-    // meanwhile: decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i, else 0) and e^{gamma_L - gamma_i}
+    // meanwhile: decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i), e^{gamma_L - gamma_i},
+    // and the state: fp16 copy for this chunk's products, then S *= e^{gamma_L} in TMEM
     {
 #pragma unroll 4
       for (int e = tid; e < 64 * 64; e += NT) {
         const int i = e >> 6, j = e & 63;
-        Ef[i * 65 + j] = j <= i ? __expf(gam[i] - gam[j]) : 0.f;
+        if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gam[j]);
       }
       if (tid < 64) decL[tid] = __expf(gam[L - 1] - gam[tid]);
+      const float egL = eg[L - 1];
+      uint8_t* half_base = smem + OFF_S + wg * 16384;
+#pragma unroll
+      for (int piece = 0; piece < 2; ++piece) {
+        const int col = wg * 64 + piece * 32;
+        float r[32];
+        tmem_ld32(lane_base + TM_S + col, r);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, piece * 4 + q), r + q * 8);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] *= egL;
+        tmem_st32(lane_base + TM_S + col, r);
+      }
+      tmem_wait_st();
+      fence_proxy_async();
     }
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
+    ok = mbar_wait(bar_m1, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     GDN_PHASE(1);
@@ -366,9 +399,15 @@ __global__ void __launch_bounds__(NT, 1)
         const int i = tl;
         const float bi = i < L ? bet[i] : 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = wg * 32 + e;
-          Af[i * 65 + j] = j < i ? bi * Ef[i * 65 + j] * x[e] : 0.f;
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          float4 v;
+          float* vf = reinterpret_cast<float*>(&v);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = wg * 32 + e4 + u;
+            vf[u] = j < i ? bi * Ef[i * ES + j] * x[e4 + u] : 0.f;
+          }
+          *reinterpret_cast<float4*>(Af + i * AS + wg * 32 + e4) = v;
         }
       } else {
         const int i = tl - 64;
@@ -378,7 +417,10 @@ __global__ void __launch_bounds__(NT, 1)
         for (int q = 0; q < 4; ++q) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = keep * Ef[i * 65 + wg * 32 + q * 8 + e] * x[q * 8 + e];
+          for (int e = 0; e < 8; ++e) {
+            const int j = wg * 32 + q * 8 + e;
+            f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
+          }
           st_half8(P, swz(i, wg * 4 + q), f);
         }
       }
@@ -397,11 +439,16 @@ __global__ void __launch_bounds__(NT, 1)
       for (int q = 0; q < 2; ++q) {
         float fb[8], fe[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = qt * 16 + q * 8 + e;
-          const float t = Tf[i * 65 + j] * bet[j];
-          fb[e] = t;
-          fe[e] = t * eg[j];
+        for (int e4 = 0; e4 < 8; e4 += 4) {
+          const int j0 = qt * 16 + q * 8 + e4;
+          const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + j0);
+          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float t = tv[u] * bet[j0 + u];
+            fb[e4 + u] = t;
+            fe[e4 + u] = t * eg[j0 + u];
+          }
         }
         st_half8(Tb, swz(i, qt * 2 + q), fb);
         st_half8(Tbe, swz(i, qt * 2 + q), fe);
@@ -411,43 +458,24 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_before();
     __syncthreads();
 
-    // ---- D2 = V^T Tb^T (= U^T), D3 = K^T Tbe^T (= W^T)
+    // ---- D3 = K^T Tbe^T (= W^T), committed alone; then D2 = V^T Tb^T (= U^T), which the
+    //      in-order tensor pipe finishes before the D2 accumulation below
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, true, false);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        mma_f16(tmem + TM_D2, sdesc_sw128(vv + kk * 2048, 8192, 1024),
-                sdesc_sw128(sb + OFF_TB + kk * 32, 16, 1024), id, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
         mma_f16(tmem + TM_D3, sdesc_sw128(kq + kk * 2048, 16384, 1024),
                 sdesc_sw128(sb + OFF_TBE + kk * 32, 16, 1024), id, kk > 0);
       }
-      mma_commit(bar_mma);
-    }
-
-    // ---- meanwhile: S -> fp16 operand (this thread: dk half wg), and S *= e^{gamma_L} in TMEM
-    {
-      const float egL = eg[L - 1];
-      uint8_t* half_base = smem + OFF_S + wg * 16384;
+      mma_commit(bar_w);
 #pragma unroll
-      for (int piece = 0; piece < 2; ++piece) {
-        const int col = wg * 64 + piece * 32;
-        float r[32];
-        tmem_ld32(lane_base + TM_S + col, r);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, piece * 4 + q), r + q * 8);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] *= egL;
-        tmem_st32(lane_base + TM_S + col, r);
+      for (int kk = 0; kk < 4; ++kk) {
+        mma_f16(tmem + TM_D2, sdesc_sw128(vv + kk * 2048, 8192, 1024),
+                sdesc_sw128(sb + OFF_TB + kk * 32, 16, 1024), id, kk > 0);
       }
-      tmem_wait_st();
     }
-    fence_proxy_async();
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
+    ok = mbar_wait(bar_w, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     GDN_PHASE(4);
@@ -465,7 +493,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_before();
     __syncthreads();
 
-    // ---- D2 += S (-W^T)  (= Vn^T),  D4 = S Q^T
+    // ---- D2 += S (-W^T)  (= Vn^T), committed alone; then D4 = S Q^T
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id_w = idesc_f16(128, 64, false, true);
@@ -477,16 +505,15 @@ __global__ void __launch_bounds__(NT, 1)
         mma_f16(tmem + TM_D2, sdesc_sw128(sb + OFF_S + aoff, 16, 1024),
                 sdesc_sw128(wt + kk * 2048, 16384, 1024), id_w, 1);
       }
+      mma_commit(bar_v);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
         mma_f16(tmem + TM_D4, sdesc_sw128(sb + OFF_S + aoff, 16, 1024),
                 sdesc_sw128(kq + aoff + 8192, 16, 1024), id_q, kk > 0);
       }
-      mma_commit(bar_mma);
     }
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
+    ok = mbar_wait(bar_v, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     GDN_PHASE(5);
@@ -528,27 +555,35 @@ __global__ void __launch_bounds__(NT, 1)
         mma_f16(tmem + TM_D5, sdesc_sw128(sb + OFF_TB + kk * 32, 16, 1024),
                 sdesc_sw128(sb + OFF_P + kk * 32, 16, 1024), id_p, kk > 0);
       }
-      mma_commit(bar_mma);
+      mma_commit(bar_o);
     }
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
+    // meanwhile: w * silu(z) for this thread's outputs (column tl, tokens wg*32 .. wg*32+31)
+    float zw[32];
+    if (norm_out) {
+      ok = mbar_wait(bar_z, par);
+      const __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) zw[j] = w_norm * silu_f(__bfloat162float(zcol[(wg * 32 + j) * 64]));
+    }
+    ok = mbar_wait(bar_o, par) && ok;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     GDN_PHASE(6);
 
-    // ---- epilogue: O^T = D4 diag(e^gamma) + D5, staged as O [token][v]; tokens wg*32 .. +31
+    // ---- epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*32 .. +31, staged as O [token][v]
+    float o[32];
     {
-      float a4[32], a5[32];
-      tmem_ld32(lane_base + TM_D4 + wg * 32, a4);
+      float a5[32];
+      tmem_ld32(lane_base + TM_D4 + wg * 32, o);
       tmem_ld32(lane_base + TM_D5 + wg * 32, a5);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int i = wg * 32 + j;
-        Os[i * D + tl] = fmaf(eg[i], a4[j], a5[j]);
+        o[j] = fmaf(eg[i], o[j], a5[j]);
+        Os[i * D + tl] = o[j];
       }
     }
-    if (norm_out) ok = mbar_wait(bar_z, (uint32_t)c & 1u);
-    if (__syncthreads_or(!ok)) break;
+    __syncthreads();
     GDN_PHASE(7);
     if (norm_out) {
       // 1 / rms per token: warp w reduces tokens 8w .. 8w+7
@@ -567,13 +602,12 @@ __global__ void __launch_bounds__(NT, 1)
       __syncthreads();
       // gated output, written over the z tile (each element read, then written, by one thread)
       __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
-#pragma unroll 8
+#pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int i = wg * 32 + j;
-        const float o = Os[i * D + tl];
-        const float zf = __bfloat162float(zcol[i * 64]);
-        zcol[i * 64] = __float2bfloat16_rn(o * rms[i] * w_norm * silu_f(zf));
+        zcol[i * 64] = __float2bfloat16_rn(o[j] * rms[i] * zw[j]);
       }
+      fence_proxy_async();  // the next chunk's z tile lands here through TMA
       __syncthreads();
       // rows 0..L-1 of the tile -> out, 16 bytes per thread and pass
       uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv + h) * D * 2;
@@ -587,14 +621,13 @@ __global__ void __launch_bounds__(NT, 1)
           *reinterpret_cast<uint4*>(obase + row * ostride + c16 * 16) = val;
         }
       }
-      fence_proxy_async();  // the next chunk's z tile lands here through TMA
     } else {
       float* ocol = p.o_raw + ((size_t)c0 * p.Hv + h) * D + tl;
       const size_t ostride = (size_t)p.Hv * D;
-#pragma unroll 8
+#pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int i = wg * 32 + j;
-        if (i < L) ocol[i * ostride] = Os[i * D + tl];
+        if (i < L) ocol[i * ostride] = o[j];
       }
     }
     __syncthreads();
@@ -610,6 +643,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (c + 1 < nchunks)
         mbar_wait(bar_load0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, 100000000ull);
       if (norm_out) mbar_wait(bar_z, (uint32_t)c & 1u, 100000000ull);
+      mbar_wait(bar_o, (uint32_t)c & 1u, 100000000ull);  // tensor-core work of this chunk
     }
   } else if (p.S_out) {
     float r[32];
