@@ -56,7 +56,12 @@ using namespace ptx;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 256;  // two warpgroups; each TMEM lane (row) is split by columns between them
+constexpr int NT = 512;   // four warpgroups; each TMEM lane (row) is split by columns between them
+constexpr int NW = NT / 32;
+constexpr int NWG = NT / 128;
+constexpr int CW = 64 / NWG;   // columns of a 64-wide accumulator per warpgroup (16)
+constexpr int SW = 128 / NWG;  // columns of the 128-wide state per warpgroup (32)
+static_assert(CW == 16 && SW == 32, "column split assumes four warpgroups");
 
 // shared memory layout, byte offsets from a 1024-aligned base
 constexpr uint32_t OFF_KQ0 = 0;       // [K;Q] tile, stage 0: two dk halves x 128 rows x 128 B
@@ -129,72 +134,82 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
     }
   }
   __syncthreads();
-  // 32 x 32 diagonal blocks: element e = tid + 256 k -> 16-block (r, r-1), r = 1 or 3
+  // 32 x 32 diagonal blocks: element e = tid + NT k -> 16-block (r, r-1), r = 1 or 3
+  constexpr int K1 = 512 / NT;
   {
-    float acc[2] = {0.f, 0.f};
+    float acc[K1];
+#pragma unroll
+    for (int k = 0; k < K1; ++k) acc[k] = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < K1; ++k) {
         const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
         acc[k] = fmaf(Af[(16 * r + i) * AS + 16 * (r - 1) + j],
                       Tf[(16 * (r - 1) + j) * AS + 16 * (r - 1) + m], acc[k]);
       }
     }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) X[tid + NT * k] = acc[k];
+    for (int k = 0; k < K1; ++k) X[tid + NT * k] = acc[k];
   }
   __syncthreads();
   {
-    float acc[2] = {0.f, 0.f};
+    float acc[K1];
+#pragma unroll
+    for (int k = 0; k < K1; ++k) acc[k] = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < K1; ++k) {
         const int e = tid + NT * k, blk = e >> 8, r = blk ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
         acc[k] = fmaf(Tf[(16 * r + i) * AS + 16 * r + j], X[blk * 256 + j * 16 + m], acc[k]);
       }
     }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < K1; ++k) {
       const int e = tid + NT * k, r = (e >> 8) ? 3 : 1, i = (e >> 4) & 15, m = e & 15;
       Tf[(16 * r + i) * AS + 16 * (r - 1) + m] = -acc[k];
     }
   }
   __syncthreads();
-  // 64 x 64: rows 32 + warp + 8k of the lower-left block, column `lane`
+  // 64 x 64: rows 32 + warp + NW k of the lower-left block, column `lane`
+  constexpr int K2 = 32 / NW;
   {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[K2];
+#pragma unroll
+    for (int k = 0; k < K2; ++k) acc[k] = 0.f;
 #pragma unroll 2
     for (int j = 0; j < 32; j += 4) {
       float t[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) t[q] = Tf[(j + q) * AS + lane];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 a4 = *reinterpret_cast<const float4*>(Af + (32 + warp + 8 * k) * AS + j);
+      for (int k = 0; k < K2; ++k) {
+        const float4 a4 = *reinterpret_cast<const float4*>(Af + (32 + warp + NW * k) * AS + j);
         acc[k] = fmaf(a4.x, t[0], fmaf(a4.y, t[1], fmaf(a4.z, t[2], fmaf(a4.w, t[3], acc[k]))));
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) X[(warp + 8 * k) * 32 + lane] = acc[k];
+    for (int k = 0; k < K2; ++k) X[(warp + NW * k) * 32 + lane] = acc[k];
   }
   __syncthreads();
   {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[K2];
+#pragma unroll
+    for (int k = 0; k < K2; ++k) acc[k] = 0.f;
 #pragma unroll 2
     for (int j = 0; j < 32; j += 4) {
       float x[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) x[q] = X[(j + q) * 32 + lane];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (32 + warp + 8 * k) * AS + 32 + j);
+      for (int k = 0; k < K2; ++k) {
+        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (32 + warp + NW * k) * AS + 32 + j);
         acc[k] = fmaf(t4.x, x[0], fmaf(t4.y, x[1], fmaf(t4.z, x[2], fmaf(t4.w, x[3], acc[k]))));
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) Tf[(32 + warp + 8 * k) * AS + lane] = -acc[k];
+    for (int k = 0; k < K2; ++k) Tf[(32 + warp + NW * k) * AS + lane] = -acc[k];
   }
   __syncthreads();
 }
@@ -225,7 +240,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 56);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wg = tid >> 7;     // warpgroup: which column half of a TMEM row this thread handles
+  const int wg = tid >> 7;     // warpgroup: which column quarter of a TMEM row this thread handles
   const int tl = tid & 127;    // TMEM lane (row) of this thread
   const int h = blockIdx.x, n = blockIdx.y;
   const int hk = h / (p.Hv / p.Hk);
@@ -287,20 +302,17 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid < 64) load_gates(0);
   const float w_norm = norm_out ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tl]) : 0.f;
 
-  // initial state -> TMEM (row tl, columns wg*64 .. wg*64+63)
+  // initial state -> TMEM (row tl, columns wg*SW .. wg*SW+SW-1)
   {
     float r[32];
+    const int col = wg * SW;
 #pragma unroll
-    for (int piece = 0; piece < 2; ++piece) {
-      const int col = wg * 64 + piece * 32;
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        float4 f = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)tl * D + col + j)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        r[j] = f.x; r[j + 1] = f.y; r[j + 2] = f.z; r[j + 3] = f.w;
-      }
-      tmem_st32(lane_base + TM_S + col, r);
+    for (int j = 0; j < 32; j += 4) {
+      float4 f = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)tl * D + col + j)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      r[j] = f.x; r[j + 1] = f.y; r[j + 2] = f.z; r[j + 3] = f.w;
     }
+    tmem_st32(lane_base + TM_S + col, r);
     tmem_wait_st();
   }
 
@@ -371,14 +383,13 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (tid < 64) decL[tid] = __expf(gam[L - 1] - gam[tid]);
       const float egL = eg[L - 1];
-      uint8_t* half_base = smem + OFF_S + wg * 16384;
-#pragma unroll
-      for (int piece = 0; piece < 2; ++piece) {
-        const int col = wg * 64 + piece * 32;
+      uint8_t* half_base = smem + OFF_S + (wg >> 1) * 16384;  // dk half holding columns wg*SW..
+      {
+        const int col = wg * SW;
         float r[32];
         tmem_ld32(lane_base + TM_S + col, r);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, piece * 4 + q), r + q * 8);
+        for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, (wg & 1) * 4 + q), r + q * 8);
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] *= egL;
         tmem_st32(lane_base + TM_S + col, r);
@@ -391,37 +402,37 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     GDN_PHASE(1);
 
-    // ---- A (rows 0..63) and P (rows 64..127); this thread: columns wg*32 .. wg*32+31
+    // ---- A (rows 0..63) and P (rows 64..127); this thread: columns wg*CW .. wg*CW+CW-1
     {
-      float x[32];
-      tmem_ld32(lane_base + TM_D1 + wg * 32, x);
+      float x[CW];
+      tmem_ld16(lane_base + TM_D1 + wg * CW, x);
       if (tl < 64) {
         const int i = tl;
         const float bi = i < L ? bet[i] : 0.f;
 #pragma unroll
-        for (int e4 = 0; e4 < 32; e4 += 4) {
+        for (int e4 = 0; e4 < CW; e4 += 4) {
           float4 v;
           float* vf = reinterpret_cast<float*>(&v);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int j = wg * 32 + e4 + u;
+            const int j = wg * CW + e4 + u;
             vf[u] = j < i ? bi * Ef[i * ES + j] * x[e4 + u] : 0.f;
           }
-          *reinterpret_cast<float4*>(Af + i * AS + wg * 32 + e4) = v;
+          *reinterpret_cast<float4*>(Af + i * AS + wg * CW + e4) = v;
         }
       } else {
         const int i = tl - 64;
         const float keep = i < L ? 1.f : 0.f;
         uint8_t* P = smem + OFF_P;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < CW / 8; ++q) {
           float f[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int j = wg * 32 + q * 8 + e;
+            const int j = wg * CW + q * 8 + e;
             f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
           }
-          st_half8(P, swz(i, wg * 4 + q), f);
+          st_half8(P, swz(i, wg * (CW / 8) + q), f);
         }
       }
     }
@@ -432,15 +443,14 @@ __global__ void __launch_bounds__(NT, 1)
     solve_unit_lower(Af, Tf, Xs, tid);
     GDN_PHASE(3);
     {
-      const int i = tid >> 2, qt = tid & 3;  // row i, 16 columns per thread
+      const int i = tid >> 3, qt = tid & 7;  // row i, 8 columns (one 16-byte chunk) per thread
       uint8_t* Tb = smem + OFF_TB;
       uint8_t* Tbe = smem + OFF_TBE;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      {
         float fb[8], fe[8];
 #pragma unroll
         for (int e4 = 0; e4 < 8; e4 += 4) {
-          const int j0 = qt * 16 + q * 8 + e4;
+          const int j0 = qt * 8 + e4;
           const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + j0);
           const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
@@ -450,8 +460,8 @@ __global__ void __launch_bounds__(NT, 1)
             fe[e4 + u] = t * eg[j0 + u];
           }
         }
-        st_half8(Tb, swz(i, qt * 2 + q), fb);
-        st_half8(Tbe, swz(i, qt * 2 + q), fe);
+        st_half8(Tb, swz(i, qt), fb);
+        st_half8(Tbe, swz(i, qt), fe);
       }
     }
     fence_proxy_async();
@@ -480,14 +490,14 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     GDN_PHASE(4);
 
-    // ---- -W^T as the MN-major B operand (row l = tl, tokens wg*32 .. wg*32+31)
+    // ---- -W^T as the MN-major B operand (row l = tl, tokens wg*CW .. wg*CW+CW-1)
     {
-      float x[32];
-      tmem_ld32(lane_base + TM_D3 + wg * 32, x);
+      float x[CW];
+      tmem_ld16(lane_base + TM_D3 + wg * CW, x);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = -x[j];
+      for (int j = 0; j < CW; ++j) x[j] = -x[j];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(wt_ptr, swz(tl, wg * 4 + q), x + q * 8);
+      for (int q = 0; q < CW / 8; ++q) st_half8(wt_ptr, swz(tl, wg * (CW / 8) + q), x + q * 8);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -520,20 +530,20 @@ __global__ void __launch_bounds__(NT, 1)
 
     // ---- Vn^T rows: plain (A of D5) and decayed to the chunk end (A of the state update)
     {
-      float x[32];
-      tmem_ld32(lane_base + TM_D2 + wg * 32, x);
+      float x[CW];
+      tmem_ld16(lane_base + TM_D2 + wg * CW, x);
       uint8_t* Vt = smem + OFF_TB;
       uint8_t* Vts = smem + OFF_VTS;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < CW / 8; ++q) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int i = wg * 32 + q * 8 + e;
+          const int i = wg * CW + q * 8 + e;
           f[e] = i < L ? x[q * 8 + e] * decL[i] : 0.f;
         }
-        st_half8(Vt, swz(tl, wg * 4 + q), x + q * 8);
-        st_half8(Vts, swz(tl, wg * 4 + q), f);
+        st_half8(Vt, swz(tl, wg * (CW / 8) + q), x + q * 8);
+        st_half8(Vts, swz(tl, wg * (CW / 8) + q), f);
       }
     }
     fence_proxy_async();
@@ -557,28 +567,28 @@ __global__ void __launch_bounds__(NT, 1)
       }
       mma_commit(bar_o);
     }
-    // meanwhile: w * silu(z) for this thread's outputs (column tl, tokens wg*32 .. wg*32+31)
-    float zw[32];
+    // meanwhile: w * silu(z) for this thread's outputs (column tl, tokens wg*CW .. wg*CW+CW-1)
+    float zw[CW];
     if (norm_out) {
       ok = mbar_wait(bar_z, par);
       const __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) zw[j] = w_norm * silu_f(__bfloat162float(zcol[(wg * 32 + j) * 64]));
+      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_f(__bfloat162float(zcol[(wg * CW + j) * 64]));
     }
     ok = mbar_wait(bar_o, par) && ok;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     GDN_PHASE(6);
 
-    // ---- epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*32 .. +31, staged as O [token][v]
-    float o[32];
+    // ---- epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*CW .. +CW-1, staged as O [token][v]
+    float o[CW];
     {
-      float a5[32];
-      tmem_ld32(lane_base + TM_D4 + wg * 32, o);
-      tmem_ld32(lane_base + TM_D5 + wg * 32, a5);
+      float a5[CW];
+      tmem_ld16(lane_base + TM_D4 + wg * CW, o);
+      tmem_ld16(lane_base + TM_D5 + wg * CW, a5);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int i = wg * 32 + j;
+      for (int j = 0; j < CW; ++j) {
+        const int i = wg * CW + j;
         o[j] = fmaf(eg[i], o[j], a5[j]);
         Os[i * D + tl] = o[j];
       }
@@ -586,25 +596,26 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     GDN_PHASE(7);
     if (norm_out) {
-      // 1 / rms per token: warp w reduces tokens 8w .. 8w+7
-      float ss[8];
+      // 1 / rms per token: warp w reduces tokens TPW*w .. TPW*w+TPW-1
+      constexpr int TPW = 64 / NW;
+      float ss[TPW];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const float* row = Os + (8 * warp + t) * D;
+      for (int t = 0; t < TPW; ++t) {
+        const float* row = Os + (TPW * warp + t) * D;
         const float o0 = row[lane], o1 = row[lane + 32], o2 = row[lane + 64], o3 = row[lane + 96];
         ss[t] = o0 * o0 + o1 * o1 + o2 * o2 + o3 * o3;
       }
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ss[t] = warp_sum(ss[t]);
+      for (int t = 0; t < TPW; ++t) ss[t] = warp_sum(ss[t]);
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
-        if (lane == t) rms[8 * warp + t] = rsqrtf(ss[t] * (1.0f / D) + p.eps_norm);
+      for (int t = 0; t < TPW; ++t)
+        if (lane == t) rms[TPW * warp + t] = rsqrtf(ss[t] * (1.0f / D) + p.eps_norm);
       __syncthreads();
       // gated output, written over the z tile (each element read, then written, by one thread)
       __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int i = wg * 32 + j;
+      for (int j = 0; j < CW; ++j) {
+        const int i = wg * CW + j;
         zcol[i * 64] = __float2bfloat16_rn(o[j] * rms[i] * zw[j]);
       }
       fence_proxy_async();  // the next chunk's z tile lands here through TMA
@@ -613,7 +624,7 @@ __global__ void __launch_bounds__(NT, 1)
       uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv + h) * D * 2;
       const size_t ostride = (size_t)p.Hv * D * 2;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 1024 / NT; ++k) {
         const int e = tid + NT * k, row = e >> 4, c16 = e & 15;
         if (row < L) {
           const uint4 val = *reinterpret_cast<const uint4*>(smem + OFF_Z + (c16 >> 3) * TILE_BYTES +
@@ -625,8 +636,8 @@ __global__ void __launch_bounds__(NT, 1)
       float* ocol = p.o_raw + ((size_t)c0 * p.Hv + h) * D + tl;
       const size_t ostride = (size_t)p.Hv * D;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int i = wg * 32 + j;
+      for (int j = 0; j < CW; ++j) {
+        const int i = wg * CW + j;
         if (i < L) ocol[i * ostride] = o[j];
       }
     }
@@ -647,15 +658,12 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (p.S_out) {
     float r[32];
+    const int col = wg * SW;
+    tmem_ld32(lane_base + TM_S + col, r);
 #pragma unroll
-    for (int piece = 0; piece < 2; ++piece) {
-      const int col = wg * 64 + piece * 32;
-      tmem_ld32(lane_base + TM_S + col, r);
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(p.S_out + sbase + (size_t)tl * D + col + j) =
-            make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
-    }
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(p.S_out + sbase + (size_t)tl * D + col + j) =
+          make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
   }
   tc_fence_before();
   __syncthreads();
