@@ -83,7 +83,8 @@ class PrefillBuffers:
         self.out = torch.empty((dp.T, dp.Hv, dp.d), dtype=dp.dtype, device=dev)
         self.final_state = torch.empty((dp.N, dp.Hv, dp.d, dp.d), dtype=torch.float32, device=dev)
         self.conv_state_out = torch.empty((dp.N, dp.Cc, 3), dtype=dp.dtype, device=dev)
-        self.ws_bytes = gdn.gdn_prefill_workspace_size(self.dims, dp.T, self.dtype_code)
+        # room for every path, including the two-kernel tensor-core one
+        self.ws_bytes = gdn.gdn_prefill_workspace_size_n(self.dims, dp.N, dp.T, self.dtype_code)
         self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
 
 

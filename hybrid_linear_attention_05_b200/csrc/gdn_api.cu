@@ -37,10 +37,12 @@ gdn_dtype mid_dtype(gdn_dtype in) { return in == GDN_BF16 ? GDN_F16 : GDN_F32; }
 
 struct Workspace {
   void* q; void* k; void* v; float* g; float* beta;
+  uint8_t* rec;  // operand records of the two-kernel tensor-core path (or null)
   size_t bytes;
 };
 
-Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base) {
+// Workspace layout; with N >= 0 it also holds the two-kernel path's records.
+Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base, int N = -1) {
   Workspace w{};
   const size_t e = esize(dt);
   const size_t nq = align_up((size_t)T * d->Hk * d->dk * e, 256);
@@ -53,19 +55,27 @@ Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base) {
   w.v = p ? p + off : nullptr; off += nv;
   w.g = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
   w.beta = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
+  w.rec = nullptr;
+  if (N >= 0) {
+    w.rec = p ? reinterpret_cast<uint8_t*>(p + off) : nullptr;
+    off += align_up(chunk_tc_split_record_bytes(N, T, d->Hv), 256);
+  }
   w.bytes = off;
   return w;
 }
 
-enum class Path { None, Simt, Tc };
+enum class Path { None, Simt, Tc, TcSplit };
 
-Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid) {
+// `records` tells whether the workspace can hold the two-kernel path's records.
+Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records) {
   const bool tc = chunk_tc_supported(d, chunk, dt_mid);
   const bool simt = chunk_simt_supported(d, chunk);
   switch (impl) {
     case GDN_IMPL_TC: return tc ? Path::Tc : Path::None;
+    case GDN_IMPL_TC_SPLIT: return tc ? Path::TcSplit : Path::None;
     case GDN_IMPL_SIMT: return simt ? Path::Simt : Path::None;
-    case GDN_IMPL_AUTO: return tc ? Path::Tc : (simt ? Path::Simt : Path::None);
+    case GDN_IMPL_AUTO:
+      return tc ? (records ? Path::TcSplit : Path::Tc) : (simt ? Path::Simt : Path::None);
   }
   return Path::None;
 }
@@ -81,6 +91,11 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dty
   return carve(dims, T_tot, dtype, nullptr).bytes;
 }
 
+size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_dtype dtype) {
+  if (check_dims(dims) != GDN_OK || T_tot < 0 || N < 0 || !dtype_ok(dtype)) return 0;
+  return carve(dims, T_tot, dtype, nullptr, N).bytes;
+}
+
 gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* stream) {
   gdn_status s = check_dims(dims);
   if (s != GDN_OK) return s;
@@ -91,8 +106,11 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
   const int Cc = 2 * dims->Hk * d + dims->Hv * d;
-  const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype));
+  const size_t full = carve(dims, a->T_tot, a->dtype, nullptr, a->N).bytes;
+  const bool records = a->workspace && a->workspace_bytes >= full;
+  const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype), records);
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
+  if (path == Path::TcSplit && !records) return GDN_ERR_WORKSPACE;
   if (!a->cu_seqlens || !a->conv_w || !a->A_log || !a->dt_bias || !a->norm_w) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->mixed_qkv || !a->a || !a->b || !a->z || !a->out || !a->workspace))
     return GDN_ERR_NULL;
@@ -110,7 +128,7 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
     return GDN_ERR_ALIAS;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Workspace ws = carve(dims, a->T_tot, a->dtype, a->workspace);
+  const Workspace ws = carve(dims, a->T_tot, a->dtype, a->workspace, path == Path::TcSplit ? a->N : -1);
 
   ConvPrepParams cp{};
   cp.x = a->mixed_qkv; cp.conv_w = a->conv_w; cp.a = a->a; cp.b = a->b;
@@ -128,10 +146,12 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   ch.z = a->z; ch.norm_w = a->norm_w; ch.out = a->out; ch.o_raw = nullptr;
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
   ch.eps_norm = dims->eps_norm;
+  ch.rec = ws.rec;
   if (a->core_event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_begin), st) != cudaSuccess)
     return GDN_ERR_CUDA;
-  s = from_cuda(path == Path::Tc ? launch_chunk_tc(ch, st)
-                                 : launch_chunk_simt(ch, d, a->dtype, mid_dtype(a->dtype), st));
+  s = from_cuda(path == Path::TcSplit ? launch_chunk_tc_split(ch, st)
+                : path == Path::Tc    ? launch_chunk_tc(ch, st)
+                                      : launch_chunk_simt(ch, d, a->dtype, mid_dtype(a->dtype), st));
   if (s != GDN_OK) return s;
   if (a->core_event_end && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_end), st) != cudaSuccess)
     return GDN_ERR_CUDA;
@@ -169,7 +189,8 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
-  const Path path = pick_path(a->impl, d, a->chunk, a->dtype);
+  // no workspace here, hence no two-kernel path
+  const Path path = a->impl == GDN_IMPL_TC_SPLIT ? Path::None : pick_path(a->impl, d, a->chunk, a->dtype, false);
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
   if (!a->cu_seqlens) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o)) return GDN_ERR_NULL;

@@ -50,6 +50,7 @@ struct ChunkParams {
   float* o_raw;               // [T, Hv, d] fp32 core output (when out == null)
   int T, N, Hk, Hv, chunk;
   float eps_norm;
+  uint8_t* rec;               // split tensor-core path: per-(chunk, head) operand records
 };
 
 // chunk_simt.cu: fp32 CUDA-core chunked core.  Supported (d, chunk) pairs:
@@ -63,6 +64,13 @@ cudaError_t launch_chunk_simt(const ChunkParams& p, int d, gdn_dtype dt_out, gdn
 // dt_mid = GDN_F16), d = 128, chunk = 64.
 bool chunk_tc_supported(int d, int chunk, gdn_dtype dt_mid);
 cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st);
+
+// chunk_tc_split.cu: the same core as two kernels -- a key-side kernel over
+// every (chunk, value head) writing operand records, then a per-head chain
+// kernel.  Needs chunk_tc_split_record_bytes(...) of extra workspace.
+size_t chunk_tc_split_record_bytes(int N, int T, int Hv);
+cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st);
+int split_error_word(int clear);  // host: read (and clear) that path's device error word
 
 // decode.cu
 struct DecodeParams {

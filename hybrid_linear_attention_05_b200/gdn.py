@@ -31,8 +31,9 @@ GDN_F16 = 2
 GDN_IMPL_AUTO = 0
 GDN_IMPL_SIMT = 1
 GDN_IMPL_TC = 2
+GDN_IMPL_TC_SPLIT = 3
 
-EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_noalloc", "gdn_decode",
+EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill", "gdn_prefill_noalloc", "gdn_decode",
             "gdn_chunk_core", "gdn_device_error", "gdn_status_string", "gdn_version"]
 
 # Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
@@ -86,6 +87,9 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         L.gdn_prefill_workspace_size.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
         L.gdn_prefill_workspace_size.restype = ctypes.c_size_t
+        L.gdn_prefill_workspace_size_n.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int]
+        L.gdn_prefill_workspace_size_n.restype = ctypes.c_size_t
         L.gdn_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args), _vp]
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_prefill_noalloc.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
@@ -154,6 +158,10 @@ def _check(status, where, raise_on_error):
 
 def gdn_prefill_workspace_size(dims: gdn_dims, T_tot: int, dtype: int) -> int:
     return int(lib().gdn_prefill_workspace_size(ctypes.byref(dims), int(T_tot), int(dtype)))
+
+
+def gdn_prefill_workspace_size_n(dims: gdn_dims, N: int, T_tot: int, dtype: int) -> int:
+    return int(lib().gdn_prefill_workspace_size_n(ctypes.byref(dims), int(N), int(T_tot), int(dtype)))
 
 
 def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,

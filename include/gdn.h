@@ -84,9 +84,14 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype;
 typedef enum {
   GDN_IMPL_AUTO = 0,   /* tensor cores when supported, else CUDA cores        */
   GDN_IMPL_SIMT = 1,   /* fp32 CUDA-core chunked kernel                       */
-  GDN_IMPL_TC = 2      /* tcgen05 tensor-core chunked kernel (bf16 inputs,
-                          fp16 operands, d = 128, chunk 64);
+  GDN_IMPL_TC = 2,     /* tcgen05 tensor-core chunked core, one kernel per call
+                          (bf16 inputs, fp16 operands, d = 128, chunk 64);
                           GDN_ERR_UNSUPPORTED otherwise                       */
+  GDN_IMPL_TC_SPLIT = 3 /* the same tensor-core core as two kernels: the
+                          state-independent key-side work of every (chunk,
+                          head) first, over all SMs, then the per-head state
+                          chain.  Needs gdn_prefill_workspace_size_n bytes
+                          of workspace (GDN_ERR_WORKSPACE otherwise).         */
 } gdn_impl;
 
 /* Layer shape.  Supported: dk == dv in {32, 64, 128}; Hv % Hk == 0;
@@ -142,6 +147,14 @@ typedef struct {
  * (fp16 for bf16 inputs, fp32 for fp32 inputs) and the gates of every token
  * between the two kernels of the call. */
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dtype);
+
+/* Bytes of workspace that also holds the per-(chunk, value head) operand
+ * records of the two-kernel tensor-core path (GDN_IMPL_TC_SPLIT): about
+ * 33 KB per 64 tokens and value head, for N sequences of T_tot tokens in
+ * total.  With at least this much, GDN_IMPL_AUTO takes the two-kernel path
+ * where the tensor cores apply; with only gdn_prefill_workspace_size bytes it
+ * takes the single-kernel one.  0 when the sizes are invalid. */
+size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_dtype dtype);
 
 /* Steps 1-5 over packed sequences.  Writes out, and final_state /
  * conv_state_out when given.  The workspace is overwritten. */

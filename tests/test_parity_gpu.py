@@ -35,7 +35,8 @@ P9B = WORKLOADS["prefill_4x8192_Hk16_Hv32_d128"]
 D9B = WORKLOADS["decode_B256_Hk16_Hv32_d128"]
 P397 = WORKLOADS["prefill_varlen8_T65536_Hk16_Hv64_d128"]
 
-IMPLS = {"simt": (gdn.GDN_IMPL_SIMT, 32), "tc": (gdn.GDN_IMPL_TC, 64)}
+IMPLS = {"simt": (gdn.GDN_IMPL_SIMT, 32), "tc": (gdn.GDN_IMPL_TC, 64),
+         "split": (gdn.GDN_IMPL_TC_SPLIT, 64)}
 
 
 def np64(t):
@@ -102,7 +103,7 @@ def test_simt_small_heads(chunk, d):
     check_full(inp, bufs)
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
 def test_qwen08b_shapes_ragged(impl):
     """16/16 heads of width 128 over several chunks with a ragged tail."""
     code, chunk = IMPLS[impl]
@@ -111,7 +112,7 @@ def test_qwen08b_shapes_ragged(impl):
     check_full(inp, bufs)
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
 def test_9b_shapes_gqa_varlen(impl):
     """16 key / 32 value heads, nonzero initial states, conv history,
     sequences of lengths 1, 2, 3, 64 and one spanning several chunks."""
@@ -121,7 +122,7 @@ def test_9b_shapes_gqa_varlen(impl):
     check_full(inp, bufs)
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
 def test_397b_shapes_varlen(impl):
     code, chunk = IMPLS[impl]
     inp = make_prefill(P397, seqlens=(65, 130, 7, 64))
@@ -168,12 +169,15 @@ def sampled_check(inp, bufs, pairs):
     ("prefill_4x8192_Hk16_Hv32_d128", [(0, 0), (1, 13), (3, 31)]),
     ("prefill_varlen8_T65536_Hk16_Hv64_d128", [(0, 0), (3, 21), (7, 63)]),
 ])
-def test_full_size_sampled(name, pairs):
-    """Full benchmark sizes in the benchmark's launch configuration; the
-    oracle recomputes a few (sequence, value head) pairs on their own."""
+@pytest.mark.parametrize("impl", ["auto", "tc"])
+def test_full_size_sampled(name, pairs, impl):
+    """Full benchmark sizes in the benchmark's launch configuration (AUTO:
+    the two-kernel tensor-core path), and the single-kernel path; the oracle
+    recomputes a few (sequence, value head) pairs on their own."""
     w = WORKLOADS[name]
     inp = make_prefill(w)
-    bufs = run_prefill(inp, gdn.GDN_IMPL_AUTO, w.chunk, guard=False)
+    code = gdn.GDN_IMPL_AUTO if impl == "auto" else gdn.GDN_IMPL_TC
+    bufs = run_prefill(inp, code, w.chunk, guard=False)
     sampled_check(inp, bufs, pairs)
     assert torch.isfinite(bufs.out.float()).all()
 
