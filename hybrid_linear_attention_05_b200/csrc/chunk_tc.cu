@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(NT, 1)
       ok = mbar_wait(bar_z, par);
       const __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE_BYTES / 2) + (tl & 63);
 #pragma unroll
-      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_f(__bfloat162float(zcol[(wg * CW + j) * 64]));
+      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_tanh(__bfloat162float(zcol[(wg * CW + j) * 64]));
     }
     ok = mbar_wait(bar_o, par) && ok;
     if (__syncthreads_or(!ok)) break;

@@ -34,6 +34,24 @@ namespace gdn {
 
 __device__ int g_split_error = 0;  // nonzero: a bounded wait in a kernel of this file gave up
 
+#ifdef GDN_PHASE_TIMING
+// Development aid (off by default): SM cycles spent by chain-kernel thread 0
+// in each phase of the chunk loop, summed over all CTAs.
+__device__ unsigned long long g_split_phase[16];
+#define GDN_SPLIT_PHASE(k)                                              \
+  do {                                                                  \
+    if (tid == 0) {                                                     \
+      const long long t_ = clock64();                                   \
+      atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
+      t_prev = t_;                                                      \
+    }                                                                   \
+  } while (0)
+#else
+#define GDN_SPLIT_PHASE(k) \
+  do {                     \
+  } while (0)
+#endif
+
 namespace {
 
 using namespace ptx;
@@ -155,11 +173,11 @@ __global__ void __launch_bounds__(NTA, 2)
     if (tid == 0) {  // D1 = [K; Q] K^T
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, false, false);
+      const uint64_t dkq = sdesc_sw128(sb + A_KQ, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + A_TM_D1, sdesc_sw128(sb + A_KQ + off, 16, 1024),
-                sdesc_sw128(sb + A_KQ + off, 16, 1024), id, kk > 0);
+        mma_f16(tmem + A_TM_D1, sdesc_add(dkq, off), sdesc_add(dkq, off), id, kk > 0);
       }
       mma_commit(bar_m1);
     }
@@ -240,10 +258,10 @@ __global__ void __launch_bounds__(NTA, 2)
     if (tid == 0) {  // D3 = K^T Tbe^T = W^T
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, true, false);
+      const uint64_t dk = sdesc_sw128(sb + A_KQ, 16384, 1024), dt = sdesc_sw128(sb + A_TBE, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + A_TM_D3, sdesc_sw128(sb + A_KQ + kk * 2048, 16384, 1024),
-                sdesc_sw128(sb + A_TBE + kk * 32, 16, 1024), id, kk > 0);
+        mma_f16(tmem + A_TM_D3, sdesc_add(dk, kk * 2048), sdesc_add(dt, kk * 32), id, kk > 0);
       mma_commit(bar_w);
     }
     ok = mbar_wait(bar_w, 0);
@@ -348,7 +366,8 @@ __global__ void __launch_bounds__(NTB, 1)
     tma_load_2d(st + B_V + 8192, &tm_v, h * D + 64, row, bar);
     bulk_load(st + B_REC, p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC, REC, bar);
   };
-  if (tid == 0) issue_loads(0, 0);
+  constexpr int LOADER = 32;  // one lane of warp 1 issues the copies (thread 0 issues the MMAs)
+  if (tid == LOADER) issue_loads(0, 0);
   const float w_norm = norm_out ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tl]) : 0.f;
 
   // initial state -> TMEM (row tl, columns wg*SW .. wg*SW+SW-1)
@@ -367,6 +386,9 @@ __global__ void __launch_bounds__(NTB, 1)
 
   bool ok = true;
   int c = 0;
+#ifdef GDN_PHASE_TIMING
+  long long t_prev = clock64();
+#endif
   for (; c < nchunks; ++c) {
     const int s = c & 1;
     const int c0 = bos + c * C;
@@ -376,7 +398,7 @@ __global__ void __launch_bounds__(NTB, 1)
     uint8_t* stp = smem + s * B_STAGE;
     const float* vec = reinterpret_cast<const float*>(stp + B_REC + R_VEC);  // e^gamma, decay to end
 
-    if (tid == 0) {
+    if (tid == LOADER) {
       if (c + 1 < nchunks) issue_loads(c + 1, s ^ 1);
       if (norm_out) {
         mbar_arrive_expect_tx(bar_z, 2 * TILE);
@@ -387,15 +409,16 @@ __global__ void __launch_bounds__(NTB, 1)
     if (tid < 64) ss[tid] = 0.f;
     ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
     if (__syncthreads_or(!ok)) break;
+    GDN_SPLIT_PHASE(0);
 
     // D2 = V^T (T diag beta)^T  (= U^T); needs no state
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, true, false);
+      const uint64_t dv = sdesc_sw128(st + B_V, 8192, 1024), dt = sdesc_sw128(st + B_REC + R_TB, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_D2, sdesc_sw128(st + B_V + kk * 2048, 8192, 1024),
-                sdesc_sw128(st + B_REC + R_TB + kk * 32, 16, 1024), id, kk > 0);
+        mma_f16(tmem + B_TM_D2, sdesc_add(dv, kk * 2048), sdesc_add(dt, kk * 32), id, kk > 0);
     }
     // meanwhile: state -> fp16 operand, then S *= e^{gamma_L} in TMEM
     {
@@ -416,27 +439,30 @@ __global__ void __launch_bounds__(NTB, 1)
     __syncthreads();
 
     // D2 += S (-W^T)  (= Vn^T), committed alone; then D4 = S Q^T
+    GDN_SPLIT_PHASE(1);
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id_w = idesc_f16(128, 64, false, true);
       constexpr uint32_t id_q = idesc_f16(128, 64, false, false);
+      const uint64_t ds = sdesc_sw128(sb + B_S16, 16, 1024);
+      const uint64_t dw = sdesc_sw128(st + B_REC + R_WT, 16384, 1024);
+      const uint64_t dq = sdesc_sw128(st + B_KQ + 8192, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + B_TM_D2, sdesc_sw128(sb + B_S16 + aoff, 16, 1024),
-                sdesc_sw128(st + B_REC + R_WT + kk * 2048, 16384, 1024), id_w, 1);
+        mma_f16(tmem + B_TM_D2, sdesc_add(ds, aoff), sdesc_add(dw, kk * 2048), id_w, 1);
       }
       mma_commit(bar_v);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + B_TM_D4, sdesc_sw128(sb + B_S16 + aoff, 16, 1024),
-                sdesc_sw128(st + B_KQ + aoff + 8192, 16, 1024), id_q, kk > 0);
+        mma_f16(tmem + B_TM_D4, sdesc_add(ds, aoff), sdesc_add(dq, aoff), id_q, kk > 0);
       }
     }
     ok = mbar_wait(bar_v, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_SPLIT_PHASE(2);
 
     // Vn^T rows: plain (A of D5, over the consumed -W^T image) and decayed to the chunk end
     // (A of the state update, over the consumed V tile)
@@ -460,18 +486,19 @@ __global__ void __launch_bounds__(NTB, 1)
     __syncthreads();
 
     // S += Vts K,  D5 = Vn^T P^T
+    GDN_SPLIT_PHASE(3);
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id_s = idesc_f16(128, 128, false, true);
       constexpr uint32_t id_p = idesc_f16(128, 64, false, false);
+      const uint64_t dvs = sdesc_sw128(st + B_V, 16, 1024), dk = sdesc_sw128(st + B_KQ, 16384, 1024);
+      const uint64_t dvt = sdesc_sw128(st + B_REC + R_WT, 16, 1024), dp = sdesc_sw128(st + B_REC + R_P, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_S, sdesc_sw128(st + B_V + kk * 32, 16, 1024),
-                sdesc_sw128(st + B_KQ + kk * 2048, 16384, 1024), id_s, 1);
+        mma_f16(tmem + B_TM_S, sdesc_add(dvs, kk * 32), sdesc_add(dk, kk * 2048), id_s, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_D5, sdesc_sw128(st + B_REC + R_WT + kk * 32, 16, 1024),
-                sdesc_sw128(st + B_REC + R_P + kk * 32, 16, 1024), id_p, kk > 0);
+        mma_f16(tmem + B_TM_D5, sdesc_add(dvt, kk * 32), sdesc_add(dp, kk * 32), id_p, kk > 0);
       mma_commit(bar_o);
     }
     // meanwhile: w * silu(z) for this thread's outputs (column tl, tokens wg*CW ..)
@@ -480,11 +507,12 @@ __global__ void __launch_bounds__(NTB, 1)
       ok = mbar_wait(bar_z, par);
       const __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE / 2) + (tl & 63);
 #pragma unroll
-      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_f(__bfloat162float(zcol[(wg * CW + j) * 64]));
+      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_tanh(__bfloat162float(zcol[(wg * CW + j) * 64]));
     }
     ok = mbar_wait(bar_o, par) && ok;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
+    GDN_SPLIT_PHASE(4);
 
     // epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*CW .. wg*CW+CW-1
     float o[CW];
@@ -515,12 +543,15 @@ __global__ void __launch_bounds__(NTB, 1)
       const int t = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
       if ((lane & 1) == 0) atomicAdd(&ss[wg * CW + t], a[0]);
       __syncthreads();
+      if (tid < 64) ss[tid] = rsqrtf(ss[tid] * (1.0f / D) + p.eps_norm);  // now 1 / rms
+      __syncthreads();
+    GDN_SPLIT_PHASE(5);
       // gated output, written over the z tile (each element read, then written, by one thread)
       __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE / 2) + (tl & 63);
 #pragma unroll
       for (int j = 0; j < CW; ++j) {
         const int i = wg * CW + j;
-        zcol[i * 64] = __float2bfloat16_rn(o[j] * rsqrtf(ss[i] * (1.0f / D) + p.eps_norm) * zw[j]);
+        zcol[i * 64] = __float2bfloat16_rn(o[j] * ss[i] * zw[j]);
       }
       fence_proxy_async();  // the next chunk's z tile lands here through TMA
       __syncthreads();
@@ -545,6 +576,7 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
     __syncthreads();
+    GDN_SPLIT_PHASE(6);
   }
 
   if (!ok) {
@@ -646,6 +678,18 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st) {
   chunk_chain_kernel<<<gb, NTB, B_SMEM, st>>>(mq, mk, mv, mz, p);
   return cudaGetLastError();
 }
+
+#ifdef GDN_PHASE_TIMING
+extern "C" int gdn_debug_phase_cycles_split(unsigned long long* out, int clear) {
+  cudaDeviceSynchronize();
+  if (cudaMemcpyFromSymbol(out, g_split_phase, sizeof(unsigned long long) * 16) != cudaSuccess) return -1;
+  if (clear) {
+    unsigned long long z[16] = {0};
+    cudaMemcpyToSymbol(g_split_phase, z, sizeof(z));
+  }
+  return 0;
+}
+#endif
 
 int split_error_word(int clear) {
   int v = 0;

@@ -5,29 +5,32 @@
 // core, and fp16 keeps three more significand bits than bf16 at the same size
 // and MMA rate (all of them are bounded: |q|, |k| <= 1 after the norm).
 //
-// One thread handles 8 consecutive channels of one token: it reads the four
-// conv inputs of those channels (the token and the three before it, or the
-// sequence's conv history before its first token), applies the depthwise
-// 4-tap conv and SiLU, and for q / k heads joins the other threads of its
-// head in a shuffle reduction for the L2 norm.  The first thread of every
+// One thread handles 8 consecutive channels of TPT consecutive tokens: it
+// keeps the conv window of those channels in registers (the three previous
+// inputs, or the sequence's conv history before its first token), applies
+// the depthwise 4-tap conv and SiLU token by token, and for q / k heads joins
+// the other threads of its head in a shuffle reduction for the L2 norm.  The first thread of every
 // value head also computes that head's gates g = -exp(A_log) softplus(a +
 // dt_bias) and beta = sigmoid(b).  A second group of threads writes the conv
 // tail (the last three raw inputs of every sequence).
 //
-// HBM traffic per token: the Cc-wide input row once (the three earlier rows
-// it also reads are the previous tokens' rows, served from L1/L2), the
+// HBM traffic per token: the Cc-wide input row once (the three rows before a
+// thread's first token are the previous thread's rows, served from L2), the
 // Cc-wide normalised row once, and the gates.
 #include "gdn_internal.h"
 
 namespace gdn {
 
+constexpr int TPT = 4;  // consecutive tokens per thread (sliding conv window)
+
 template <typename T, typename TM, int D>
 __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
   constexpr int TPS = D / 8;  // threads per head segment
   const int Cc = p.Cc;
-  const int groups = Cc / 8;  // threads per token row
+  const int groups = Cc / 8;  // threads per block of TPT tokens
   const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const size_t n_tok = (size_t)p.T * groups;
+  const int n_blocks_tok = (p.T + TPT - 1) / TPT;
+  const size_t n_tok = (size_t)n_blocks_tok * groups;
   const T* __restrict__ x = static_cast<const T*>(p.x);
   const T* __restrict__ hist_all = static_cast<const T*>(p.conv_state_in);
   const int lane = threadIdx.x & 31;
@@ -35,14 +38,17 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
 
   if (blockIdx.x < p.tok_blocks) {
     // ------------------------------------------------------ token threads
+    // This thread: channels c0 .. c0+7 of tokens t0 .. t0+TPT-1.  Segments
+    // (the TPS threads of one head) share t0, so their shuffles line up.
     const bool valid = gid < n_tok;
-    const int t = valid ? (int)(gid / groups) : 0;
+    const int tb = valid ? (int)(gid / groups) : 0;
     const int cg = valid ? (int)(gid % groups) : 0;
     const int c0 = cg * 8;
     const int seg = c0 / D;
-    const int n = seq_of_token(p.cu_seqlens, p.N, t);
-    const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
-    const T* hist = hist_all ? hist_all + (size_t)n * Cc * 3 : nullptr;
+    const int t0 = tb * TPT;
+    const int two_hk = 2 * p.Hk;
+    const bool is_qk = seg < two_hk;
+    const bool is_q = seg < p.Hk;
 
     float w[8][4];
     {
@@ -55,55 +61,86 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
         for (int i = 0; i < 8; ++i) w[(r * 8 + i) / 4][(r * 8 + i) % 4] = tmp[i];
       }
     }
-    float y[8];
+    // the TPT new input rows, issued together
+    float xr[TPT][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = 0.0f;
+    for (int k = 0; k < TPT; ++k) {
+      const int t = min(t0 + k, p.T - 1);
+      load8(x + (size_t)t * Cc + c0, xr[k]);
+    }
+    // conv window before token t0 (positions t0-3 .. t0-1) of t0's sequence
+    int n = seq_of_token(p.cu_seqlens, p.N, min(t0, p.T - 1));
+    int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
+    int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
+    float win[3][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int tau = t - 3 + j;
-      float xv[8];
+    for (int j = 0; j < 3; ++j) {
+      const int tau = t0 - 3 + j;
       if (tau >= bos) {
-        load8(x + (size_t)tau * Cc + c0, xv);
-      } else if (hist) {
-        const int hidx = 3 - (bos - tau);  // 0..2, oldest first
+        load8(x + (size_t)tau * Cc + c0, win[j]);
+      } else if (hist_all) {
+        const T* hist = hist_all + (size_t)n * Cc * 3;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xv[i] = ld_f(hist + (size_t)(c0 + i) * 3 + hidx);
+        for (int i = 0; i < 8; ++i) win[j][i] = ld_f(hist + (size_t)(c0 + i) * 3 + (3 - (bos - tau)));
       } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xv[i] = 0.0f;
+        for (int i = 0; i < 8; ++i) win[j][i] = 0.f;
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = fmaf(w[i][j], xv[i], y[i]);
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = silu_f(y[i]);
 
-    const int two_hk = 2 * p.Hk;
-    if (seg < two_hk) {
-      float ss = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(y[i], y[i], ss);
+    for (int k = 0; k < TPT; ++k) {
+      const int t = t0 + k;
+      if (t >= p.T) break;  // the whole segment shares t: no divergent shuffle
+      if (t >= eos) {
+        // first token of a later sequence: its window is that sequence's history
+        while (n + 1 < p.N && t >= __ldg(p.cu_seqlens + n + 1)) ++n;
+        bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
+        eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
+        const T* hist = hist_all ? hist_all + (size_t)n * Cc * 3 : nullptr;
 #pragma unroll
-      for (int o = TPS / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(seg_mask, ss, o, 32);
-      const bool is_q = seg < p.Hk;
-      const float r = rsqrtf(ss + p.eps_l2) * (is_q ? p.scale : 1.0f);
+        for (int j = 0; j < 3; ++j)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] *= r;
-      if (valid) {
-        TM* dst = static_cast<TM*>(is_q ? p.q : p.k);
-        const int col = c0 - (is_q ? 0 : p.Hk * D);
-        store8(dst + (size_t)t * p.Hk * D + col, y);
+          for (int i = 0; i < 8; ++i)
+            win[j][i] = hist ? ld_f(hist + (size_t)(c0 + i) * 3 + j) : 0.f;
       }
-    } else if (valid) {
-      const int col = c0 - two_hk * D;
-      store8(static_cast<TM*>(p.v) + (size_t)t * p.Hv * D + col, y);
-      if ((c0 % D) == 0) {
-        const int h = seg - two_hk;
-        const float av = ld_f(static_cast<const T*>(p.a) + (size_t)t * p.Hv + h);
-        const float bv = ld_f(static_cast<const T*>(p.b) + (size_t)t * p.Hv + h);
-        const float gg = -expf(__ldg(p.A_log + h)) * softplus_f(av + __ldg(p.dt_bias + h));
-        p.g[(size_t)h * p.T + t] = gg;
-        p.beta[(size_t)h * p.T + t] = sigmoid_f(bv);
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float acc = w[i][0] * win[0][i];
+        acc = fmaf(w[i][1], win[1][i], acc);
+        acc = fmaf(w[i][2], win[2][i], acc);
+        acc = fmaf(w[i][3], xr[k][i], acc);
+        y[i] = silu_f(acc);
+        win[0][i] = win[1][i];
+        win[1][i] = win[2][i];
+        win[2][i] = xr[k][i];
+      }
+      if (is_qk) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(y[i], y[i], ss);
+#pragma unroll
+        for (int o = TPS / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(seg_mask, ss, o, 32);
+        const float r = rsqrtf(ss + p.eps_l2) * (is_q ? p.scale : 1.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] *= r;
+        if (valid) {
+          TM* dst = static_cast<TM*>(is_q ? p.q : p.k);
+          const int col = c0 - (is_q ? 0 : p.Hk * D);
+          store8(dst + (size_t)t * p.Hk * D + col, y);
+        }
+      } else if (valid) {
+        const int col = c0 - two_hk * D;
+        store8(static_cast<TM*>(p.v) + (size_t)t * p.Hv * D + col, y);
+        if ((c0 % D) == 0) {
+          const int hh = seg - two_hk;
+          const float av = ld_f(static_cast<const T*>(p.a) + (size_t)t * p.Hv + hh);
+          const float bv = ld_f(static_cast<const T*>(p.b) + (size_t)t * p.Hv + hh);
+          const float gg = -expf(__ldg(p.A_log + hh)) * softplus_f(av + __ldg(p.dt_bias + hh));
+          p.g[(size_t)hh * p.T + t] = gg;
+          p.beta[(size_t)hh * p.T + t] = sigmoid_f(bv);
+        }
       }
     }
   } else {
@@ -140,7 +177,7 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
 cudaError_t launch_conv_prep(const ConvPrepParams& p0, int d, gdn_dtype dt, cudaStream_t st) {
   ConvPrepParams p = p0;
   const int groups = p.Cc / 8;
-  const size_t n_tok = (size_t)p.T * groups;
+  const size_t n_tok = (size_t)((p.T + TPT - 1) / TPT) * groups;
   const size_t n_tail = (size_t)p.N * groups;
   p.tok_blocks = (int)((n_tok + 255) / 256);
   const int tail_blocks = (int)((n_tail + 255) / 256);

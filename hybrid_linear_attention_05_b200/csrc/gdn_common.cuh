@@ -79,6 +79,13 @@ __device__ __forceinline__ void store8(float* p, const float* f) {
 // ------------------------------------------------------------------- math
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x sigmoid(x) = x (1 + tanh(x/2)) / 2 with the hardware tanh
+// approximation (one MUFU operation; relative error of silu below 3e-4).
+__device__ __forceinline__ float silu_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return x * fmaf(0.5f, t, 0.5f);
+}
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
 // log(1 + e^x) without overflow; above 20 the correction is below 2.1e-9.
 __device__ __forceinline__ float softplus_f(float x) {
