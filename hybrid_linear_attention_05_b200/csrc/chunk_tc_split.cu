@@ -1,26 +1,38 @@
 // Chunked gated delta rule on the tensor cores, as two kernels.
 //
 // The single-kernel path (chunk_tc.cu) runs everything for one (value head,
-// sequence) on one SM, so a batch with few heads x sequences leaves most SMs
-// idle, and every chunk pays the key-side work (which does not depend on the
-// state) inside the serial state chain.  Here that work moves out:
+// sequence) on one SM: a batch with few heads x sequences leaves most SMs
+// idle, and each chunk pays the key-side work (which does not depend on the
+// state) inside the serial state chain.  Here the chain keeps only what needs
+// the state.  With Tb = T diag(beta), Tbe = T diag(beta e^gamma), W = Tbe K
+// and U = Tb V, the new values and the chunk output are
+//     Vn = U - W S0^T,
+//     O  = Qt S0^T + Pt V,   Qt = diag(e^gamma) Q - P W,   Pt = P Tb,
+// so one M = 128 accumulator [-W; Qt] S0^T plus [U; Pt V] holds both.
 //
 //  1. chunk_keys_kernel, one CTA per (chunk, value head), on every SM:
-//       D1 = [K; Q] K^T  ->  A = beta e^{gamma_i-gamma_j} K K^T,  P = (Q K^T) o decay
-//       T  = (I + A)^-1                (CUDA cores, fp32)
-//       D3 = K^T (T diag(beta e^gamma))^T = W^T
-//     and writes one record per (chunk, head): fp16 images of -W^T, of
-//     T diag(beta) and of P, laid out exactly as the tensor cores read them
-//     from shared memory (128-byte swizzle), plus e^{gamma_i} and
-//     e^{gamma_L - gamma_i}.
-//  2. chunk_chain_kernel, one CTA per (value head, sequence), walks the
-//     chunks with the fp32 state in TMEM.  Each chunk's record arrives in
-//     shared memory by one bulk copy, next to the TMA tiles of K, Q, V:
-//       D2  = V^T (T diag beta)^T + S (-W^T)   = Vn^T
-//       D4  = S Q^T
-//       S   = e^{gamma_L} S + (Vn^T diag(e^{gamma_L-gamma})) K
-//       D5  = Vn^T P^T
-//       O^T = D4 diag(e^gamma) + D5, then the gated RMSNorm per token.
+//       D1 = [K; Q] K^T              ->  A = beta e^{gamma_i-gamma_j} K K^T,  P
+//       T  = (I + A)^-1              (CUDA cores, fp32)
+//       D2 = [Tb; P] [Tb | Tbe]      ->  Pt = P Tb,  Ph = P Tbe
+//       D3 = [Tbe 0; Ph -E] [K; Q]   =   [W; -Qt]    (E = diag(e^gamma))
+//       D4 = [Tb; Pt] V              =   [U; Pt V]
+//     and writes one record per (chunk, head): fp16 images of [-W; Qt] (the
+//     A operand of the chain, 128-byte swizzle) and of [U; Pt V] (swizzled
+//     rows, split into 64-column value blocks), then e^{gamma_L - gamma_i}
+//     and e^{gamma_L}.
+//  2. chunk_chain_kernel walks the chunks of one (value head, sequence) with
+//     the fp32 state slice S^T[dk][v] in TMEM.  The value columns are split
+//     over a cluster of CL CTAs (each state row evolves on its own); only the
+//     gated RMSNorm needs whole rows, and the CTAs swap per-token sums of
+//     squares through distributed shared memory.  One thread streams the K
+//     tile and the record into a ring of stages.  Per chunk:
+//       D   = [-W; Qt] S0^T                      (tensor cores)
+//       Vn  = D[0:64] + U,   O = D[64:128] + Pt V
+//       S^T = e^{gamma_L} S^T + K^T (diag(e^{gamma_L-gamma}) Vn)
+//     Threads owning Vn rows feed the state update; threads owning O rows
+//     reduce the per-token sums of squares of chunk c while the state moves
+//     on, and write chunk c's gated output during chunk c+1 from the
+//     w * silu(z) tile that the key-side kernel left in the record.
 // The algebra is the chunked (WY / UT transform) form of the recurrence, exact
 // in real arithmetic ("Qwen (text & vision-language)", Verified parity).
 // No TMA multicast is used.
@@ -37,18 +49,29 @@ __device__ int g_split_error = 0;  // nonzero: a bounded wait in a kernel of thi
 #ifdef GDN_PHASE_TIMING
 // Development aid (off by default): SM cycles spent by chain-kernel thread 0
 // in each phase of the chunk loop, summed over all CTAs.
-__device__ unsigned long long g_split_phase[16];
-#define GDN_SPLIT_PHASE(k)                                              \
+__device__ unsigned long long g_split_phase[32];
+#define GDN_SPLIT_MARK(k)                                               \
   do {                                                                  \
-    if (tid == 0) {                                                     \
+    if (tid == 64) {                                                    \
       const long long t_ = clock64();                                   \
       atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
+      t_prev = t_;                                                      \
+    }                                                                   \
+  } while (0)
+#define GDN_SPLIT_PHASE(k)                                              \
+  do {                                                                  \
+    if (tid == 0 || tid == 64) {                                        \
+      const long long t_ = clock64();                                   \
+      atomicAdd(&g_split_phase[(k) + (tid ? 8 : 0)], (unsigned long long)(t_ - t_prev));  \
       t_prev = t_;                                                      \
     }                                                                   \
   } while (0)
 #else
 #define GDN_SPLIT_PHASE(k) \
   do {                     \
+  } while (0)
+#define GDN_SPLIT_MARK(k) \
+  do {                    \
   } while (0)
 #endif
 
@@ -62,11 +85,11 @@ constexpr int D = 128;
 constexpr uint32_t TILE = 64 * 128;  // one 64 x 64 16-bit box
 
 // ---- record written by the key-side kernel for one (chunk, value head)
-constexpr uint32_t R_WT = 0;       // -W^T: MN-major B image, 128 rows (dk) x 128 B (64 tokens)
-constexpr uint32_t R_TB = 16384;   // T diag(beta): K-major B image, 64 rows (i) x 128 B (j)
-constexpr uint32_t R_P = 24576;    // P: K-major B image, 64 rows (i) x 128 B (j)
-constexpr uint32_t R_VEC = 32768;  // fp32 e^{gamma_i} [64], then e^{gamma_L - gamma_i} [64]
-constexpr uint32_t REC = 33280;
+constexpr uint32_t R_WQ = 0;       // [-W; Qt]: K-major image, 128 rows x 128 dk (two 16 KiB dk atoms)
+constexpr uint32_t R_UO = 32768;   // [U; Pt V]: 128 rows x 128 v as two 16 KiB swizzled value blocks
+constexpr uint32_t R_ZW = 65536;   // w * silu(z) in fp16: two 8 KiB value blocks, 64 rows x 128 B, swizzled
+constexpr uint32_t R_VEC = 81920;  // fp32 e^{gamma_L - gamma_i} [64] (0 past the chunk), e^{gamma_L}
+constexpr uint32_t REC = 82432;
 
 // Record slot of chunk c of sequence n is slot_start(n) + c; slot_start is
 // strictly increasing in n and the slots of different chunks never collide.
@@ -77,19 +100,22 @@ __device__ __forceinline__ int slot_start(const int32_t* cu, int n, int T) {
 // ===================================================== key-side kernel
 constexpr int NTA = 256;
 constexpr uint32_t A_KQ = 0;                     // [K;Q] tile: two dk halves x 128 rows x 128 B
-constexpr uint32_t A_TBE = 32768;                // T diag(beta e^gamma), fp16 K-major image
-constexpr uint32_t A_AF = 40960;                 // fp32 A [64][AS]
+constexpr uint32_t A_TBP = 32768;                // [Tb; P], later [Tb; Pt]: K-major, 128 rows x 64
+constexpr uint32_t A_V = 49152;                  // V tile: two 64-column halves x 64 rows
+constexpr uint32_t A_AW = 65536;                 // [Tbe 0; Ph -E]: two 16 KiB K atoms
+constexpr uint32_t A_AF = A_AW;                  // fp32 A [64][AS] (dead before A_AW is written)
 constexpr uint32_t A_TF = A_AF + 64 * AS * 4;    // fp32 T [64][AS]; before it the decay table E
 constexpr uint32_t A_X = A_TF + 64 * AS * 4;     // fp32 scratch of the inverse, 1024 floats
 constexpr uint32_t A_MISC = A_X + 4096;          // gamma, e^gamma, beta, scan
 constexpr uint32_t A_BAR = A_MISC + 3 * 256 + 64;
 constexpr uint32_t A_SMEM = A_BAR + 64 + 1024;   // + alignment slack
-constexpr uint32_t A_TM_D1 = 0, A_TM_D3 = 64, A_TM_COLS = 128;
+constexpr uint32_t A_TM_D1 = 0, A_TM_D3 = 0, A_TM_D2 = 128, A_TM_D4 = 128, A_TM_COLS = 256;
+static_assert(A_AW + 32768 <= A_MISC, "AW image inside the dead fp32 scratch");
 static_assert(2 * A_SMEM <= 232448, "two key-side CTAs per SM");
 
 __global__ void __launch_bounds__(NTA, 2)
     chunk_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      ChunkParams p) {
+                      const __grid_constant__ CUtensorMap tm_v, ChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -101,8 +127,9 @@ __global__ void __launch_bounds__(NTA, 2)
   float* eg = gam + 64;
   float* bet = eg + 64;
   float* scan = bet + 64;
-  const uint32_t bar_load = sb + A_BAR, bar_m1 = sb + A_BAR + 8, bar_w = sb + A_BAR + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + A_BAR + 24);
+  const uint32_t bar_load = sb + A_BAR, bar_m1 = sb + A_BAR + 8, bar_m2 = sb + A_BAR + 16,
+                 bar_m3 = sb + A_BAR + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + A_BAR + 32);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7, tl = tid & 127;
@@ -126,7 +153,8 @@ __global__ void __launch_bounds__(NTA, 2)
   if (tid == 0) {
     mbar_init(bar_load, 1);
     mbar_init(bar_m1, 1);
-    mbar_init(bar_w, 1);
+    mbar_init(bar_m2, 1);
+    mbar_init(bar_m3, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -140,13 +168,28 @@ __global__ void __launch_bounds__(NTA, 2)
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_load, 4 * TILE);
+    mbar_arrive_expect_tx(bar_load, 6 * TILE);
     tma_load_2d(sb + A_KQ, &tm_k, hk * D, c0, bar_load);
     tma_load_2d(sb + A_KQ + 16384, &tm_k, hk * D + 64, c0, bar_load);
     tma_load_2d(sb + A_KQ + 8192, &tm_q, hk * D, c0, bar_load);
     tma_load_2d(sb + A_KQ + 16384 + 8192, &tm_q, hk * D + 64, c0, bar_load);
+    tma_load_2d(sb + A_V, &tm_v, h * D, c0, bar_load);
+    tma_load_2d(sb + A_V + TILE, &tm_v, h * D + 64, c0, bar_load);
   }
-  // gates of the chunk: gamma = cumulative g, e^gamma, beta
+  // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
+  // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
+  const bool gated = p.out != nullptr;
+  uint4 zv[4];
+  if (gated) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+      zv[k] = r < L ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.z) +
+                                                           (size_t)(c0 + r) * p.Hv * D + h * D + ch * 8))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
   float gv = 0.f, bv = 0.f;
   if (tid < 64) {
     if (tid < L) {
@@ -188,14 +231,33 @@ __global__ void __launch_bounds__(NTA, 2)
     }
     if (tid < 64) {
       float* vec = reinterpret_cast<float*>(rec + R_VEC);
-      vec[tid] = eg[tid];
-      vec[64 + tid] = __expf(gam[L - 1] - gam[tid]);
+      vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
+      if (tid == 0) vec[64] = eg[L - 1];
+    }
+    // w * silu(z) -> record, in the chain's tile layout (block ch / 8, row r, swizzled chunk)
+    if (gated) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+        const uint4 wq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.norm_w) + ch * 8));
+        const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
+        uint4 res;
+        __half2* r2 = reinterpret_cast<__half2*>(&res);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 wf = __bfloat1622float2(w2[q]), zf = __bfloat1622float2(z2[q]);
+          r2[q] = __floats2half2_rn(wf.x * silu_tanh(zf.x), wf.y * silu_tanh(zf.y));
+        }
+        *reinterpret_cast<uint4*>(rec + R_ZW + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
+      }
     }
     ok = mbar_wait(bar_m1, 0);
   }
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
-    // A (rows 0..63) and P (rows 64..127); this thread: columns wg*32 .. wg*32+31
+    // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
+    // This thread: row tl, columns wg*32 .. wg*32+31.
     {
       float x[32];
       tmem_ld32(lane_base + A_TM_D1 + wg * 32, x);
@@ -224,61 +286,118 @@ __global__ void __launch_bounds__(NTA, 2)
             const int j = wg * 32 + q * 8 + e;
             f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
           }
-          st_half8(rec + R_P, swz(i, wg * 4 + q), f);
+          st_half8(smem + A_TBP, swz(tl, wg * 4 + q), f);
         }
       }
     }
     __syncthreads();
     solve_unit_lower<NTA>(Af, Tf, Xs, tid);
-    // T diag(beta) -> record, T diag(beta e^gamma) -> shared memory (B of W^T)
-    {
-      const int i = tid >> 2, qt = tid & 3;
+    // this thread's 16 entries of T, row i = tid / 4, columns (tid % 4) * 16 ..
+    const int i = tid >> 2, qt = tid & 3;
+    float tv[16];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float fb[8], fe[8];
+    for (int e4 = 0; e4 < 16; e4 += 4) {
+      const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + qt * 16 + e4);
+      tv[e4] = t4.x; tv[e4 + 1] = t4.y; tv[e4 + 2] = t4.z; tv[e4 + 3] = t4.w;
+    }
+    __syncthreads();  // the fp32 scratch is dead from here: the AW image goes over it
 #pragma unroll
-        for (int e4 = 0; e4 < 8; e4 += 4) {
-          const int j0 = qt * 16 + q * 8 + e4;
-          const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + j0);
-          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+    for (int q = 0; q < 2; ++q) {
+      float fb[8], fe[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float t = tv[u] * bet[j0 + u];
-            fb[e4 + u] = t;
-            fe[e4 + u] = t * eg[j0 + u];
-          }
-        }
-        st_half8(rec + R_TB, swz(i, qt * 2 + q), fb);
-        st_half8(smem + A_TBE, swz(i, qt * 2 + q), fe);
+      for (int e = 0; e < 8; ++e) {
+        const int j = qt * 16 + q * 8 + e;
+        fb[e] = tv[q * 8 + e] * bet[j];
+        fe[e] = fb[e] * eg[j];
+      }
+      st_half8(smem + A_TBP, swz(i, qt * 2 + q), fb);  // Tb: A rows 0..63 and B block 0 of D2
+      st_half8(smem + A_AW, swz(i, qt * 2 + q), fe);   // Tbe: AW rows 0..63 and B block 1 of D2
+    }
+    // AW's second K atom: zero on rows 0..63, -E on rows 64..127
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + NTA * k, r = e >> 3, ch = e & 7;
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int ii = r - 64, j = ch * 8 + u;
+        f[u] = (r >= 64 && j == ii && ii < L) ? -eg[ii] : 0.f;
+      }
+      st_half8(smem + A_AW + 16384, swz(r, ch), f);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {  // D2 = [Tb; P] [Tb | Tbe]
+      tc_fence_after();
+      constexpr uint32_t id = idesc_f16(128, 128, false, true);
+      const uint64_t da = sdesc_sw128(sb + A_TBP, 16, 1024);
+      const uint64_t db = sdesc_sw128(sb + A_TBP, A_AW - A_TBP, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f16(tmem + A_TM_D2, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
+      mma_commit(bar_m2);
+    }
+    ok = mbar_wait(bar_m2, 0);
+  }
+  if (!__syncthreads_or(!ok)) {
+    tc_fence_after();
+    // rows 64..127 of D2: Pt (columns 0..63) over P in [Tb; P], Ph (64..127) -> AW rows 64..127
+    if (tl >= 64) {
+      float x[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(lane_base + A_TM_D2 + wg * 64 + hh * 32, x);
+        uint8_t* dst = smem + (wg == 0 ? A_TBP : A_AW);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_half8(dst, swz(tl, hh * 4 + q), x + q * 8);
       }
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {  // D3 = K^T Tbe^T = W^T
+    if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 64, true, false);
-      const uint64_t dk = sdesc_sw128(sb + A_KQ, 16384, 1024), dt = sdesc_sw128(sb + A_TBE, 16, 1024);
+      // D3 = [Tbe 0; Ph -E] [K; Q] = [W; -Qt]
+      constexpr uint32_t id = idesc_f16(128, 128, false, true);
+      const uint64_t da = sdesc_sw128(sb + A_AW, 16, 1024);
+      const uint64_t db = sdesc_sw128(sb + A_KQ, 16384, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_f16(tmem + A_TM_D3, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(db, kk * 2048),
+                id, kk > 0);
+      // D4 = [Tb; Pt] V = [U; Pt V]
+      const uint64_t dt = sdesc_sw128(sb + A_TBP, 16, 1024);
+      const uint64_t dv = sdesc_sw128(sb + A_V, TILE, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + A_TM_D3, sdesc_add(dk, kk * 2048), sdesc_add(dt, kk * 32), id, kk > 0);
-      mma_commit(bar_w);
+        mma_f16(tmem + A_TM_D4, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
+      mma_commit(bar_m3);
     }
-    ok = mbar_wait(bar_w, 0);
+    ok = mbar_wait(bar_m3, 0);
   }
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
-    // -W^T -> record (row l = tl, tokens wg*32 .. wg*32+31)
+    // row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg -> record
     float x[32];
-    tmem_ld32(lane_base + A_TM_D3 + wg * 32, x);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] = -x[j];
+    for (int hh = 0; hh < 2; ++hh) {
+      tmem_ld32(lane_base + A_TM_D3 + wg * 64 + hh * 32, x);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) st_half8(rec + R_WT, swz(tl, wg * 4 + q), x + q * 8);
+      for (int j = 0; j < 32; ++j) x[j] = -x[j];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st_half8(rec + R_WQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      tmem_ld32(lane_base + A_TM_D4 + wg * 64 + hh * 32, x);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st_half8(rec + R_UO + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+    }
   } else if (tid == 0) {
     atomicExch(&g_split_error, 1);
     mbar_wait(bar_load, 0, 100000000ull);
-    mbar_wait(bar_w, 0, 100000000ull);
+    mbar_wait(bar_m3, 0, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();
@@ -289,319 +408,374 @@ __global__ void __launch_bounds__(NTA, 2)
 }
 
 // ========================================================= chain kernel
-constexpr int NTB = 512;
-constexpr int CW = 16;                            // columns of a 64-wide accumulator per warpgroup
-constexpr int SW = 32;                            // columns of the state per warpgroup
-constexpr uint32_t B_KQ = 0;                      // per stage: [K;Q] tile (32 KiB)
-constexpr uint32_t B_V = 32768;                   //            V tile (16 KiB), later Vn^T decayed
-constexpr uint32_t B_REC = 49152;                 //            record; its -W^T image later Vn^T
-constexpr uint32_t B_STAGE = 83968;               // 82 KiB per stage
-constexpr uint32_t B_Z = 2 * B_STAGE;             // z tile, then the output tile
-constexpr uint32_t B_S16 = B_Z + 16384;           // fp16 state (K-major A operand, two dk halves)
-constexpr uint32_t B_MISC = B_S16 + 32768;        // per-token sum of squares
-constexpr uint32_t B_BAR = B_MISC + 512;
-constexpr uint32_t B_SMEM = B_BAR + 64 + 1024;
-static_assert(B_REC + REC <= B_STAGE, "record fits its stage");
-static_assert(B_SMEM <= 232448, "shared memory");
-constexpr uint32_t B_TM_S = 0, B_TM_D2 = 128, B_TM_D4 = 192, B_TM_D5 = 256, B_TM_COLS = 512;
+// VS value columns per CTA; CL = 128 / VS CTAs (one cluster) per (head, sequence).
+template <int VS>
+struct ChainCfg {
+  static constexpr int CL = D / VS;
+  static constexpr int NA = VS / 64;                  // 64-wide value blocks
+  static constexpr int CW = VS / 4;                   // value columns per warpgroup
+  static constexpr int NST = VS == 64 ? 3 : 2;        // stages in the ring
+  static constexpr uint32_t S_K = 0;                  // per stage: K tile (two dk halves, 16 KiB)
+  static constexpr uint32_t S_WQ = 16384;             //   [-W; Qt] (32 KiB)
+  static constexpr uint32_t S_UO = 49152;             //   this CTA's blocks of [U; Pt V]
+  static constexpr uint32_t S_VEC = S_UO + NA * 16384;
+  static constexpr uint32_t STAGE = (S_VEC + 512 + 1023) / 1024 * 1024;
+  static constexpr uint32_t S16 = NST * STAGE;        // fp16 S0^T (NA x 16 KiB); then decayed Vn (NA x 8 KiB)
+  static constexpr uint32_t ZT = S16 + NA * 16384;    // z of the pending chunk, then its output (NA x 8 KiB)
+  static constexpr uint32_t SSP = ZT + NA * 8192;     // per-token partial sums of squares [4][64]
+  static constexpr uint32_t OWN = SSP + 1024;         // this CTA's per-token sums [2][64]
+  static constexpr uint32_t XB = OWN + 512;           // the other CTA's per-token sums [2][64]
+  static constexpr uint32_t BAR = XB + 512;
+  static constexpr uint32_t SMEM = BAR + 128 + 1024;
+  static constexpr uint32_t TM_S = 0, TM_D = VS;      // state, then two [Vn; O] accumulators
+  static constexpr uint32_t TM_COLS = 3 * VS <= 256 ? 256 : 512;
+  static_assert(SMEM <= 232448, "shared memory");
+};
+constexpr int NCW = 512;        // four warpgroups
+constexpr int NTB = NCW;
+constexpr int BAR_COMPUTE = 1;  // named barrier of the compute threads
+constexpr int BAR_OUT = 2;      // the 256 threads that own output rows
+constexpr int BAR_VN = 3;       // the 256 threads that own new-value rows
 
+template <int CW>
+__device__ __forceinline__ void tmem_ldw(uint32_t taddr, float* v) {
+  if constexpr (CW == 16) tmem_ld16(taddr, v); else tmem_ld32(taddr, v);
+}
+template <int CW>
+__device__ __forceinline__ void tmem_stw(uint32_t taddr, const float* v) {
+  if constexpr (CW == 16) tmem_st16(taddr, v); else tmem_st32(taddr, v);
+}
+// x[0..8q) += eight fp16 values at base + off, q times along swizzled 16-byte chunks
+__device__ __forceinline__ void add_half8(const uint8_t* base, uint32_t off, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(base + off);
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h2[e]);
+    x[2 * e] += f.x;
+    x[2 * e + 1] += f.y;
+  }
+}
+
+template <int VS>
 __global__ void __launch_bounds__(NTB, 1)
-    chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
-                       ChunkParams p) {
+    chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_k, ChunkParams p) {
+  using G = ChainCfg<VS>;
+  constexpr int CL = G::CL, NA = G::NA, CW = G::CW, NST = G::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
-  __nv_bfloat16* Zs = reinterpret_cast<__nv_bfloat16*>(smem + B_Z);
-  float* ss = reinterpret_cast<float*>(smem + B_MISC);
-  const uint32_t bar_load0 = sb + B_BAR, bar_z = sb + B_BAR + 16, bar_v = sb + B_BAR + 24,
-                 bar_o = sb + B_BAR + 32;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + B_BAR + 40);
+  float* ssp = reinterpret_cast<float*>(smem + G::SSP);
+  float* own = reinterpret_cast<float*>(smem + G::OWN);
+  float* xb = reinterpret_cast<float*>(smem + G::XB);
+  const uint32_t bar_full = sb + G::BAR, bar_free = bar_full + 8 * NST, bar_a = bar_free + 8 * NST,
+                 bar_s = bar_a + 8, bar_x = bar_s + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR + 8 * (2 * NST + 4));
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7, tl = tid & 127;
-  const int h = blockIdx.x, n = blockIdx.y;
+  const int h = blockIdx.x / CL, vs = blockIdx.x % CL, n = blockIdx.y;
   const int hk = h / (p.Hv / p.Hk);
   const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
   const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
   const int nchunks = (eos - bos + C - 1) / C;
-  const size_t sbase = ((size_t)n * p.Hv + h) * D * D;
+  const size_t sbase = ((size_t)n * p.Hv + h) * D * D + (size_t)vs * VS * D;  // first row of the slice
   const bool norm_out = p.out != nullptr;
 
-  if (nchunks == 0) {  // empty sequence: the state passes through
+  if (nchunks == 0) {  // empty sequence: the state passes through (every CTA of the cluster returns here)
     if (p.S_out)
-      for (int idx = tid; idx < D * D; idx += NTB) p.S_out[sbase + idx] = p.S0 ? p.S0[sbase + idx] : 0.f;
+      for (int idx = tid; idx < VS * D; idx += NTB) p.S_out[sbase + idx] = p.S0 ? p.S0[sbase + idx] : 0.f;
     return;
   }
   const int slot0 = slot_start(p.cu_seqlens, n, p.T);
 
   if (tid == 0) {
-    mbar_init(bar_load0, 1);
-    mbar_init(bar_load0 + 8, 1);
-    mbar_init(bar_z, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar_o, 1);
+    for (int k = 0; k < NST; ++k) {
+      mbar_init(bar_full + 8 * k, 1);
+      mbar_init(bar_free + 8 * k, 1 + 256);  // the state-update MMAs and the output-row threads
+    }
+    mbar_init(bar_a, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_x, 1);
+    mbar_init(bar_x + 8, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), B_TM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), G::TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CL > 1) cluster_sync();  // the other CTA's barriers exist before anyone arrives on them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-
-  auto issue_loads = [&](int cc, int s) {
-    const int row = bos + cc * C;
-    const uint32_t bar = bar_load0 + 8 * s;
-    const uint32_t st = sb + s * B_STAGE;
-    mbar_arrive_expect_tx(bar, 6 * TILE + REC);
-    tma_load_2d(st + B_KQ, &tm_k, hk * D, row, bar);
-    tma_load_2d(st + B_KQ + 16384, &tm_k, hk * D + 64, row, bar);
-    tma_load_2d(st + B_KQ + 8192, &tm_q, hk * D, row, bar);
-    tma_load_2d(st + B_KQ + 16384 + 8192, &tm_q, hk * D + 64, row, bar);
-    tma_load_2d(st + B_V, &tm_v, h * D, row, bar);
-    tma_load_2d(st + B_V + 8192, &tm_v, h * D + 64, row, bar);
-    bulk_load(st + B_REC, p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC, REC, bar);
-  };
-  constexpr int LOADER = 32;  // one lane of warp 1 issues the copies (thread 0 issues the MMAs)
-  if (tid == LOADER) issue_loads(0, 0);
-  const float w_norm = norm_out ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tl]) : 0.f;
-
-  // initial state -> TMEM (row tl, columns wg*SW .. wg*SW+SW-1)
-  {
-    float r[32];
-    const int col = wg * SW;
-#pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      float4 f = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)tl * D + col + j)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      r[j] = f.x; r[j + 1] = f.y; r[j + 2] = f.z; r[j + 3] = f.w;
-    }
-    tmem_st32(lane_base + B_TM_S + col, r);
-    tmem_wait_st();
-  }
-
-  bool ok = true;
+  bool bad = false;  // uniform over the compute threads: a bounded wait gave up
   int c = 0;
-#ifdef GDN_PHASE_TIMING
-  long long t_prev = clock64();
-#endif
-  for (; c < nchunks; ++c) {
-    const int s = c & 1;
-    const int c0 = bos + c * C;
-    const int L = min(C, eos - c0);
-    const uint32_t par = (uint32_t)c & 1u;
-    const uint32_t st = sb + s * B_STAGE;
-    uint8_t* stp = smem + s * B_STAGE;
-    const float* vec = reinterpret_cast<const float*>(stp + B_REC + R_VEC);  // e^gamma, decay to end
 
-    if (tid == LOADER) {
-      if (c + 1 < nchunks) issue_loads(c + 1, s ^ 1);
-      if (norm_out) {
-        mbar_arrive_expect_tx(bar_z, 2 * TILE);
-        tma_load_2d(sb + B_Z, &tm_z, h * D, c0, bar_z);
-        tma_load_2d(sb + B_Z + TILE, &tm_z, h * D + 64, c0, bar_z);
-      }
-    }
-    if (tid < 64) ss[tid] = 0.f;
-    ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
-    if (__syncthreads_or(!ok)) break;
-    GDN_SPLIT_PHASE(0);
+  // thread LOADER streams K and the records: chunks 0 .. NST-1 up front, then
+  // chunk c - 1 + NST once chunk c - 1 has released its stage
+  constexpr int LOADER = 32;
+  auto issue_loads = [&](int cc) {
+    const int s = cc % NST;
+    const int row = bos + cc * C;
+    const uint32_t bar = bar_full + 8 * s, st = sb + s * G::STAGE;
+    const uint8_t* rec = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC;
+    mbar_arrive_expect_tx(bar, 2 * TILE + 32768 + NA * 16384 + 512);
+    tma_load_2d(st + G::S_K, &tm_k, hk * D, row, bar);
+    tma_load_2d(st + G::S_K + TILE, &tm_k, hk * D + 64, row, bar);
+    bulk_load(st + G::S_WQ, rec + R_WQ, 32768, bar);
+    bulk_load(st + G::S_UO, rec + R_UO + vs * NA * 16384, NA * 16384, bar);
+    bulk_load(st + G::S_VEC, rec + R_VEC, 512, bar);
+  };
+  if (tid == LOADER)
+    for (int cc = 0; cc < NST && cc < nchunks; ++cc) issue_loads(cc);
 
-    // D2 = V^T (T diag beta)^T  (= U^T); needs no state
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 64, true, false);
-      const uint64_t dv = sdesc_sw128(st + B_V, 8192, 1024), dt = sdesc_sw128(st + B_REC + R_TB, 16, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_D2, sdesc_add(dv, kk * 2048), sdesc_add(dt, kk * 32), id, kk > 0);
-    }
-    // meanwhile: state -> fp16 operand, then S *= e^{gamma_L} in TMEM
+  {
+    // ----------------------------------------------------------- compute
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int col = wg * CW;                     // this thread's value columns in the slice
+    const int vcol = h * D + vs * VS + col;      // ... as columns of [T, Hv * d]
+    const uint32_t blk = (uint32_t)(col >> 6) * 16384;        // its 64-column block in S16 / [U; Pt V]
+    const int ch0 = (col & 63) >> 3;                          // its first 16-byte chunk in a block row
+    const bool orow = tl >= 64;                  // owns output row tl - 64 (else new-value row tl)
+    const int t = tl - 64;
+
+    // initial state: S^T[dk = tl][v] = S0[v][dk]
     {
-      const float egL = vec[L - 1];
-      uint8_t* half_base = smem + B_S16 + (wg >> 1) * 16384;
-      const int col = wg * SW;
-      float r[32];
-      tmem_ld32(lane_base + B_TM_S + col, r);
+      float r[CW];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(half_base, swz(tl, (wg & 1) * 4 + q), r + q * 8);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] *= egL;
-      tmem_st32(lane_base + B_TM_S + col, r);
+      for (int j = 0; j < CW; ++j) r[j] = p.S0 ? p.S0[sbase + (size_t)(col + j) * D + tl] : 0.f;
+      tmem_stw<CW>(lane_base + G::TM_S + col, r);
       tmem_wait_st();
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
 
-    // D2 += S (-W^T)  (= Vn^T), committed alone; then D4 = S Q^T
-    GDN_SPLIT_PHASE(1);
-    if (tid == 0) {
+#ifdef GDN_PHASE_TIMING
+    long long t_prev = clock64();
+#endif
+    // w * silu(z) tile: output-row thread io copies (and later stores) the
+    // 16-byte chunks at tile offsets (io + 256 k) * 16; the record holds the
+    // tile in this layout, so both global transfers are coalesced
+    constexpr int ZK = 64 * (VS / 8) / 256;
+    const int io = wg * 64 + t;
+    auto z_copy = [&](int cc) {
+      const uint8_t* src = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC + R_ZW + vs * NA * 8192;
+#pragma unroll
+      for (int k = 0; k < ZK; ++k) {
+        const uint32_t pos = (uint32_t)(io + 256 * k) * 16;
+        cp_async16(sb + G::ZT + pos, src + pos, 16u);
+      }
+      cp_async_commit();
+    };
+
+    // gated output of chunk co (output-row threads): its O rows were
+    // completed and their sums of squares published during chunk co; the
+    // other CTA's sums arrive on bar_x, z waits in the tile
+    float o[CW];  // O rows of the chunk whose output is pending (plus Pt V)
+#pragma unroll
+    for (int j = 0; j < CW; ++j) o[j] = 0.f;
+    auto finish_output = [&](int co) -> bool {
+      bool okk = true;
+      const int bo = co & 1;
+      const int c0o = bos + co * C, Lo = min(C, eos - c0o);
+      GDN_SPLIT_MARK(16);
+      if (norm_out) {
+        float tot = own[bo * 64 + t];
+        if constexpr (CL > 1) {
+          okk = mbar_wait_cluster(bar_x + 8 * bo, (uint32_t)(co >> 1) & 1u);
+          tot += xb[bo * 64 + t];
+        }
+        const float ri = rsqrtf(tot * (1.0f / D) + p.eps_norm);
+        GDN_SPLIT_MARK(17);
+#pragma unroll
+        for (int q = 0; q < CW / 8; ++q) {
+          uint4* zq = reinterpret_cast<uint4*>(smem + G::ZT + (blk >> 1) + swz(t, ch0 + q));
+          const uint4 zv = *zq;
+          const __half2* z2 = reinterpret_cast<const __half2*>(&zv);
+          uint4 res;
+          __nv_bfloat162* r2 = reinterpret_cast<__nv_bfloat162*>(&res);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 zf = __half22float2(z2[e]);
+            r2[e] = __floats2bfloat162_rn(o[q * 8 + 2 * e] * ri * zf.x, o[q * 8 + 2 * e + 1] * ri * zf.y);
+          }
+          *zq = res;  // the output over its own w * silu(z)
+        }
+        GDN_SPLIT_MARK(18);
+        bar_named(BAR_OUT, 256);
+        GDN_SPLIT_MARK(19);
+        uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0o * p.Hv * D + h * D + vs * VS) * 2;
+#pragma unroll
+        for (int k = 0; k < ZK; ++k) {
+          const uint32_t pos = (uint32_t)(io + 256 * k) * 16;
+          const int r = (pos & 8191) >> 7, ch = (int)(pos >> 13) * 8 + ((int)((pos >> 4) & 7) ^ (r & 7));
+          if (r < Lo)
+            *reinterpret_cast<uint4*>(obase + ((size_t)r * p.Hv * D + ch * 8) * 2) =
+                *reinterpret_cast<const uint4*>(smem + G::ZT + pos);
+        }
+        // the next chunk's z over the chunks this thread just stored
+        if (co + 1 < nchunks) z_copy(co + 1);
+        GDN_SPLIT_MARK(20);
+      } else if (t < Lo) {
+        float* dst = p.o_raw + (size_t)(c0o + t) * p.Hv * D + vcol;
+#pragma unroll
+        for (int q = 0; q < CW / 4; ++q)
+          *reinterpret_cast<float4*>(dst + q * 4) = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+      return okk;
+    };
+    if (norm_out && orow) z_copy(0);
+
+    bool ok = true;
+    for (; c < nchunks; ++c) {
+      const int s = c % NST, b = c & 1;
+      const int c0 = bos + c * C;
+      const int L = min(C, eos - c0);
+      uint8_t* stp = smem + s * G::STAGE;
+      const uint32_t st = sb + s * G::STAGE;
+      const float* vec = reinterpret_cast<const float*>(stp + G::S_VEC);
+
+      // the previous chunk's z (copied during that chunk) is in the tile once
+      // every output-row thread has waited here and passed the barrier below
+      if (norm_out && orow) cp_async_wait_all();
+      ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;
+      GDN_SPLIT_PHASE(0);
+      // state -> fp16 operand, then S *= e^{gamma_L} in TMEM
+      if (c > 0) ok = mbar_wait(bar_s, (uint32_t)(c - 1) & 1u) && ok;
       tc_fence_after();
-      constexpr uint32_t id_w = idesc_f16(128, 64, false, true);
-      constexpr uint32_t id_q = idesc_f16(128, 64, false, false);
-      const uint64_t ds = sdesc_sw128(sb + B_S16, 16, 1024);
-      const uint64_t dw = sdesc_sw128(st + B_REC + R_WT, 16384, 1024);
-      const uint64_t dq = sdesc_sw128(st + B_KQ + 8192, 16, 1024);
+      GDN_SPLIT_PHASE(1);
+      {
+        const float egL = vec[64];
+        float r[CW];
+        tmem_ldw<CW>(lane_base + G::TM_S + col, r);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + B_TM_D2, sdesc_add(ds, aoff), sdesc_add(dw, kk * 2048), id_w, 1);
+        for (int q = 0; q < CW / 8; ++q) st_half8(smem + G::S16 + blk, swz(tl, ch0 + q), r + q * 8);
+#pragma unroll
+        for (int j = 0; j < CW; ++j) r[j] *= egL;
+        tmem_stw<CW>(lane_base + G::TM_S + col, r);
+        tmem_wait_st();
       }
-      mma_commit(bar_v);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + B_TM_D4, sdesc_add(ds, aoff), sdesc_add(dq, aoff), id_q, kk > 0);
+      fence_proxy_async();
+      tc_fence_before();
+      if (bar_named_or(BAR_COMPUTE, NCW, !ok)) { bad = true; break; }
+      GDN_SPLIT_PHASE(2);
+      if (tid == LOADER && c >= 1 && c - 1 + NST < nchunks) {
+        // the state MMAs of chunk c-1 are done; its output rows arrived in its iteration
+        const int cc = c - 1 + NST;
+        if (mbar_wait(bar_free + 8 * (cc % NST), (uint32_t)(cc / NST - 1) & 1u))
+          issue_loads(cc);
+        else
+          ok = false;
       }
-    }
-    ok = mbar_wait(bar_v, par);
-    if (__syncthreads_or(!ok)) break;
-    tc_fence_after();
-    GDN_SPLIT_PHASE(2);
-
-    // Vn^T rows: plain (A of D5, over the consumed -W^T image) and decayed to the chunk end
-    // (A of the state update, over the consumed V tile)
-    {
-      float x[CW];
-      tmem_ld16(lane_base + B_TM_D2 + wg * CW, x);
+      if (warp == 0) {  // D = [-W; Qt] S0^T (descriptors warp-uniform, one lane issues)
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16(128, VS, false, true);
+        const uint64_t da = sdesc_sw128(st + G::S_WQ, 16, 1024);
+        const uint64_t db = sdesc_sw128(sb + G::S16, 16384, 1024);
+        if (elect_one()) {
 #pragma unroll
-      for (int q = 0; q < CW / 8; ++q) {
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int i = wg * CW + q * 8 + e;
-          f[e] = i < L ? x[q * 8 + e] * vec[64 + i] : 0.f;
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem + G::TM_D + b * VS, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
+                    sdesc_add(db, kk * 2048), id, kk > 0);
+          mma_commit(bar_a);
         }
-        st_half8(stp + B_REC + R_WT, swz(tl, wg * (CW / 8) + q), x + q * 8);
-        st_half8(stp + B_V, swz(tl, wg * (CW / 8) + q), f);
+        __syncwarp();
       }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
+      // meanwhile: the previous chunk's gated output
+      if (c > 0 && orow) ok = finish_output(c - 1) && ok;
 
-    // S += Vts K,  D5 = Vn^T P^T
-    GDN_SPLIT_PHASE(3);
-    if (tid == 0) {
+      GDN_SPLIT_PHASE(3);  // output rows: the previous chunk's output
+      ok = mbar_wait(bar_a, (uint32_t)c & 1u) && ok;
       tc_fence_after();
-      constexpr uint32_t id_s = idesc_f16(128, 128, false, true);
-      constexpr uint32_t id_p = idesc_f16(128, 64, false, false);
-      const uint64_t dvs = sdesc_sw128(st + B_V, 16, 1024), dk = sdesc_sw128(st + B_KQ, 16384, 1024);
-      const uint64_t dvt = sdesc_sw128(st + B_REC + R_WT, 16, 1024), dp = sdesc_sw128(st + B_REC + R_P, 16, 1024);
+      GDN_SPLIT_PHASE(4);
+      if (!orow) {
+        // Vn = D + U, decayed to the chunk end -> B operand of the state update (over S16)
+        float x[CW];
+        tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, x);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_S, sdesc_add(dvs, kk * 32), sdesc_add(dk, kk * 2048), id_s, 1);
+        for (int q = 0; q < CW / 8; ++q) add_half8(stp + G::S_UO + blk, swz(tl, ch0 + q), x + q * 8);
+        const float dec = vec[tl];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + B_TM_D5, sdesc_add(dvt, kk * 32), sdesc_add(dp, kk * 32), id_p, kk > 0);
-      mma_commit(bar_o);
-    }
-    // meanwhile: w * silu(z) for this thread's outputs (column tl, tokens wg*CW ..)
-    float zw[CW];
-    if (norm_out) {
-      ok = mbar_wait(bar_z, par);
-      const __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE / 2) + (tl & 63);
+        for (int j = 0; j < CW; ++j) x[j] *= dec;
 #pragma unroll
-      for (int j = 0; j < CW; ++j) zw[j] = w_norm * silu_tanh(__bfloat162float(zcol[(wg * CW + j) * 64]));
-    }
-    ok = mbar_wait(bar_o, par) && ok;
-    if (__syncthreads_or(!ok)) break;
-    tc_fence_after();
-    GDN_SPLIT_PHASE(4);
-
-    // epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*CW .. wg*CW+CW-1
-    float o[CW];
-    {
-      float a5[CW];
-      tmem_ld16(lane_base + B_TM_D4 + wg * CW, o);
-      tmem_ld16(lane_base + B_TM_D5 + wg * CW, a5);
+        for (int q = 0; q < CW / 8; ++q) st_half8(smem + G::S16 + (blk >> 1), swz(tl, ch0 + q), x + q * 8);
+        fence_proxy_async();
+        tc_fence_before();
+        ok = !bar_named_or(BAR_VN, 256, !ok);
+        GDN_SPLIT_PHASE(5);
+        if (warp == 0 && ok) {  // S^T += K^T Vts; with the output rows' arrivals the stage is free
+          tc_fence_after();
+          constexpr uint32_t id = idesc_f16(128, VS, true, true);
+          const uint64_t da = sdesc_sw128(st + G::S_K, TILE, 1024);
+          const uint64_t db = sdesc_sw128(sb + G::S16, TILE, 1024);
+          if (elect_one()) {
 #pragma unroll
-      for (int j = 0; j < CW; ++j) o[j] = fmaf(vec[wg * CW + j], o[j], a5[j]);
-    }
-    if (norm_out) {
-      // sum over v of o^2 per token: each lane holds one v; fold the 16 token
-      // values across the warp's 32 lanes, then one shared atomic per token
-      float a[CW];
-#pragma unroll
-      for (int j = 0; j < CW; ++j) a[j] = o[j] * o[j];
-#pragma unroll
-      for (int off = 16, cnt = CW; off >= 2; off >>= 1, cnt >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < cnt / 2; ++i) {
-          const float send = upper ? a[i] : a[i + cnt / 2];
-          const float keep = upper ? a[i + cnt / 2] : a[i];
-          a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(tmem + G::TM_S, sdesc_add(da, kk * 2048), sdesc_add(db, kk * 2048), id, 1);
+            mma_commit(bar_s);
+            mma_commit(bar_free + 8 * s);
+          }
+          __syncwarp();
         }
-      }
-      a[0] += __shfl_xor_sync(0xffffffffu, a[0], 1);
-      const int t = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-      if ((lane & 1) == 0) atomicAdd(&ss[wg * CW + t], a[0]);
-      __syncthreads();
-      if (tid < 64) ss[tid] = rsqrtf(ss[tid] * (1.0f / D) + p.eps_norm);  // now 1 / rms
-      __syncthreads();
-    GDN_SPLIT_PHASE(5);
-      // gated output, written over the z tile (each element read, then written, by one thread)
-      __nv_bfloat16* zcol = Zs + (tl >> 6) * (TILE / 2) + (tl & 63);
+      } else {
+        // O = D + Pt V, kept in registers until the next chunk writes it out;
+        // per-token sum of squares -> this CTA's total and the other CTA
+        tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, o);
 #pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int i = wg * CW + j;
-        zcol[i * 64] = __float2bfloat16_rn(o[j] * ss[i] * zw[j]);
-      }
-      fence_proxy_async();  // the next chunk's z tile lands here through TMA
-      __syncthreads();
-      uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv + h) * D * 2;
-      const size_t ostride = (size_t)p.Hv * D * 2;
+        for (int q = 0; q < CW / 8; ++q) add_half8(stp + G::S_UO + blk, swz(tl, ch0 + q), o + q * 8);
+        mbar_arrive(bar_free + 8 * s);
+        if (norm_out) {
+          float ps = 0.f;
 #pragma unroll
-      for (int k = 0; k < 1024 / NTB; ++k) {
-        const int e = tid + NTB * k, row = e >> 4, c16 = e & 15;
-        if (row < L) {
-          const uint4 val = *reinterpret_cast<const uint4*>(smem + B_Z + (c16 >> 3) * TILE + row * 128 +
-                                                           (c16 & 7) * 16);
-          *reinterpret_cast<uint4*>(obase + row * ostride + c16 * 16) = val;
+          for (int j = 0; j < CW; ++j) ps = fmaf(o[j], o[j], ps);
+          ssp[wg * 64 + t] = ps;
+          GDN_SPLIT_PHASE(5);
+          bar_named(BAR_OUT, 256);
+          GDN_SPLIT_PHASE(6);
+          if (wg == 0) {
+            const float tot = (ssp[t] + ssp[64 + t]) + (ssp[128 + t] + ssp[192 + t]);
+            own[b * 64 + t] = tot;
+            if constexpr (CL > 1) {
+              const uint32_t peer = (uint32_t)(vs ^ 1);
+              st_async_f32(mapa_shared(sb + G::XB + (uint32_t)(b * 64 + t) * 4, peer), tot,
+                           mapa_shared(bar_x + 8 * b, peer));
+              if (t == 0) mbar_arrive_expect_tx(bar_x + 8 * b, 64 * 4);  // the other CTA's sums of this chunk
+            }
+          }
         }
-      }
-    } else {
-      float* ocol = p.o_raw + ((size_t)c0 * p.Hv + h) * D + tl;
-      const size_t ostride = (size_t)p.Hv * D;
-#pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int i = wg * CW + j;
-        if (i < L) ocol[i * ostride] = o[j];
+        GDN_SPLIT_PHASE(7);
       }
     }
-    __syncthreads();
-    GDN_SPLIT_PHASE(6);
-  }
-
-  if (!ok) {
-    if (tid == 0) {
+    if (!bad) {
+      bool okk = true;
+      if (norm_out && orow) cp_async_wait_all();
+      bar_named(BAR_COMPUTE, NCW);  // the last chunk's z tile is complete
+      if (orow) okk = finish_output(nchunks - 1);
+      okk = mbar_wait(bar_s, (uint32_t)(nchunks - 1) & 1u) && okk;
+      tc_fence_after();
+      if (!okk) {
+        atomicExch(&g_split_error, 1);
+      } else if (p.S_out) {
+        float r[CW];
+        tmem_ldw<CW>(lane_base + G::TM_S + col, r);
+#pragma unroll
+        for (int j = 0; j < CW; ++j) p.S_out[sbase + (size_t)(col + j) * D + tl] = r[j];
+      }
+    } else if (tid == 0) {
+      // let the copies and MMAs in flight finish before the CTA leaves (the
+      // output-row threads drain their own z copies below)
       atomicExch(&g_split_error, 1);
-      mbar_wait(bar_load0 + 8 * (c & 1), (uint32_t)(c >> 1) & 1u, 100000000ull);
-      if (c + 1 < nchunks)
-        mbar_wait(bar_load0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, 100000000ull);
-      if (norm_out) mbar_wait(bar_z, (uint32_t)c & 1u, 100000000ull);
-      mbar_wait(bar_o, (uint32_t)c & 1u, 100000000ull);
+      for (int k = 0; k < NST && c + k < nchunks; ++k)
+        mbar_wait(bar_full + 8 * ((c + k) % NST), (uint32_t)((c + k) / NST) & 1u, 100000000ull);
+      if (c > 0) mbar_wait(bar_s, (uint32_t)(c - 1) & 1u, 100000000ull);
     }
-  } else if (p.S_out) {
-    float r[32];
-    const int col = wg * SW;
-    tmem_ld32(lane_base + B_TM_S + col, r);
-#pragma unroll
-    for (int j = 0; j < 32; j += 4)
-      *reinterpret_cast<float4*>(p.S_out + sbase + (size_t)tl * D + col + j) =
-          make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+    if (norm_out && orow) cp_async_wait_all();
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CL > 1) cluster_sync();  // no CTA leaves while the other may still write to it
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, B_TM_COLS);
+    tmem_dealloc(tmem, G::TM_COLS);
   }
 }
 
@@ -645,14 +819,52 @@ size_t chunk_tc_split_record_bytes(int N, int T, int Hv) {
   return record_slots(N, T) * (size_t)Hv * REC;
 }
 
+namespace {
+
+int sm_count() {
+  static int count = 0;
+  if (count == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      count = v;
+    else
+      return 148;
+  }
+  return count;
+}
+
+template <int VS>
+cudaError_t launch_chain(const CUtensorMap& mk, const ChunkParams& p, cudaStream_t st) {
+  using G = ChainCfg<VS>;
+  cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel<VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)G::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(G::CL * p.Hv), (unsigned)p.N, 1);
+  cfg.blockDim = dim3(NTB, 1, 1);
+  cfg.dynamicSmemBytes = G::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G::CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<VS>, mk, p);
+}
+
+}  // namespace
+
 cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st) {
   if (p.N == 0 || p.Hv == 0) return cudaSuccess;
   if (!p.rec) return cudaErrorInvalidValue;
-  CUtensorMap mq, mk, mv, mz;
+  CUtensorMap mq, mk, mv;
   memset(&mq, 0, sizeof(mq));
   memset(&mk, 0, sizeof(mk));
   memset(&mv, 0, sizeof(mv));
-  memset(&mz, 0, sizeof(mz));
   if (p.T > 0) {
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -660,31 +872,27 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st) {
         !make_map(&mk, p.k, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
         !make_map(&mv, p.v, (uint64_t)p.T, (uint64_t)p.Hv * D, f16, sw))
       return cudaErrorInvalidValue;
-    if (p.out && !make_map(&mz, p.z, (uint64_t)p.T, (uint64_t)p.Hv * D,
-                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)A_SMEM);
     if (e != cudaSuccess) return e;
     dim3 ga((unsigned)record_slots(p.N, p.T), p.Hv);
-    chunk_keys_kernel<<<ga, NTA, A_SMEM, st>>>(mq, mk, p);
+    chunk_keys_kernel<<<ga, NTA, A_SMEM, st>>>(mq, mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)B_SMEM);
-  if (e != cudaSuccess) return e;
-  dim3 gb(p.Hv, p.N);
-  chunk_chain_kernel<<<gb, NTB, B_SMEM, st>>>(mq, mk, mv, mz, p);
-  return cudaGetLastError();
+  // Half-width value slices (two CTAs per chain) while that still fits the
+  // machine in one wave; otherwise one CTA per chain.
+  const long chains = (long)p.Hv * p.N;
+  if (2 * chains <= sm_count()) return launch_chain<64>(mk, p, st);
+  return launch_chain<128>(mk, p, st);
 }
 
 #ifdef GDN_PHASE_TIMING
 extern "C" int gdn_debug_phase_cycles_split(unsigned long long* out, int clear) {
   cudaDeviceSynchronize();
-  if (cudaMemcpyFromSymbol(out, g_split_phase, sizeof(unsigned long long) * 16) != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(out, g_split_phase, sizeof(unsigned long long) * 32) != cudaSuccess) return -1;
   if (clear) {
-    unsigned long long z[16] = {0};
+    unsigned long long z[32] = {0};
     cudaMemcpyToSymbol(g_split_phase, z, sizeof(z));
   }
   return 0;
