@@ -66,7 +66,18 @@ __device__ unsigned long long g_split_phase[32];
       t_prev = t_;                                                      \
     }                                                                   \
   } while (0)
+#define GDN_KEYS_MARK(k)                                                \
+  do {                                                                  \
+    if (tid == 0) {                                                     \
+      const long long t_ = clock64();                                   \
+      atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
+      t_prev = t_;                                                      \
+    }                                                                   \
+  } while (0)
 #else
+#define GDN_KEYS_MARK(k) \
+  do {                   \
+  } while (0)
 #define GDN_SPLIT_PHASE(k) \
   do {                     \
   } while (0)
@@ -106,8 +117,8 @@ constexpr uint32_t A_AW = 65536;                 // [Tbe 0; Ph -E]: two 16 KiB K
 constexpr uint32_t A_AF = A_AW;                  // fp32 A [64][AS] (dead before A_AW is written)
 constexpr uint32_t A_TF = A_AF + 64 * AS * 4;    // fp32 T [64][AS]; before it the decay table E
 constexpr uint32_t A_X = A_TF + 64 * AS * 4;     // fp32 scratch of the inverse, 1024 floats
-constexpr uint32_t A_MISC = A_X + 4096;          // gamma, e^gamma, beta, scan
-constexpr uint32_t A_BAR = A_MISC + 3 * 256 + 64;
+constexpr uint32_t A_MISC = A_X + 4096;          // gamma, e^gamma, beta, scan, norm weights
+constexpr uint32_t A_BAR = A_MISC + 3 * 256 + 64 + 512;
 constexpr uint32_t A_SMEM = A_BAR + 64 + 1024;   // + alignment slack
 constexpr uint32_t A_TM_D1 = 0, A_TM_D3 = 0, A_TM_D2 = 128, A_TM_D4 = 128, A_TM_COLS = 256;
 static_assert(A_AW + 32768 <= A_MISC, "AW image inside the dead fp32 scratch");
@@ -127,6 +138,7 @@ __global__ void __launch_bounds__(NTA, 2)
   float* eg = gam + 64;
   float* bet = eg + 64;
   float* scan = bet + 64;
+  float* wsm = scan + 16;  // norm weights, fp32 [128]
   const uint32_t bar_load = sb + A_BAR, bar_m1 = sb + A_BAR + 8, bar_m2 = sb + A_BAR + 16,
                  bar_m3 = sb + A_BAR + 24;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + A_BAR + 32);
@@ -166,6 +178,9 @@ __global__ void __launch_bounds__(NTA, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#ifdef GDN_PHASE_TIMING
+  long long t_prev = clock64();
+#endif
 
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_load, 6 * TILE);
@@ -189,6 +204,7 @@ __global__ void __launch_bounds__(NTA, 2)
                     : make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  if (gated && tid < D) wsm[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tid]);
   // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
   float gv = 0.f, bv = 0.f;
   if (tid < 64) {
@@ -211,7 +227,9 @@ __global__ void __launch_bounds__(NTA, 2)
     bet[tid] = bv;
   }
 
+  GDN_KEYS_MARK(21);
   bool ok = mbar_wait(bar_load, 0);
+  GDN_KEYS_MARK(22);
   if (!__syncthreads_or(!ok)) {
     if (tid == 0) {  // D1 = [K; Q] K^T
       tc_fence_after();
@@ -234,26 +252,10 @@ __global__ void __launch_bounds__(NTA, 2)
       vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
       if (tid == 0) vec[64] = eg[L - 1];
     }
-    // w * silu(z) -> record, in the chain's tile layout (block ch / 8, row r, swizzled chunk)
-    if (gated) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
-        const uint4 wq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.norm_w) + ch * 8));
-        const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
-        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
-        uint4 res;
-        __half2* r2 = reinterpret_cast<__half2*>(&res);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 wf = __bfloat1622float2(w2[q]), zf = __bfloat1622float2(z2[q]);
-          r2[q] = __floats2half2_rn(wf.x * silu_tanh(zf.x), wf.y * silu_tanh(zf.y));
-        }
-        *reinterpret_cast<uint4*>(rec + R_ZW + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
-      }
-    }
+    GDN_KEYS_MARK(23);
     ok = mbar_wait(bar_m1, 0);
   }
+  GDN_KEYS_MARK(24);
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
     // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
@@ -291,7 +293,9 @@ __global__ void __launch_bounds__(NTA, 2)
       }
     }
     __syncthreads();
+    GDN_KEYS_MARK(25);
     solve_unit_lower<NTA>(Af, Tf, Xs, tid);
+    GDN_KEYS_MARK(26);
     // this thread's 16 entries of T, row i = tid / 4, columns (tid % 4) * 16 ..
     const int i = tid >> 2, qt = tid & 3;
     float tv[16];
@@ -338,6 +342,7 @@ __global__ void __launch_bounds__(NTA, 2)
         mma_f16(tmem + A_TM_D2, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
       mma_commit(bar_m2);
     }
+    GDN_KEYS_MARK(27);
     ok = mbar_wait(bar_m2, 0);
   }
   if (!__syncthreads_or(!ok)) {
@@ -374,11 +379,16 @@ __global__ void __launch_bounds__(NTA, 2)
         mma_f16(tmem + A_TM_D4, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
       mma_commit(bar_m3);
     }
+    GDN_KEYS_MARK(28);
     ok = mbar_wait(bar_m3, 0);
   }
+  GDN_KEYS_MARK(29);
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
-    // row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg -> record
+    // The record is assembled in shared memory regions the MMAs no longer
+    // read, then leaves in three bulk copies: [-W; Qt] over AW, [U; Pt V]
+    // over [K; Q], w * silu(z) over [Tb; Pt].
+    // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.
     float x[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -386,19 +396,45 @@ __global__ void __launch_bounds__(NTA, 2)
 #pragma unroll
       for (int j = 0; j < 32; ++j) x[j] = -x[j];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(rec + R_WQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+      for (int q = 0; q < 4; ++q) st_half8(smem + A_AW + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
     }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       tmem_ld32(lane_base + A_TM_D4 + wg * 64 + hh * 32, x);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(rec + R_UO + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+      for (int q = 0; q < 4; ++q) st_half8(smem + A_KQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+    }
+    // w * silu(z) in the chain's tile layout (value block ch / 8, row r, swizzled chunk)
+    if (gated) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
+        uint4 res;
+        __half2* r2 = reinterpret_cast<__half2*>(&res);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 zf = __bfloat1622float2(z2[q]);
+          r2[q] = __floats2half2_rn(wsm[ch * 8 + 2 * q] * silu_tanh(zf.x), wsm[ch * 8 + 2 * q + 1] * silu_tanh(zf.y));
+        }
+        *reinterpret_cast<uint4*>(smem + A_TBP + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store(rec + R_WQ, sb + A_AW, 32768);
+      bulk_store(rec + R_UO, sb + A_KQ, 32768);
+      if (gated) bulk_store(rec + R_ZW, sb + A_TBP, 16384);
+      bulk_commit();
+      bulk_wait_read();  // shared memory stays valid until the copies have read it
     }
   } else if (tid == 0) {
     atomicExch(&g_split_error, 1);
     mbar_wait(bar_load, 0, 100000000ull);
     mbar_wait(bar_m3, 0, 100000000ull);
   }
+  GDN_KEYS_MARK(30);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

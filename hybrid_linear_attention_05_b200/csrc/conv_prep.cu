@@ -5,7 +5,8 @@
 // core, and fp16 keeps three more significand bits than bf16 at the same size
 // and MMA rate (all of them are bounded: |q|, |k| <= 1 after the norm).
 //
-// One thread handles 8 consecutive channels of TPT consecutive tokens: it
+// One thread handles 8 consecutive channels of TPT consecutive tokens (all
+// TPT input rows are requested before the first is used): it
 // keeps the conv window of those channels in registers (the three previous
 // inputs, or the sequence's conv history before its first token), applies
 // the depthwise 4-tap conv and SiLU token by token, and for q / k heads joins
@@ -21,7 +22,35 @@
 
 namespace gdn {
 
-constexpr int TPT = 4;  // consecutive tokens per thread (sliding conv window)
+constexpr int TPT = 8;  // consecutive tokens per thread (sliding conv window)
+
+// Eight input elements kept as loaded (16 B of bf16, 32 B of fp32) until use,
+// so that all TPT rows of a thread can be in flight at once.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ void to_f(float* f) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = reinterpret_cast<const float4*>(p)[0];
+    b = reinterpret_cast<const float4*>(p)[1];
+  }
+  __device__ __forceinline__ void to_f(float* f) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
 
 template <typename T, typename TM, int D>
 __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
@@ -62,11 +91,11 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
       }
     }
     // the TPT new input rows, issued together
-    float xr[TPT][8];
+    Raw8<T> xr[TPT];
 #pragma unroll
     for (int k = 0; k < TPT; ++k) {
       const int t = min(t0 + k, p.T - 1);
-      load8(x + (size_t)t * Cc + c0, xr[k]);
+      xr[k].load(x + (size_t)t * Cc + c0);
     }
     // conv window before token t0 (positions t0-3 .. t0-1) of t0's sequence
     int n = seq_of_token(p.cu_seqlens, p.N, min(t0, p.T - 1));
@@ -104,17 +133,18 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
           for (int i = 0; i < 8; ++i)
             win[j][i] = hist ? ld_f(hist + (size_t)(c0 + i) * 3 + j) : 0.f;
       }
-      float y[8];
+      float xk[8], y[8];
+      xr[k].to_f(xk);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float acc = w[i][0] * win[0][i];
         acc = fmaf(w[i][1], win[1][i], acc);
         acc = fmaf(w[i][2], win[2][i], acc);
-        acc = fmaf(w[i][3], xr[k][i], acc);
+        acc = fmaf(w[i][3], xk[i], acc);
         y[i] = silu_f(acc);
         win[0][i] = win[1][i];
         win[1][i] = win[2][i];
-        win[2][i] = xr[k][i];
+        win[2][i] = xk[i];
       }
       if (is_qk) {
         float ss = 0.0f;
