@@ -29,10 +29,11 @@
 //       D   = [-W; Qt] S0^T                      (tensor cores)
 //       Vn  = D[0:64] + U,   O = D[64:128] + Pt V
 //       S^T = e^{gamma_L} S^T + K^T (diag(e^{gamma_L-gamma}) Vn)
-//     Threads owning Vn rows feed the state update; threads owning O rows
-//     reduce the per-token sums of squares of chunk c while the state moves
-//     on, and write chunk c's gated output during chunk c+1 from the
-//     w * silu(z) tile that the key-side kernel left in the record.
+//     Four warpgroups carry the state; a fifth (the output group) takes the
+//     O rows of each chunk as soon as its MMAs complete, adds Pt V, swaps
+//     per-token sums of squares with the other CTA and writes the gated
+//     output from the w * silu(z) tile that the key-side kernel left in the
+//     record, while the state moves on to the next chunks.
 // The algebra is the chunked (WY / UT transform) form of the recurrence, exact
 // in real arithmetic ("Qwen (text & vision-language)", Verified parity).
 // No TMA multicast is used.
@@ -52,7 +53,7 @@ __device__ int g_split_error = 0;  // nonzero: a bounded wait in a kernel of thi
 __device__ unsigned long long g_split_phase[32];
 #define GDN_SPLIT_MARK(k)                                               \
   do {                                                                  \
-    if (tid == 64) {                                                    \
+    if (tid == NCW + 64) {                                              \
       const long long t_ = clock64();                                   \
       atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
       t_prev = t_;                                                      \
@@ -449,7 +450,7 @@ template <int VS>
 struct ChainCfg {
   static constexpr int CL = D / VS;
   static constexpr int NA = VS / 64;                  // 64-wide value blocks
-  static constexpr int CW = VS / 4;                   // value columns per warpgroup
+  static constexpr int CW = VS / 4;                   // state columns per main warpgroup
   static constexpr int NST = VS == 64 ? 3 : 2;        // stages in the ring
   static constexpr uint32_t S_K = 0;                  // per stage: K tile (two dk halves, 16 KiB)
   static constexpr uint32_t S_WQ = 16384;             //   [-W; Qt] (32 KiB)
@@ -457,21 +458,25 @@ struct ChainCfg {
   static constexpr uint32_t S_VEC = S_UO + NA * 16384;
   static constexpr uint32_t STAGE = (S_VEC + 512 + 1023) / 1024 * 1024;
   static constexpr uint32_t S16 = NST * STAGE;        // fp16 S0^T (NA x 16 KiB); then decayed Vn (NA x 8 KiB)
-  static constexpr uint32_t ZT = S16 + NA * 16384;    // z of the pending chunk, then its output (NA x 8 KiB)
-  static constexpr uint32_t SSP = ZT + NA * 8192;     // per-token partial sums of squares [4][64]
-  static constexpr uint32_t OWN = SSP + 1024;         // this CTA's per-token sums [2][64]
-  static constexpr uint32_t XB = OWN + 512;           // the other CTA's per-token sums [2][64]
-  static constexpr uint32_t BAR = XB + 512;
+  static constexpr uint32_t ZT = S16 + NA * 16384;    // w * silu(z) of a chunk, then its output (NA x 8 KiB)
+  static constexpr uint32_t SSP = ZT + NA * 8192;     // this CTA's per-token half-row sums of squares [2][64]
+  static constexpr uint32_t XB = SSP + 512;           // the other CTA's half-row sums [2 buffers][2][64]
+  static constexpr uint32_t BAR = XB + 1024;
   static constexpr uint32_t SMEM = BAR + 128 + 1024;
   static constexpr uint32_t TM_S = 0, TM_D = VS;      // state, then two [Vn; O] accumulators
   static constexpr uint32_t TM_COLS = 3 * VS <= 256 ? 256 : 512;
   static_assert(SMEM <= 232448, "shared memory");
 };
-constexpr int NCW = 512;        // four warpgroups
-constexpr int NTB = NCW;
-constexpr int BAR_COMPUTE = 1;  // named barrier of the compute threads
-constexpr int BAR_OUT = 2;      // the 256 threads that own output rows
-constexpr int BAR_VN = 3;       // the 256 threads that own new-value rows
+// Warps 0..15: the state chain (four warpgroups; TMEM lane quarter = warp % 4).
+// Warps 16..23: the output group; warps 18, 19, 22 and 23 reach TMEM lanes
+// 64..127, where the O rows are: two threads per token row, half the
+// columns each.
+constexpr int NCW = 512;
+constexpr int NOG = 256;
+constexpr int NTB = NCW + NOG;
+constexpr int BAR_COMPUTE = 1;  // named barrier of the state-chain threads
+constexpr int BAR_OG = 2;       // the output group
+constexpr int BAR_VN = 3;       // the 256 state-chain threads that own new-value rows
 
 template <int CW>
 __device__ __forceinline__ void tmem_ldw(uint32_t taddr, float* v) {
@@ -481,7 +486,7 @@ template <int CW>
 __device__ __forceinline__ void tmem_stw(uint32_t taddr, const float* v) {
   if constexpr (CW == 16) tmem_st16(taddr, v); else tmem_st32(taddr, v);
 }
-// x[0..8q) += eight fp16 values at base + off, q times along swizzled 16-byte chunks
+// x[0..8) += eight fp16 values at base + off
 __device__ __forceinline__ void add_half8(const uint8_t* base, uint32_t off, float* x) {
   const uint4 u = *reinterpret_cast<const uint4*>(base + off);
   const __half2* h2 = reinterpret_cast<const __half2*>(&u);
@@ -501,12 +506,14 @@ __global__ void __launch_bounds__(NTB, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
-  float* ssp = reinterpret_cast<float*>(smem + G::SSP);
-  float* own = reinterpret_cast<float*>(smem + G::OWN);
   float* xb = reinterpret_cast<float*>(smem + G::XB);
+  float* ssp = reinterpret_cast<float*>(smem + G::SSP);
+  // bar_a[b], bar_x[b], bar_dfree[b] follow accumulator buffer b = chunk & 1: the state
+  // chain cannot finish chunk c + 2 in buffer b before the output group released
+  // chunk c, so nobody waits on these barriers more than one phase late
   const uint32_t bar_full = sb + G::BAR, bar_free = bar_full + 8 * NST, bar_a = bar_free + 8 * NST,
-                 bar_s = bar_a + 8, bar_x = bar_s + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR + 8 * (2 * NST + 4));
+                 bar_s = bar_a + 16, bar_x = bar_s + 8, bar_dfree = bar_x + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR + 8 * (2 * NST + 7));
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7, tl = tid & 127;
@@ -528,12 +535,15 @@ __global__ void __launch_bounds__(NTB, 1)
   if (tid == 0) {
     for (int k = 0; k < NST; ++k) {
       mbar_init(bar_full + 8 * k, 1);
-      mbar_init(bar_free + 8 * k, 1 + 256);  // the state-update MMAs and the output-row threads
+      mbar_init(bar_free + 8 * k, 1 + 128);  // the state-update MMAs and the 128 O-row threads
     }
     mbar_init(bar_a, 1);
+    mbar_init(bar_a + 8, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_x, 1);
     mbar_init(bar_x + 8, 1);
+    mbar_init(bar_dfree, 128);
+    mbar_init(bar_dfree + 8, 128);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -545,8 +555,10 @@ __global__ void __launch_bounds__(NTB, 1)
   if constexpr (CL > 1) cluster_sync();  // the other CTA's barriers exist before anyone arrives on them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  bool bad = false;  // uniform over the compute threads: a bounded wait gave up
-  int c = 0;
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#ifdef GDN_PHASE_TIMING
+  long long t_prev = clock64();
+#endif
 
   // thread LOADER streams K and the records: chunks 0 .. NST-1 up front, then
   // chunk c - 1 + NST once chunk c - 1 has released its stage
@@ -566,120 +578,31 @@ __global__ void __launch_bounds__(NTB, 1)
   if (tid == LOADER)
     for (int cc = 0; cc < NST && cc < nchunks; ++cc) issue_loads(cc);
 
-  {
-    // ----------------------------------------------------------- compute
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int col = wg * CW;                     // this thread's value columns in the slice
-    const int vcol = h * D + vs * VS + col;      // ... as columns of [T, Hv * d]
-    const uint32_t blk = (uint32_t)(col >> 6) * 16384;        // its 64-column block in S16 / [U; Pt V]
-    const int ch0 = (col & 63) >> 3;                          // its first 16-byte chunk in a block row
-    const bool orow = tl >= 64;                  // owns output row tl - 64 (else new-value row tl)
-    const int t = tl - 64;
-
-    // initial state: S^T[dk = tl][v] = S0[v][dk]
-    {
+  if (warp < NCW / 32) {
+    // ============================================ state chain (warps 0..15)
+    const int col = wg * CW;                            // this thread's state columns in the slice
+    const uint32_t blk = (uint32_t)(col >> 6) * 16384;  // their 64-column block in S16 / [U; Pt V]
+    const int ch0 = (col & 63) >> 3;                    // their first 16-byte chunk in a block row
+    {  // initial state: S^T[dk = tl][v] = S0[v][dk]
       float r[CW];
 #pragma unroll
       for (int j = 0; j < CW; ++j) r[j] = p.S0 ? p.S0[sbase + (size_t)(col + j) * D + tl] : 0.f;
       tmem_stw<CW>(lane_base + G::TM_S + col, r);
       tmem_wait_st();
     }
-
-#ifdef GDN_PHASE_TIMING
-    long long t_prev = clock64();
-#endif
-    // w * silu(z) tile: output-row thread io copies (and later stores) the
-    // 16-byte chunks at tile offsets (io + 256 k) * 16; the record holds the
-    // tile in this layout, so both global transfers are coalesced
-    constexpr int ZK = 64 * (VS / 8) / 256;
-    const int io = wg * 64 + t;
-    auto z_copy = [&](int cc) {
-      const uint8_t* src = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC + R_ZW + vs * NA * 8192;
-#pragma unroll
-      for (int k = 0; k < ZK; ++k) {
-        const uint32_t pos = (uint32_t)(io + 256 * k) * 16;
-        cp_async16(sb + G::ZT + pos, src + pos, 16u);
-      }
-      cp_async_commit();
-    };
-
-    // gated output of chunk co (output-row threads): its O rows were
-    // completed and their sums of squares published during chunk co; the
-    // other CTA's sums arrive on bar_x, z waits in the tile
-    float o[CW];  // O rows of the chunk whose output is pending (plus Pt V)
-#pragma unroll
-    for (int j = 0; j < CW; ++j) o[j] = 0.f;
-    auto finish_output = [&](int co) -> bool {
-      bool okk = true;
-      const int bo = co & 1;
-      const int c0o = bos + co * C, Lo = min(C, eos - c0o);
-      GDN_SPLIT_MARK(16);
-      if (norm_out) {
-        float tot = own[bo * 64 + t];
-        if constexpr (CL > 1) {
-          okk = mbar_wait_cluster(bar_x + 8 * bo, (uint32_t)(co >> 1) & 1u);
-          tot += xb[bo * 64 + t];
-        }
-        const float ri = rsqrtf(tot * (1.0f / D) + p.eps_norm);
-        GDN_SPLIT_MARK(17);
-#pragma unroll
-        for (int q = 0; q < CW / 8; ++q) {
-          uint4* zq = reinterpret_cast<uint4*>(smem + G::ZT + (blk >> 1) + swz(t, ch0 + q));
-          const uint4 zv = *zq;
-          const __half2* z2 = reinterpret_cast<const __half2*>(&zv);
-          uint4 res;
-          __nv_bfloat162* r2 = reinterpret_cast<__nv_bfloat162*>(&res);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 zf = __half22float2(z2[e]);
-            r2[e] = __floats2bfloat162_rn(o[q * 8 + 2 * e] * ri * zf.x, o[q * 8 + 2 * e + 1] * ri * zf.y);
-          }
-          *zq = res;  // the output over its own w * silu(z)
-        }
-        GDN_SPLIT_MARK(18);
-        bar_named(BAR_OUT, 256);
-        GDN_SPLIT_MARK(19);
-        uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0o * p.Hv * D + h * D + vs * VS) * 2;
-#pragma unroll
-        for (int k = 0; k < ZK; ++k) {
-          const uint32_t pos = (uint32_t)(io + 256 * k) * 16;
-          const int r = (pos & 8191) >> 7, ch = (int)(pos >> 13) * 8 + ((int)((pos >> 4) & 7) ^ (r & 7));
-          if (r < Lo)
-            *reinterpret_cast<uint4*>(obase + ((size_t)r * p.Hv * D + ch * 8) * 2) =
-                *reinterpret_cast<const uint4*>(smem + G::ZT + pos);
-        }
-        // the next chunk's z over the chunks this thread just stored
-        if (co + 1 < nchunks) z_copy(co + 1);
-        GDN_SPLIT_MARK(20);
-      } else if (t < Lo) {
-        float* dst = p.o_raw + (size_t)(c0o + t) * p.Hv * D + vcol;
-#pragma unroll
-        for (int q = 0; q < CW / 4; ++q)
-          *reinterpret_cast<float4*>(dst + q * 4) = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      }
-      return okk;
-    };
-    if (norm_out && orow) z_copy(0);
-
-    bool ok = true;
+    bool ok = true, bad = false;
+    int c = 0;
     for (; c < nchunks; ++c) {
       const int s = c % NST, b = c & 1;
-      const int c0 = bos + c * C;
-      const int L = min(C, eos - c0);
       uint8_t* stp = smem + s * G::STAGE;
       const uint32_t st = sb + s * G::STAGE;
       const float* vec = reinterpret_cast<const float*>(stp + G::S_VEC);
-
-      // the previous chunk's z (copied during that chunk) is in the tile once
-      // every output-row thread has waited here and passed the barrier below
-      if (norm_out && orow) cp_async_wait_all();
       ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;
       GDN_SPLIT_PHASE(0);
-      // state -> fp16 operand, then S *= e^{gamma_L} in TMEM
       if (c > 0) ok = mbar_wait(bar_s, (uint32_t)(c - 1) & 1u) && ok;
       tc_fence_after();
       GDN_SPLIT_PHASE(1);
-      {
+      {  // state -> fp16 operand, then S *= e^{gamma_L} in TMEM
         const float egL = vec[64];
         float r[CW];
         tmem_ldw<CW>(lane_base + G::TM_S + col, r);
@@ -695,7 +618,7 @@ __global__ void __launch_bounds__(NTB, 1)
       if (bar_named_or(BAR_COMPUTE, NCW, !ok)) { bad = true; break; }
       GDN_SPLIT_PHASE(2);
       if (tid == LOADER && c >= 1 && c - 1 + NST < nchunks) {
-        // the state MMAs of chunk c-1 are done; its output rows arrived in its iteration
+        // the state MMAs of chunk c-1 are done; its O rows were read right after them
         const int cc = c - 1 + NST;
         if (mbar_wait(bar_free + 8 * (cc % NST), (uint32_t)(cc / NST - 1) & 1u))
           issue_loads(cc);
@@ -704,27 +627,29 @@ __global__ void __launch_bounds__(NTB, 1)
       }
       if (warp == 0) {  // D = [-W; Qt] S0^T (descriptors warp-uniform, one lane issues)
         tc_fence_after();
+        // D[b] was last read by the output group for chunk c - 2
+        bool go = ok;
+        if (c >= 2) go = mbar_wait(bar_dfree + 8 * b, (uint32_t)((c >> 1) - 1) & 1u) && go;
+        tc_fence_after();
         constexpr uint32_t id = idesc_f16(128, VS, false, true);
         const uint64_t da = sdesc_sw128(st + G::S_WQ, 16, 1024);
         const uint64_t db = sdesc_sw128(sb + G::S16, 16384, 1024);
-        if (elect_one()) {
+        if (go && elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16(tmem + G::TM_D + b * VS, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
                     sdesc_add(db, kk * 2048), id, kk > 0);
-          mma_commit(bar_a);
+          mma_commit(bar_a + 8 * b);
         }
         __syncwarp();
+        ok = go;
       }
-      // meanwhile: the previous chunk's gated output
-      if (c > 0 && orow) ok = finish_output(c - 1) && ok;
-
-      GDN_SPLIT_PHASE(3);  // output rows: the previous chunk's output
-      ok = mbar_wait(bar_a, (uint32_t)c & 1u) && ok;
-      tc_fence_after();
-      GDN_SPLIT_PHASE(4);
-      if (!orow) {
+      GDN_SPLIT_PHASE(3);
+      if (tl < 64) {
         // Vn = D + U, decayed to the chunk end -> B operand of the state update (over S16)
+        ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
+        tc_fence_after();
+        GDN_SPLIT_PHASE(4);
         float x[CW];
         tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, x);
 #pragma unroll
@@ -738,7 +663,7 @@ __global__ void __launch_bounds__(NTB, 1)
         tc_fence_before();
         ok = !bar_named_or(BAR_VN, 256, !ok);
         GDN_SPLIT_PHASE(5);
-        if (warp == 0 && ok) {  // S^T += K^T Vts; with the output rows' arrivals the stage is free
+        if (warp == 0 && ok) {  // S^T += K^T Vts; with the O-row threads' arrivals the stage is free
           tc_fence_after();
           constexpr uint32_t id = idesc_f16(128, VS, true, true);
           const uint64_t da = sdesc_sw128(st + G::S_K, TILE, 1024);
@@ -752,41 +677,10 @@ __global__ void __launch_bounds__(NTB, 1)
           }
           __syncwarp();
         }
-      } else {
-        // O = D + Pt V, kept in registers until the next chunk writes it out;
-        // per-token sum of squares -> this CTA's total and the other CTA
-        tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, o);
-#pragma unroll
-        for (int q = 0; q < CW / 8; ++q) add_half8(stp + G::S_UO + blk, swz(tl, ch0 + q), o + q * 8);
-        mbar_arrive(bar_free + 8 * s);
-        if (norm_out) {
-          float ps = 0.f;
-#pragma unroll
-          for (int j = 0; j < CW; ++j) ps = fmaf(o[j], o[j], ps);
-          ssp[wg * 64 + t] = ps;
-          GDN_SPLIT_PHASE(5);
-          bar_named(BAR_OUT, 256);
-          GDN_SPLIT_PHASE(6);
-          if (wg == 0) {
-            const float tot = (ssp[t] + ssp[64 + t]) + (ssp[128 + t] + ssp[192 + t]);
-            own[b * 64 + t] = tot;
-            if constexpr (CL > 1) {
-              const uint32_t peer = (uint32_t)(vs ^ 1);
-              st_async_f32(mapa_shared(sb + G::XB + (uint32_t)(b * 64 + t) * 4, peer), tot,
-                           mapa_shared(bar_x + 8 * b, peer));
-              if (t == 0) mbar_arrive_expect_tx(bar_x + 8 * b, 64 * 4);  // the other CTA's sums of this chunk
-            }
-          }
-        }
-        GDN_SPLIT_PHASE(7);
       }
     }
     if (!bad) {
-      bool okk = true;
-      if (norm_out && orow) cp_async_wait_all();
-      bar_named(BAR_COMPUTE, NCW);  // the last chunk's z tile is complete
-      if (orow) okk = finish_output(nchunks - 1);
-      okk = mbar_wait(bar_s, (uint32_t)(nchunks - 1) & 1u) && okk;
+      const bool okk = mbar_wait(bar_s, (uint32_t)(nchunks - 1) & 1u);
       tc_fence_after();
       if (!okk) {
         atomicExch(&g_split_error, 1);
@@ -797,14 +691,139 @@ __global__ void __launch_bounds__(NTB, 1)
         for (int j = 0; j < CW; ++j) p.S_out[sbase + (size_t)(col + j) * D + tl] = r[j];
       }
     } else if (tid == 0) {
-      // let the copies and MMAs in flight finish before the CTA leaves (the
-      // output-row threads drain their own z copies below)
+      // let the copies and MMAs in flight finish before the CTA leaves
       atomicExch(&g_split_error, 1);
       for (int k = 0; k < NST && c + k < nchunks; ++k)
         mbar_wait(bar_full + 8 * ((c + k) % NST), (uint32_t)((c + k) / NST) & 1u, 100000000ull);
       if (c > 0) mbar_wait(bar_s, (uint32_t)(c - 1) & 1u, 100000000ull);
     }
-    if (norm_out && orow) cp_async_wait_all();
+  } else {
+    // ========================================== output group (warps 16..19)
+    // Thread og owns the 16-byte chunks (og + NOG k) * 16 of the w * silu(z)
+    // tile for the copies in and the output stores; the O-row threads (warps
+    // 18, 19, 22, 23) own half of token row t each.
+    const int og = tid - NCW;
+    const bool orow = (warp & 3) >= 2;
+    const int t = (og & 127) - 64;       // token row (O-row threads)
+    const int half = og >> 7;            // which half of the columns
+    constexpr int HV = VS / 2;
+    const int hc = half * HV;
+    constexpr int ZK = NA * 8192 / 16 / NOG;
+    auto z_copy = [&](int cc) {
+      const uint8_t* src = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC + R_ZW + vs * NA * 8192;
+#pragma unroll
+      for (int k = 0; k < ZK; ++k) {
+        const uint32_t pos = (uint32_t)(og + NOG * k) * 16;
+        cp_async16(sb + G::ZT + pos, src + pos, 16u);
+      }
+      cp_async_commit();
+    };
+    if (norm_out) z_copy(0);
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % NST, b = c & 1;
+      const int c0 = bos + c * C, L = min(C, eos - c0);
+      const uint8_t* stp = smem + s * G::STAGE;
+      const uint32_t dcol = G::TM_D + b * VS;
+      float ss = 0.f;
+      if (orow) {
+        // O = D + Pt V, back into TMEM, and its sum of squares over this CTA's columns
+        ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;  // the stage's copies are seen here too
+        ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
+        tc_fence_after();
+        GDN_SPLIT_MARK(16);
+#pragma unroll 1
+        for (int j0 = hc; j0 < hc + HV; j0 += 32) {
+          float o[32];
+          tmem_ld32(lane_base + dcol + j0, o);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            add_half8(stp + G::S_UO + (j0 >> 6) * 16384, swz(64 + t, ((j0 & 63) >> 3) + q), o + q * 8);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
+          tmem_st32(lane_base + dcol + j0, o);
+          tmem_wait_st();
+        }
+        mbar_arrive(bar_free + 8 * s);  // Pt V read
+        if (norm_out) {
+          ssp[half * 64 + t] = ss;
+          if constexpr (CL > 1) {
+            const uint32_t peer = (uint32_t)(vs ^ 1);
+            st_async_f32(mapa_shared(sb + G::XB + (uint32_t)((b * 2 + half) * 64 + t) * 4, peer), ss,
+                         mapa_shared(bar_x + 8 * b, peer));
+            if (og == 64) mbar_arrive_expect_tx(bar_x + 8 * b, 128 * 4);  // the other CTA's sums of this chunk
+          }
+        }
+        GDN_SPLIT_MARK(17);
+      }
+      if (norm_out) {
+        cp_async_wait_all();
+        bar_named(BAR_OG, NOG);  // the chunk's w * silu(z) tile is complete
+        if (orow) {
+          ss = ssp[t] + ssp[64 + t];
+          if constexpr (CL > 1) {
+            ok = mbar_wait_cluster(bar_x + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
+            ss += xb[(b * 2) * 64 + t] + xb[(b * 2 + 1) * 64 + t];
+          }
+          GDN_SPLIT_MARK(18);
+          const float ri = rsqrtf(ss * (1.0f / D) + p.eps_norm);
+#pragma unroll 1
+          for (int j0 = hc; j0 < hc + HV; j0 += 32) {
+            float o[32];
+            tmem_ld32(lane_base + dcol + j0, o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4* zq = reinterpret_cast<uint4*>(smem + G::ZT + (j0 >> 6) * 8192 + swz(t, ((j0 & 63) >> 3) + q));
+              const uint4 zv = *zq;
+              const __half2* z2 = reinterpret_cast<const __half2*>(&zv);
+              uint4 res;
+              __nv_bfloat162* r2 = reinterpret_cast<__nv_bfloat162*>(&res);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 zf = __half22float2(z2[e]);
+                r2[e] = __floats2bfloat162_rn(o[q * 8 + 2 * e] * ri * zf.x, o[q * 8 + 2 * e + 1] * ri * zf.y);
+              }
+              *zq = res;  // the output over its own w * silu(z)
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_dfree + 8 * b);  // D[b] read for the last time
+          GDN_SPLIT_MARK(19);
+        }
+        if (bar_named_or(BAR_OG, NOG, !ok)) { ok = false; break; }  // the output tile is complete
+        uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv * D + h * D + vs * VS) * 2;
+#pragma unroll
+        for (int k = 0; k < ZK; ++k) {
+          const uint32_t pos = (uint32_t)(og + NOG * k) * 16;
+          const int r = (pos & 8191) >> 7, chn = (int)(pos >> 13) * 8 + ((int)((pos >> 4) & 7) ^ (r & 7));
+          if (r < L)
+            *reinterpret_cast<uint4*>(obase + ((size_t)r * p.Hv * D + chn * 8) * 2) =
+                *reinterpret_cast<const uint4*>(smem + G::ZT + pos);
+        }
+        // the next chunk's w * silu(z) over the chunks this thread just stored
+        if (c + 1 < nchunks) z_copy(c + 1);
+        GDN_SPLIT_MARK(20);
+      } else {
+        if (orow) {
+#pragma unroll 1
+          for (int j0 = hc; j0 < hc + HV; j0 += 32) {
+            float o[32];
+            tmem_ld32(lane_base + dcol + j0, o);
+            if (t < L) {
+              float* dst = p.o_raw + (size_t)(c0 + t) * p.Hv * D + h * D + vs * VS + j0;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(dst + q * 4) = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_dfree + 8 * b);
+        }
+        if (bar_named_or(BAR_OG, NOG, !ok)) { ok = false; break; }
+      }
+    }
+    if (!ok) atomicExch(&g_split_error, 1);
+    if (norm_out) cp_async_wait_all();
   }
   tc_fence_before();
   __syncthreads();
