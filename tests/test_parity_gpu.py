@@ -63,6 +63,7 @@ def run_prefill(inp, impl, chunk, guard=True):
         pytest.skip("implementation not available for this shape")
     assert status == gdn.GDN_OK, gdn.status_string(status)
     torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0, "a bounded wait inside a kernel gave up"
     if guard:
         for name in ("out", "final_state", "conv_state_out"):
             big = getattr(bufs, name + "_guard")
@@ -119,6 +120,17 @@ def test_9b_shapes_gqa_varlen(impl):
     code, chunk = IMPLS[impl]
     inp = make_prefill(P9B, seqlens=(200, 1, 2, 3, 64, 0, 129), with_conv_state=True)
     bufs = run_prefill(inp, code, chunk)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("seqlens", [(200, 0), (3, 190), (64, 129)])
+def test_split_value_pairs_varlen(seqlens):
+    """Two-kernel path with few (value head, sequence) chains, where each chain
+    runs as a pair of CTAs over half the value columns: GQA, initial states,
+    conv history, an empty sequence, one shorter than the conv window, and
+    sequences ending on and off a chunk boundary."""
+    inp = make_prefill(P9B, seqlens=seqlens, with_conv_state=True)
+    bufs = run_prefill(inp, gdn.GDN_IMPL_TC_SPLIT, 64)
     check_full(inp, bufs)
 
 
