@@ -462,7 +462,7 @@ struct ChainCfg {
   static constexpr uint32_t SSP = ZT + NA * 8192;     // this CTA's per-token half-row sums of squares [2][64]
   static constexpr uint32_t XB = SSP + 512;           // the other CTA's half-row sums [2 buffers][2][64]
   static constexpr uint32_t BAR = XB + 1024;
-  static constexpr uint32_t SMEM = BAR + 128 + 1024;
+  static constexpr uint32_t SMEM = BAR + 256 + 1024;
   static constexpr uint32_t TM_S = 0, TM_D = VS;      // state, then two [Vn; O] accumulators
   static constexpr uint32_t TM_COLS = 3 * VS <= 256 ? 256 : 512;
   static_assert(SMEM <= 232448, "shared memory");
@@ -508,12 +508,12 @@ __global__ void __launch_bounds__(NTB, 1)
   const uint32_t sb = smem_u32(smem);
   float* xb = reinterpret_cast<float*>(smem + G::XB);
   float* ssp = reinterpret_cast<float*>(smem + G::SSP);
-  // bar_a[b], bar_x[b], bar_dfree[b] follow accumulator buffer b = chunk & 1: the state
+  // bar_a[b], bar_s[b], bar_x[b], bar_dfree[b] follow accumulator buffer b = chunk & 1: the state
   // chain cannot finish chunk c + 2 in buffer b before the output group released
   // chunk c, so nobody waits on these barriers more than one phase late
   const uint32_t bar_full = sb + G::BAR, bar_free = bar_full + 8 * NST, bar_a = bar_free + 8 * NST,
-                 bar_s = bar_a + 16, bar_x = bar_s + 8, bar_dfree = bar_x + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR + 8 * (2 * NST + 7));
+                 bar_s = bar_a + 16, bar_x = bar_s + 16, bar_dfree = bar_x + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR + 8 * (2 * NST + 8));
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7, tl = tid & 127;
@@ -540,6 +540,7 @@ __global__ void __launch_bounds__(NTB, 1)
     mbar_init(bar_a, 1);
     mbar_init(bar_a + 8, 1);
     mbar_init(bar_s, 1);
+    mbar_init(bar_s + 8, 1);
     mbar_init(bar_x, 1);
     mbar_init(bar_x + 8, 1);
     mbar_init(bar_dfree, 128);
@@ -568,6 +569,9 @@ __global__ void __launch_bounds__(NTB, 1)
     const int row = bos + cc * C;
     const uint32_t bar = bar_full + 8 * s, st = sb + s * G::STAGE;
     const uint8_t* rec = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC;
+#ifdef GDN_PHASE_TIMING
+    reinterpret_cast<long long*>(smem + G::BAR + 8 * (2 * NST + 9))[s] = clock64();
+#endif
     mbar_arrive_expect_tx(bar, 2 * TILE + 32768 + NA * 16384 + 512);
     tma_load_2d(st + G::S_K, &tm_k, hk * D, row, bar);
     tma_load_2d(st + G::S_K + TILE, &tm_k, hk * D + 64, row, bar);
@@ -598,9 +602,23 @@ __global__ void __launch_bounds__(NTB, 1)
       const uint32_t st = sb + s * G::STAGE;
       const float* vec = reinterpret_cast<const float*>(stp + G::S_VEC);
       ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;
+#ifdef GDN_PHASE_TIMING
+      if (tid == 0) {  // cycles from the issue of this stage's copies to their arrival being seen
+        atomicAdd(&g_split_phase[14], (unsigned long long)(clock64() - reinterpret_cast<volatile long long*>(
+                                                                          smem + G::BAR + 8 * (2 * NST + 9))[s]));
+        atomicAdd(&g_split_phase[15], 1ull);
+      }
+#endif
       GDN_SPLIT_PHASE(0);
-      if (c > 0) ok = mbar_wait(bar_s, (uint32_t)(c - 1) & 1u) && ok;
+      if (c > 0) ok = mbar_wait(bar_s + 8 * (b ^ 1), (uint32_t)((c - 1) >> 1) & 1u) && ok;
       tc_fence_after();
+      // the stage of chunk c - 1 is free once its output rows have also read it:
+      // refill it now if they have, else after the barrier below
+      bool loads_due = tid == LOADER && c >= 1 && c - 1 + NST < nchunks;
+      if (loads_due && mbar_try_wait(bar_free + 8 * ((c - 1) % NST), (uint32_t)((c - 1) / NST) & 1u)) {
+        issue_loads(c - 1 + NST);
+        loads_due = false;
+      }
       GDN_SPLIT_PHASE(1);
       {  // state -> fp16 operand, then S *= e^{gamma_L} in TMEM
         const float egL = vec[64];
@@ -617,7 +635,7 @@ __global__ void __launch_bounds__(NTB, 1)
       tc_fence_before();
       if (bar_named_or(BAR_COMPUTE, NCW, !ok)) { bad = true; break; }
       GDN_SPLIT_PHASE(2);
-      if (tid == LOADER && c >= 1 && c - 1 + NST < nchunks) {
+      if (loads_due) {
         // the state MMAs of chunk c-1 are done; its O rows were read right after them
         const int cc = c - 1 + NST;
         if (mbar_wait(bar_free + 8 * (cc % NST), (uint32_t)(cc / NST - 1) & 1u))
@@ -672,7 +690,7 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_f16(tmem + G::TM_S, sdesc_add(da, kk * 2048), sdesc_add(db, kk * 2048), id, 1);
-            mma_commit(bar_s);
+            mma_commit(bar_s + 8 * b);
             mma_commit(bar_free + 8 * s);
           }
           __syncwarp();
@@ -680,7 +698,7 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
     if (!bad) {
-      const bool okk = mbar_wait(bar_s, (uint32_t)(nchunks - 1) & 1u);
+      const bool okk = mbar_wait(bar_s + 8 * ((nchunks - 1) & 1), (uint32_t)((nchunks - 1) >> 1) & 1u);
       tc_fence_after();
       if (!okk) {
         atomicExch(&g_split_error, 1);
@@ -695,7 +713,7 @@ __global__ void __launch_bounds__(NTB, 1)
       atomicExch(&g_split_error, 1);
       for (int k = 0; k < NST && c + k < nchunks; ++k)
         mbar_wait(bar_full + 8 * ((c + k) % NST), (uint32_t)((c + k) / NST) & 1u, 100000000ull);
-      if (c > 0) mbar_wait(bar_s, (uint32_t)(c - 1) & 1u, 100000000ull);
+      if (c > 0) mbar_wait(bar_s + 8 * ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, 100000000ull);
     }
   } else {
     // ========================================== output group (warps 16..19)
@@ -730,6 +748,9 @@ __global__ void __launch_bounds__(NTB, 1)
         // O = D + Pt V, back into TMEM, and its sum of squares over this CTA's columns
         ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;  // the stage's copies are seen here too
         ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
+        // start once the state update of this chunk is under way: the new-value
+        // threads' TMEM reads come first
+        ok = mbar_wait(bar_s + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
         tc_fence_after();
         GDN_SPLIT_MARK(16);
 #pragma unroll 1
