@@ -303,12 +303,19 @@ def run_ours(args, rank, world, local_rank):
     core_avg_s = statistics.mean(core_ms) * 1e-3
     hbm = peaks["hbm_gbs"]
     # AUTO with room for the records runs the two-kernel tensor-core core
-    # (chunk_keys_kernel + chunk_chain_kernel); the library's core events
-    # bracket both launches
+    # (chunk_keys_kernel, then the chains: with segmented chains the segment
+    # maps and the scan of their start states come first); the library's core
+    # events bracket all of its launches
     split = dp.chunk == 64
+    nseg = gdn.gdn_prefill_auto_segments(gdn.make_dims(wp.Hk, wp.Hv, wp.d), inp.N, inp.T) if split else 1
+    core_launches = (2 + (2 if nseg > 1 else 0)) if split else 1
     core_src = "chunk_tc_split.cu" if split else "chunk_simt.cu"
+    core_name = "chunk_simt_kernel"
+    if split:
+        core_name = ("chunk_keys_kernel + chunk_chain_kernel<xfer> + seg_scan_kernel + chunk_chain_kernel"
+                     " (%d segments)" % nseg if nseg > 1 else "chunk_keys_kernel + chunk_chain_kernel")
     roofline = {
-        "kernel": "chunk_keys_kernel + chunk_chain_kernel" if split else "chunk_simt_kernel",
+        "kernel": core_name,
         "bound": "hbm",
         "achieved": cnt["core_bytes"] / core_avg_s / 1e9,
         "peak": hbm,
@@ -411,8 +418,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "decode": decode,
         "e2e": e2e,
-        # conv_prep + the core (two kernels on the split path) per prefill step
-        "gpu_launches": (3 if split else 2) * args.steps,
+        # conv_prep + the core's launches per prefill step
+        "gpu_launches": (1 + core_launches) * args.steps,
         "clocks": clk.summary(),
     }
     return result, inp, dinp

@@ -89,7 +89,7 @@ class PrefillBuffers:
 
 
 def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[PrefillBuffers] = None,
-            core_events=None) -> PrefillOut:
+            core_events=None, segments: int = 0) -> PrefillOut:
     bufs = bufs or PrefillBuffers(dp)
     ev0, ev1 = (None, None) if core_events is None else (core_events[0].cuda_event,
                                                          core_events[1].cuda_event)
@@ -100,7 +100,7 @@ def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[Pre
         workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
         initial_state=dp.initial_state, final_state=bufs.final_state,
         conv_state_in=dp.conv_state_in, conv_state_out=bufs.conv_state_out, impl=impl,
-        core_event_begin=ev0, core_event_end=ev1)
+        core_event_begin=ev0, core_event_end=ev1, segments=segments)
     return PrefillOut(bufs.out, bufs.final_state, bufs.conv_state_out)
 
 

@@ -34,10 +34,21 @@
 //     per-token sums of squares with the other CTA and writes the gated
 //     output from the w * silu(z) tile that the key-side kernel left in the
 //     record, while the state moves on to the next chunks.
+//  3. Segmented chains (few heads x sequences): one serial chain per (value
+//     head, sequence) leaves most SMs idle and takes one chain step per chunk.
+//     Each chunk maps the state affinely, S -> S M_c + R_c with
+//       M_c = e^{gamma_L} I - W^T diag(e^{gamma_L - gamma}) K,
+//       R_c = U^T diag(e^{gamma_L - gamma}) K,
+//     so the chunks are cut into segments and chunk_chain_kernel<D, true> runs
+//     every segment but the last at once, twice: from S = I with U = 0 (which
+//     leaves the segment's M) and from S = 0 (its R).  seg_scan_kernel then
+//     walks the segments, S_start(s+1) = S_start(s) M_s + R_s in fp32, and the
+//     output chains run all segments at once from their start states.
 // The algebra is the chunked (WY / UT transform) form of the recurrence, exact
 // in real arithmetic ("Qwen (text & vision-language)", Verified parity).
 // No TMA multicast is used.
 #include <cuda.h>
+#include <math.h>
 
 #include "gdn_internal.h"
 #include "tc_chunk_common.cuh"
@@ -108,6 +119,8 @@ constexpr uint32_t REC = 82432;
 __device__ __forceinline__ int slot_start(const int32_t* cu, int n, int T) {
   return clampi(__ldg(cu + n), 0, T) / C + n;
 }
+// First chunk of segment s when nch chunks are cut into P segments.
+__device__ __forceinline__ int seg_lo(int nch, int s, int P) { return (int)(((long long)nch * s) / P); }
 
 // ===================================================== key-side kernel
 constexpr int NTA = 256;
@@ -498,11 +511,17 @@ __device__ __forceinline__ void add_half8(const uint8_t* base, uint32_t off, flo
   }
 }
 
-template <int VS>
-__global__ void __launch_bounds__(NTB, 1)
+// XFER = false: the output chain of one segment (the whole sequence when
+// p.nseg == 1) of one (value head, sequence), CL CTAs over the value columns.
+// XFER = true: the affine map of one segment that is not the last, one CTA
+// per role: role 0 runs the chain from S = I with U = 0 and leaves M, role 1
+// from S = 0 and leaves R; neither writes outputs (no output group).
+template <int VS, bool XFER>
+__global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
     chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_k, ChunkParams p) {
   using G = ChainCfg<VS>;
   constexpr int CL = G::CL, NA = G::NA, CW = G::CW, NST = G::NST;
+  static_assert(!XFER || CL == 1, "a transfer chain owns whole state rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -517,25 +536,51 @@ __global__ void __launch_bounds__(NTB, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7, tl = tid & 127;
-  const int h = blockIdx.x / CL, vs = blockIdx.x % CL, n = blockIdx.y;
+  const int P = p.nseg;
+  const int h = XFER ? (int)blockIdx.x >> 1 : (int)blockIdx.x / CL;
+  const int vs = XFER ? 0 : (int)blockIdx.x % CL;
+  const int role = XFER ? (int)blockIdx.x & 1 : 1;  // 0: the map M (from S = I, U = 0)
+  const int n = XFER ? (int)blockIdx.y / (P - 1) : (int)blockIdx.y / P;
+  const int sg = XFER ? (int)blockIdx.y % (P - 1) : (int)blockIdx.y % P;
   const int hk = h / (p.Hv / p.Hk);
-  const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
-  const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
-  const int nchunks = (eos - bos + C - 1) / C;
-  const size_t sbase = ((size_t)n * p.Hv + h) * D * D + (size_t)vs * VS * D;  // first row of the slice
-  const bool norm_out = p.out != nullptr;
+  const int bos0 = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
+  const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos0, p.T);
+  const int nch_all = (eos - bos0 + C - 1) / C;
+  const int cb = seg_lo(nch_all, sg, P);
+  const int nchunks = seg_lo(nch_all, sg + 1, P) - cb;  // chunks of this segment
+  const int bos = bos0 + cb * C;                          // its first token
+  const size_t hd = (size_t)D * D;
+  const size_t slice = (size_t)vs * VS * D;  // first state row of this CTA's slice
+  const size_t nh = (size_t)n * p.Hv + h;
+  // the state this CTA starts from (null: zero; transfer chains build theirs)
+  // and where its last state goes (null: nowhere)
+  auto start_state = [&]() -> const float* {
+    if (XFER) return nullptr;
+    if (P == 1) return p.S0 ? p.S0 + nh * hd + slice : nullptr;
+    return p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd + slice;
+  };
+  auto final_state = [&]() -> float* {
+    if (XFER) return p.seg_mr + ((((size_t)n * (P - 1) + sg) * p.Hv + h) * 2 + role) * hd;
+    return sg == P - 1 && p.S_out ? p.S_out + nh * hd + slice : nullptr;
+  };
+  const bool norm_out = !XFER && p.out != nullptr;
+  const bool want_u = !XFER || role == 1;  // the chain adds U to its new values
 
-  if (nchunks == 0) {  // empty sequence: the state passes through (every CTA of the cluster returns here)
-    if (p.S_out)
-      for (int idx = tid; idx < VS * D; idx += NTB) p.S_out[sbase + idx] = p.S0 ? p.S0[sbase + idx] : 0.f;
+  if (nchunks == 0) {
+    // empty segment; the last one is empty only for an empty sequence, whose
+    // state passes through (every CTA of the cluster returns here)
+    const float* Sin = start_state();
+    float* Sfin = final_state();
+    if (!XFER && Sfin)
+      for (int idx = tid; idx < VS * D; idx += NTB) Sfin[idx] = Sin ? Sin[idx] : 0.f;
     return;
   }
-  const int slot0 = slot_start(p.cu_seqlens, n, p.T);
+  const int slot0 = slot_start(p.cu_seqlens, n, p.T) + cb;
 
   if (tid == 0) {
     for (int k = 0; k < NST; ++k) {
       mbar_init(bar_full + 8 * k, 1);
-      mbar_init(bar_free + 8 * k, 1 + 128);  // the state-update MMAs and the 128 O-row threads
+      mbar_init(bar_free + 8 * k, XFER ? 1 : 1 + 128);  // the state-update MMAs (and the 128 O-row threads)
     }
     mbar_init(bar_a, 1);
     mbar_init(bar_a + 8, 1);
@@ -572,25 +617,42 @@ __global__ void __launch_bounds__(NTB, 1)
 #ifdef GDN_PHASE_TIMING
     reinterpret_cast<long long*>(smem + G::BAR + 8 * (2 * NST + 9))[s] = clock64();
 #endif
-    mbar_arrive_expect_tx(bar, 2 * TILE + 32768 + NA * 16384 + 512);
-    tma_load_2d(st + G::S_K, &tm_k, hk * D, row, bar);
-    tma_load_2d(st + G::S_K + TILE, &tm_k, hk * D + 64, row, bar);
-    bulk_load(st + G::S_WQ, rec + R_WQ, 32768, bar);
-    bulk_load(st + G::S_UO, rec + R_UO + vs * NA * 16384, NA * 16384, bar);
-    bulk_load(st + G::S_VEC, rec + R_VEC, 512, bar);
+    if constexpr (XFER) {
+      // only the -W rows (the first 64 of each dk atom) and the U rows (the
+      // first 64 of each value block); the MMA rows they leave stale are never read
+      mbar_arrive_expect_tx(bar, 2 * TILE + 16384 + (want_u ? 16384 : 0) + 512);
+      tma_load_2d(st + G::S_K, &tm_k, hk * D, row, bar);
+      tma_load_2d(st + G::S_K + TILE, &tm_k, hk * D + 64, row, bar);
+      bulk_load(st + G::S_WQ, rec + R_WQ, 8192, bar);
+      bulk_load(st + G::S_WQ + 16384, rec + R_WQ + 16384, 8192, bar);
+      if (want_u) {
+        bulk_load(st + G::S_UO, rec + R_UO, 8192, bar);
+        bulk_load(st + G::S_UO + 16384, rec + R_UO + 16384, 8192, bar);
+      }
+      bulk_load(st + G::S_VEC, rec + R_VEC, 512, bar);
+    } else {
+      mbar_arrive_expect_tx(bar, 2 * TILE + 32768 + NA * 16384 + 512);
+      tma_load_2d(st + G::S_K, &tm_k, hk * D, row, bar);
+      tma_load_2d(st + G::S_K + TILE, &tm_k, hk * D + 64, row, bar);
+      bulk_load(st + G::S_WQ, rec + R_WQ, 32768, bar);
+      bulk_load(st + G::S_UO, rec + R_UO + vs * NA * 16384, NA * 16384, bar);
+      bulk_load(st + G::S_VEC, rec + R_VEC, 512, bar);
+    }
   };
   if (tid == LOADER)
     for (int cc = 0; cc < NST && cc < nchunks; ++cc) issue_loads(cc);
 
-  if (warp < NCW / 32) {
+  if (XFER || warp < NCW / 32) {
     // ============================================ state chain (warps 0..15)
     const int col = wg * CW;                            // this thread's state columns in the slice
     const uint32_t blk = (uint32_t)(col >> 6) * 16384;  // their 64-column block in S16 / [U; Pt V]
     const int ch0 = (col & 63) >> 3;                    // their first 16-byte chunk in a block row
-    {  // initial state: S^T[dk = tl][v] = S0[v][dk]
+    {  // initial state: S^T[dk = tl][v] = S_start[v][dk]; I for the map M
+      const float* Sin = start_state();
       float r[CW];
 #pragma unroll
-      for (int j = 0; j < CW; ++j) r[j] = p.S0 ? p.S0[sbase + (size_t)(col + j) * D + tl] : 0.f;
+      for (int j = 0; j < CW; ++j)
+        r[j] = XFER ? (role == 0 && col + j == tl ? 1.f : 0.f) : (Sin ? Sin[(size_t)(col + j) * D + tl] : 0.f);
       tmem_stw<CW>(lane_base + G::TM_S + col, r);
       tmem_wait_st();
     }
@@ -647,7 +709,7 @@ __global__ void __launch_bounds__(NTB, 1)
         tc_fence_after();
         // D[b] was last read by the output group for chunk c - 2
         bool go = ok;
-        if (c >= 2) go = mbar_wait(bar_dfree + 8 * b, (uint32_t)((c >> 1) - 1) & 1u) && go;
+        if (!XFER && c >= 2) go = mbar_wait(bar_dfree + 8 * b, (uint32_t)((c >> 1) - 1) & 1u) && go;
         tc_fence_after();
         constexpr uint32_t id = idesc_f16(128, VS, false, true);
         const uint64_t da = sdesc_sw128(st + G::S_WQ, 16, 1024);
@@ -670,8 +732,10 @@ __global__ void __launch_bounds__(NTB, 1)
         GDN_SPLIT_PHASE(4);
         float x[CW];
         tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, x);
+        if (want_u) {
 #pragma unroll
-        for (int q = 0; q < CW / 8; ++q) add_half8(stp + G::S_UO + blk, swz(tl, ch0 + q), x + q * 8);
+          for (int q = 0; q < CW / 8; ++q) add_half8(stp + G::S_UO + blk, swz(tl, ch0 + q), x + q * 8);
+        }
         const float dec = vec[tl];
 #pragma unroll
         for (int j = 0; j < CW; ++j) x[j] *= dec;
@@ -700,13 +764,14 @@ __global__ void __launch_bounds__(NTB, 1)
     if (!bad) {
       const bool okk = mbar_wait(bar_s + 8 * ((nchunks - 1) & 1), (uint32_t)((nchunks - 1) >> 1) & 1u);
       tc_fence_after();
+      float* Sfin = final_state();
       if (!okk) {
         atomicExch(&g_split_error, 1);
-      } else if (p.S_out) {
+      } else if (Sfin) {
         float r[CW];
         tmem_ldw<CW>(lane_base + G::TM_S + col, r);
 #pragma unroll
-        for (int j = 0; j < CW; ++j) p.S_out[sbase + (size_t)(col + j) * D + tl] = r[j];
+        for (int j = 0; j < CW; ++j) Sfin[(size_t)(col + j) * D + tl] = r[j];
       }
     } else if (tid == 0) {
       // let the copies and MMAs in flight finish before the CTA leaves
@@ -715,8 +780,8 @@ __global__ void __launch_bounds__(NTB, 1)
         mbar_wait(bar_full + 8 * ((c + k) % NST), (uint32_t)((c + k) / NST) & 1u, 100000000ull);
       if (c > 0) mbar_wait(bar_s + 8 * ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, 100000000ull);
     }
-  } else {
-    // ========================================== output group (warps 16..19)
+  } else if constexpr (!XFER) {
+    // ========================================== output group (warps 16..23)
     // Thread og owns the 16-byte chunks (og + NOG k) * 16 of the w * silu(z)
     // tile for the copies in and the output stores; the O-row threads (warps
     // 18, 19, 22, 23) own half of token row t each.
@@ -855,6 +920,107 @@ __global__ void __launch_bounds__(NTB, 1)
   }
 }
 
+// ========================================================== segment scan
+// Start states of the segments of one (value head, sequence), SR state rows
+// per CTA, in fp32 on the CUDA cores: S_start(0) = S0 (or 0), then
+// S_start(s+1) = S_start(s) M_s + R_s for every segment s but the last (an
+// empty segment maps the state to itself).  The CTA keeps its rows
+// transposed in shared memory (sT[i][r]) and each M_s in a double buffer
+// filled by cp.async one segment ahead.  Thread (warp w, lane l) owns the 4 x
+// 4 tile rows 4 (l >> 3) .. +3, columns 4 (8 w + (l & 7)) .. +3: per index i
+// a warp reads 64 contiguous bytes of sT and 128 of M (one wavefront each)
+// for 16 FMAs.
+constexpr int SR = 16;                 // state rows per CTA
+constexpr int SCAN_THREADS = SR * 8;   // 4 x 4 outputs per thread
+constexpr uint32_t SCAN_SMEM = 2 * D * D * 4 + D * SR * 4 + 128;
+__global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
+  extern __shared__ uint8_t scan_raw[];
+  float* Mb = reinterpret_cast<float*>(scan_raw + ((128u - (smem_u32(scan_raw) & 127u)) & 127u));
+  float* sT = Mb + 2 * D * D;  // [D][SR]
+  const int P = p.nseg;
+  const int h = blockIdx.x / (D / SR), r0 = (blockIdx.x % (D / SR)) * SR;
+  const int n = blockIdx.y;
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int rr = (l >> 3) * 4, cc = (w * 8 + (l & 7)) * 4;  // this thread's tile within the CTA's rows
+  const size_t hd = (size_t)D * D;
+  const size_t nh = (size_t)n * p.Hv + h;
+  const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
+  const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
+  const int nch = (eos - bos + C - 1) / C;
+  auto nonempty = [&](int sg) { return seg_lo(nch, sg + 1, P) > seg_lo(nch, sg, P); };
+  auto map_of = [&](int sg) { return p.seg_mr + ((((size_t)n * (P - 1) + sg) * p.Hv + h) * 2) * hd; };
+  // next non-empty segment at or after sg that has a map (sg < P - 1), or P - 1
+  auto next_map = [&](int sg) {
+    while (sg < P - 1 && !nonempty(sg)) ++sg;
+    return sg;
+  };
+  auto prefetch = [&](int sg, int buf) {
+    const float* M = map_of(sg);
+    const uint32_t dst = smem_u32(Mb + buf * D * D);
+    for (int e = tid; e < D * D / 4; e += SCAN_THREADS) cp_async16(dst + e * 16, M + e * 4, 16u);
+    cp_async_commit();
+  };
+  int sg_next = next_map(0);
+  int buf = 0;
+  if (sg_next < P - 1) prefetch(sg_next, buf);
+
+  float acc[4][4];
+  {
+    const float* S0 = p.S0 ? p.S0 + nh * hd : nullptr;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 v = S0 ? *reinterpret_cast<const float4*>(S0 + (size_t)(r0 + rr + r) * D + cc)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[r][0] = v.x; acc[r][1] = v.y; acc[r][2] = v.z; acc[r][3] = v.w;
+    }
+  }
+  for (int sg = 0;; ++sg) {
+    float* dst = p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      *reinterpret_cast<float4*>(dst + (size_t)(r0 + rr + r) * D + cc) =
+          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    if (sg + 1 >= P) break;
+    if (sg != sg_next) continue;  // empty segment: the state passes through
+    // this segment's map: S <- S M + R
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) = make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
+    // R is added after the products, so its loads overlap them
+    const float* R = map_of(sg) + hd;
+    float4 rv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      rv[r] = __ldg(reinterpret_cast<const float4*>(R + (size_t)(r0 + rr + r) * D + cc));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    }
+    cp_async_wait_all();
+    __syncthreads();  // sT and this segment's M are complete
+    sg_next = next_map(sg + 1);
+    if (sg_next < P - 1) prefetch(sg_next, buf ^ 1);
+    const float* M = Mb + buf * D * D;
+#pragma unroll 4
+    for (int i = 0; i < D; ++i) {
+      const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
+      const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+      const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(sv[r], mv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      acc[r][0] += rv[r].x; acc[r][1] += rv[r].y; acc[r][2] += rv[r].z; acc[r][3] += rv[r].w;
+    }
+    __syncthreads();  // everyone is done with sT and this buffer
+    buf ^= 1;
+  }
+  cp_async_wait_all();
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -895,6 +1061,12 @@ size_t chunk_tc_split_record_bytes(int N, int T, int Hv) {
   return record_slots(N, T) * (size_t)Hv * REC;
 }
 
+size_t chunk_tc_split_seg_bytes(int N, int Hv) {
+  if ((long)N * Hv > kSegMaxChains) return 0;
+  // seg_mr [N][kSegMax-1][Hv][2][D][D] then seg_start [N][kSegMax][Hv][D][D]
+  return (size_t)N * Hv * (2 * (kSegMax - 1) + kSegMax) * D * D * sizeof(float);
+}
+
 namespace {
 
 int sm_count() {
@@ -910,16 +1082,19 @@ int sm_count() {
   return count;
 }
 
-template <int VS>
+// Launch the chains: the output chains of every segment (XFER = false), or
+// the transfer chains of every segment but the last (XFER = true, VS = D).
+template <int VS, bool XFER>
 cudaError_t launch_chain(const CUtensorMap& mk, const ChunkParams& p, cudaStream_t st) {
   using G = ChainCfg<VS>;
-  cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel<VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel<VS, XFER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)G::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)(G::CL * p.Hv), (unsigned)p.N, 1);
-  cfg.blockDim = dim3(NTB, 1, 1);
+  cfg.gridDim = XFER ? dim3((unsigned)(2 * p.Hv), (unsigned)(p.N * (p.nseg - 1)), 1)
+                     : dim3((unsigned)(G::CL * p.Hv), (unsigned)(p.N * p.nseg), 1);
+  cfg.blockDim = dim3(XFER ? NCW : NTB, 1, 1);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -929,13 +1104,15 @@ cudaError_t launch_chain(const CUtensorMap& mk, const ChunkParams& p, cudaStream
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<VS>, mk, p);
+  return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<VS, XFER>, mk, p);
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st) {
-  if (p.N == 0 || p.Hv == 0) return cudaSuccess;
+cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
+  if (p0.N == 0 || p0.Hv == 0) return cudaSuccess;
+  ChunkParams p = p0;
+  if (p.nseg < 1) p.nseg = 1;
   if (!p.rec) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
   memset(&mq, 0, sizeof(mq));
@@ -956,11 +1133,48 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  const int P = p.nseg;
+  if (P > 1) {
+    if (!p.seg_mr || !p.seg_start || P > kSegMax) return cudaErrorInvalidValue;
+    cudaError_t e = launch_chain<D, true>(mk, p, st);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCAN_SMEM);
+    if (e != cudaSuccess) return e;
+    seg_scan_kernel<<<dim3((unsigned)(p.Hv * (D / SR)), (unsigned)p.N), SCAN_THREADS, SCAN_SMEM, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   // Half-width value slices (two CTAs per chain) while that still fits the
   // machine in one wave; otherwise one CTA per chain.
-  const long chains = (long)p.Hv * p.N;
-  if (2 * chains <= sm_count()) return launch_chain<64>(mk, p, st);
-  return launch_chain<128>(mk, p, st);
+  const long ctas = (long)p.Hv * p.N * P;
+  if (2 * ctas <= sm_count()) return launch_chain<64, false>(mk, p, st);
+  return launch_chain<128, false>(mk, p, st);
+}
+
+// Segments per sequence for the chain: the count that minimises an estimate
+// of the serial chain steps -- ceil(chunks / P) steps for the transfer chains
+// (per wave of them) plus as many for the output chains, about two per scan
+// step and two for the extra launches -- among those whose output chains fit
+// the SMs in one wave.  One serial chain takes `chunks` steps.
+int chunk_tc_split_auto_segments(int N, int T, int Hv) {
+  const long chains = (long)N * Hv;
+  if (N <= 0 || chains > kSegMaxChains) return 1;
+  const int sms = sm_count();
+  const double nch = (double)T / C / N;  // chunks per sequence, on average
+  int best = 1;
+  double best_cost = nch;
+  for (int P = 3; P <= kSegMax; ++P) {
+    if (chains * P > sms) break;
+    const double seg = ceil(nch / P);
+    const double waves = ceil(2.0 * chains * (P - 1) / sms);
+    const double out_step = 2 * chains * P <= sms ? 1.0 : 1.15;  // whole-row chains are a little slower
+    const double cost = seg * waves + seg * out_step + 2.0 * (P - 1) + 2.0;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = P;
+    }
+  }
+  return best;
 }
 
 #ifdef GDN_PHASE_TIMING

@@ -38,6 +38,8 @@ gdn_dtype mid_dtype(gdn_dtype in) { return in == GDN_BF16 ? GDN_F16 : GDN_F32; }
 struct Workspace {
   void* q; void* k; void* v; float* g; float* beta;
   uint8_t* rec;  // operand records of the two-kernel tensor-core path (or null)
+  float* seg_mr;     // segment maps and start states of its segmented chain (or null)
+  float* seg_start;
   size_t bytes;
 };
 
@@ -56,9 +58,16 @@ Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base, int N = -1) 
   w.g = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
   w.beta = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
   w.rec = nullptr;
+  w.seg_mr = w.seg_start = nullptr;
   if (N >= 0) {
     w.rec = p ? reinterpret_cast<uint8_t*>(p + off) : nullptr;
     off += align_up(chunk_tc_split_record_bytes(N, T, d->Hv), 256);
+    const size_t sb = chunk_tc_split_seg_bytes(N, d->Hv);
+    if (sb > 0 && p) {
+      w.seg_mr = reinterpret_cast<float*>(p + off);
+      w.seg_start = w.seg_mr + (size_t)N * d->Hv * 2 * (kSegMax - 1) * d->dk * d->dk;
+    }
+    off += align_up(sb, 256);
   }
   w.bytes = off;
   return w;
@@ -96,6 +105,11 @@ size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_
   return carve(dims, T_tot, dtype, nullptr, N).bytes;
 }
 
+int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot) {
+  if (check_dims(dims) != GDN_OK || N < 1 || T_tot < 0) return 0;
+  return chunk_tc_split_auto_segments(N, T_tot, dims->Hv);
+}
+
 gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* stream) {
   gdn_status s = check_dims(dims);
   if (s != GDN_OK) return s;
@@ -103,6 +117,8 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   if (a->N < 0 || a->T_tot < 0) return GDN_ERR_DIMS;
   if (!dtype_ok(a->dtype)) return GDN_ERR_DIMS;
   if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (a->segments < 0 || a->segments > kSegMax) return GDN_ERR_UNSUPPORTED;
+  if (a->segments > 1 && (long)a->N * dims->Hv > kSegMaxChains) return GDN_ERR_UNSUPPORTED;
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
   const int Cc = 2 * dims->Hk * d + dims->Hv * d;
@@ -147,6 +163,12 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
   ch.eps_norm = dims->eps_norm;
   ch.rec = ws.rec;
+  ch.nseg = 1;
+  if (path == Path::TcSplit && ws.seg_mr) {
+    ch.nseg = a->segments > 0 ? a->segments : chunk_tc_split_auto_segments(a->N, a->T_tot, dims->Hv);
+    ch.seg_mr = ws.seg_mr;
+    ch.seg_start = ws.seg_start;
+  }
   if (a->core_event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_begin), st) != cudaSuccess)
     return GDN_ERR_CUDA;
   s = from_cuda(path == Path::TcSplit ? launch_chunk_tc_split(ch, st)
@@ -207,6 +229,7 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   ch.z = nullptr; ch.norm_w = nullptr; ch.out = nullptr; ch.o_raw = a->o;
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
   ch.eps_norm = dims->eps_norm;
+  ch.nseg = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return from_cuda(path == Path::Tc ? launch_chunk_tc(ch, st)
                                     : launch_chunk_simt(ch, d, GDN_F32, a->dtype, st));

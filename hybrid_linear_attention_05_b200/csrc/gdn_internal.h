@@ -51,6 +51,13 @@ struct ChunkParams {
   int T, N, Hk, Hv, chunk;
   float eps_norm;
   uint8_t* rec;               // split tensor-core path: per-(chunk, head) operand records
+  // split tensor-core path, segmented state chain (nseg > 1): each sequence's
+  // chunks are cut into nseg segments; seg_mr holds the affine map (M, R) of
+  // every segment but the last, [N][nseg-1][Hv][2][d][d], seg_start the state
+  // at the start of every segment, [N][nseg][Hv][d][d] (both fp32)
+  int nseg;
+  float* seg_mr;
+  float* seg_start;
 };
 
 // chunk_simt.cu: fp32 CUDA-core chunked core.  Supported (d, chunk) pairs:
@@ -69,6 +76,14 @@ cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st);
 // every (chunk, value head) writing operand records, then a per-head chain
 // kernel.  Needs chunk_tc_split_record_bytes(...) of extra workspace.
 size_t chunk_tc_split_record_bytes(int N, int T, int Hv);
+// Segmented state chains: at most this many segments per sequence, and only
+// while N * Hv <= kSegMaxChains; chunk_tc_split_seg_bytes is the workspace
+// they take (0 beyond that bound).
+constexpr int kSegMax = 8;
+constexpr int kSegMaxChains = 64;
+size_t chunk_tc_split_seg_bytes(int N, int Hv);
+// Segments chosen for these sizes when the caller asks for none in particular.
+int chunk_tc_split_auto_segments(int N, int T, int Hv);
 cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st);
 int split_error_word(int clear);  // host: read (and clear) that path's device error word
 

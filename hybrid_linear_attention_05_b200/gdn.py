@@ -33,8 +33,9 @@ GDN_IMPL_SIMT = 1
 GDN_IMPL_TC = 2
 GDN_IMPL_TC_SPLIT = 3
 
-EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill", "gdn_prefill_noalloc", "gdn_decode",
-            "gdn_chunk_core", "gdn_device_error", "gdn_status_string", "gdn_version"]
+EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
+            "gdn_prefill_auto_segments", "gdn_prefill_noalloc", "gdn_decode", "gdn_chunk_core",
+            "gdn_device_error", "gdn_status_string", "gdn_version"]
 
 # Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
 GDN_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -57,7 +58,7 @@ class gdn_prefill_args(ctypes.Structure):
                 ("initial_state", _vp), ("final_state", _vp), ("conv_state_in", _vp),
                 ("conv_state_out", _vp), ("out", _vp), ("workspace", _vp),
                 ("workspace_bytes", ctypes.c_size_t), ("core_event_begin", _vp),
-                ("core_event_end", _vp)]
+                ("core_event_end", _vp), ("segments", ctypes.c_int)]
 
 
 class gdn_decode_args(ctypes.Structure):
@@ -90,6 +91,8 @@ def lib():
         L.gdn_prefill_workspace_size_n.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int]
         L.gdn_prefill_workspace_size_n.restype = ctypes.c_size_t
+        L.gdn_prefill_auto_segments.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
+        L.gdn_prefill_auto_segments.restype = ctypes.c_int
         L.gdn_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args), _vp]
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_prefill_noalloc.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
@@ -164,16 +167,21 @@ def gdn_prefill_workspace_size_n(dims: gdn_dims, N: int, T_tot: int, dtype: int)
     return int(lib().gdn_prefill_workspace_size_n(ctypes.byref(dims), int(N), int(T_tot), int(dtype)))
 
 
+def gdn_prefill_auto_segments(dims: gdn_dims, N: int, T_tot: int) -> int:
+    """Segments per sequence the two-kernel path picks by itself (gdn.h)."""
+    return int(lib().gdn_prefill_auto_segments(ctypes.byref(dims), int(N), int(T_tot)))
+
+
 def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,
                 cu_seqlens, N, T_tot, chunk, dtype, out, workspace, workspace_bytes,
                 initial_state=None, final_state=None, conv_state_in=None, conv_state_out=None,
-                impl=GDN_IMPL_AUTO, core_event_begin=None, core_event_end=None, stream=None,
-                raise_on_error=True) -> int:
+                impl=GDN_IMPL_AUTO, core_event_begin=None, core_event_end=None, segments=0,
+                stream=None, raise_on_error=True) -> int:
     args = gdn_prefill_args(
         ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
         ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
         ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
-        ptr(workspace), int(workspace_bytes), core_event_begin, core_event_end)
+        ptr(workspace), int(workspace_bytes), core_event_begin, core_event_end, int(segments))
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill(ctypes.byref(dims), ctypes.byref(args), s), "gdn_prefill",
                   raise_on_error)
@@ -190,7 +198,7 @@ def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bi
         ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
         ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
         ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
-        None, 0, None, None)
+        None, 0, None, None, 0)
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill_noalloc(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_prefill_noalloc", raise_on_error)

@@ -9,6 +9,8 @@ Value distributions (N(mu, s) means mean mu and *standard deviation* s):
   conv weight  [Cc, 4]      N(0, 0.25)
   a, b         [T, Hv]      N(0, 1)
   A_log        [Hv]         U(0, ln 16)   -> exp(A_log) in [1, 16]
+                            (tests also draw U(-7, -5): a slow decay that
+                            carries the state across many chunks)
   dt_bias      [Hv]         N(0, 0.1)
   z            [T, Hv*dv]   N(0, 1)
   norm weight  [dv]         1 + N(0, 0.1)
@@ -49,6 +51,7 @@ class Workload:
     varlen_total: int = 0     # >0: lengths drawn at random summing to this
     varlen_n: int = 0
     q_scale: Optional[float] = None  # factor on the normalised q; None -> d ** -0.5
+    A_log_range: tuple = (0.0, LN16)  # A_log ~ U(lo, hi)
 
     @property
     def Cc(self) -> int:
@@ -148,7 +151,7 @@ def _cast(x: np.ndarray, dtype: str) -> np.ndarray:
 
 def _weights(w: Workload, rng):
     conv_w = _cast(_normal(rng, (w.Cc, 4), 0.25), w.dtype)
-    A_log = rng.uniform(0.0, LN16, size=(w.Hv,)).astype(np.float32)
+    A_log = rng.uniform(w.A_log_range[0], w.A_log_range[1], size=(w.Hv,)).astype(np.float32)
     dt_bias = _normal(rng, (w.Hv,), 0.1)
     norm_w = _cast(_normal(rng, (w.d,), 0.1, 1.0), w.dtype)
     return conv_w, A_log, dt_bias, norm_w

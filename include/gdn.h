@@ -140,6 +140,14 @@ typedef struct {
                                   before / after the chunked-core kernel (timing
                                   of that kernel alone); NULL to skip           */
   void* core_event_end;
+  int segments;                /* two-kernel tensor-core path only: the number of
+                                  segments each sequence's state chain is cut
+                                  into and run in parallel (0 = chosen from the
+                                  sizes and the SM count, 1 = one serial chain,
+                                  2..8 = that many).  Other values, or more than 1
+                                  when N*Hv > 64, return GDN_ERR_UNSUPPORTED.
+                                  Every choice computes the same result up to
+                                  rounding.                                      */
 } gdn_prefill_args;
 
 /* Bytes of device workspace gdn_prefill needs for these sizes (0 when the
@@ -150,15 +158,26 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dty
 
 /* Bytes of workspace that also holds the per-(chunk, value head) operand
  * records of the two-kernel tensor-core path (GDN_IMPL_TC_SPLIT): about
- * 33 KB per 64 tokens and value head, for N sequences of T_tot tokens in
- * total.  With at least this much, GDN_IMPL_AUTO takes the two-kernel path
- * where the tensor cores apply; with only gdn_prefill_workspace_size bytes it
- * takes the single-kernel one.  0 when the sizes are invalid. */
+ * 82 KB per 64 tokens and value head, for N sequences of T_tot tokens in
+ * total, plus, when N*Hv <= 64, 1.4 MB per (sequence, value head) for the
+ * segment maps and start states of a segmented state chain (see
+ * gdn_prefill_args.segments).  With at least this much, GDN_IMPL_AUTO takes
+ * the two-kernel path where the tensor cores apply; with only
+ * gdn_prefill_workspace_size bytes it takes the single-kernel one.  0 when
+ * the sizes are invalid. */
 size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_dtype dtype);
 
 /* Steps 1-5 over packed sequences.  Writes out, and final_state /
  * conv_state_out when given.  The workspace is overwritten. */
 gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* args, void* stream);
+
+/* Number of segments the two-kernel tensor-core path cuts each sequence's
+ * state chain into when gdn_prefill_args.segments is 0, for N sequences of
+ * T_tot tokens in total on the current device (1: one serial chain per
+ * (sequence, value head)).  With more than one segment the path launches
+ * two more kernels: the segments' affine maps and the scan of their start
+ * states.  0 when the sizes are invalid. */
+int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot);
 
 /* ------------------------------------------------ prefill without workspace
  * No counterpart on the pages: this is an addition of this library for

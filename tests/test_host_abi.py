@@ -95,10 +95,29 @@ def test_prefill_rejects_bad_dims(L, dims, status):
     (dict(conv_state_in=FAKE, conv_state_out=FAKE + 1024), gdn.GDN_ERR_ALIAS),
     (dict(initial_state=FAKE, final_state=FAKE + 4096), gdn.GDN_ERR_ALIAS),
     (dict(chunk=16, impl=gdn.GDN_IMPL_TC), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(segments=-1), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(segments=9), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(segments=2, N=17, T_tot=17), gdn.GDN_ERR_UNSUPPORTED),  # 17 x 4 chains > 64
 ])
 def test_prefill_rejects_bad_args(L, over, status):
     dims = gdn.make_dims(2, 4, 128)
     assert gdn.gdn_prefill(dims, **prefill_kwargs(**over)) == status
+
+
+def test_workspace_size_with_segments():
+    """The two-kernel workspace adds the records and, for at most 64 chains,
+    room for 8-segment chains: 7 maps (M, R) and 8 start states of d x d fp32
+    per (sequence, value head)."""
+    dims = gdn.make_dims(2, 4, 128)
+    base = gdn.gdn_prefill_workspace_size(dims, 1000, gdn.GDN_BF16)
+    rec = (1000 // 64 + 3 + 1) * 4 * 82432
+    seg = 3 * 4 * (2 * 7 + 8) * 128 * 128 * 4
+    n = gdn.gdn_prefill_workspace_size_n(dims, 3, 1000, gdn.GDN_BF16)
+    assert base + rec + seg <= n <= base + rec + seg + 2 * 256
+    # 17 sequences x 4 value heads = 68 chains: no segment buffers
+    n17 = gdn.gdn_prefill_workspace_size_n(dims, 17, 1000, gdn.GDN_BF16)
+    rec17 = (1000 // 64 + 17 + 1) * 4 * 82432
+    assert base + rec17 <= n17 <= base + rec17 + 2 * 256
 
 
 def test_prefill_empty_batch_is_noop(L):

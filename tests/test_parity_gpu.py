@@ -37,13 +37,17 @@ P397 = WORKLOADS["prefill_varlen8_T65536_Hk16_Hv64_d128"]
 
 IMPLS = {"simt": (gdn.GDN_IMPL_SIMT, 32), "tc": (gdn.GDN_IMPL_TC, 64),
          "split": (gdn.GDN_IMPL_TC_SPLIT, 64)}
+# A_log range of a slow decay (alpha ~ 0.995-0.9995 per token): the workloads'
+# own U(0, ln 16) decays the state by e^-45 or more per 64-token chunk, so only
+# slow-decay cases show whether the state is carried right across chunks
+SLOW_DECAY = (-7.0, -5.0)
 
 
 def np64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_prefill(inp, impl, chunk, guard=True):
+def run_prefill(inp, impl, chunk, guard=True, segments=0):
     dp = api.to_device(inp, chunk=chunk)
     bufs = api.PrefillBuffers(dp)
     if guard:  # canaries on both sides of every output
@@ -58,7 +62,7 @@ def run_prefill(inp, impl, chunk, guard=True):
         T_tot=dp.T, chunk=dp.chunk, dtype=bufs.dtype_code, out=bufs.out, workspace=bufs.workspace,
         workspace_bytes=bufs.ws_bytes, initial_state=dp.initial_state,
         final_state=bufs.final_state, conv_state_in=dp.conv_state_in,
-        conv_state_out=bufs.conv_state_out, impl=impl, raise_on_error=False)
+        conv_state_out=bufs.conv_state_out, impl=impl, segments=segments, raise_on_error=False)
     if status == gdn.GDN_ERR_UNSUPPORTED:
         pytest.skip("implementation not available for this shape")
     assert status == gdn.GDN_OK, gdn.status_string(status)
@@ -132,6 +136,79 @@ def test_split_value_pairs_varlen(seqlens):
     inp = make_prefill(P9B, seqlens=seqlens, with_conv_state=True)
     bufs = run_prefill(inp, gdn.GDN_IMPL_TC_SPLIT, 64)
     check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("segments,seqlens,decay", [
+    (3, (64 * 11 + 5, 130, 0, 64 * 3, 1), "slow"),
+    (5, (64 * 5, 64 * 9 + 63, 2), "slow"),
+    (8, (64 * 11 + 5, 130, 0, 64 * 3, 1), "slow"),
+    (8, (64 * 8, 64 * 16 + 1), "workload"),
+])
+def test_split_segmented_chain_varlen(segments, seqlens, decay):
+    """Segmented state chains: each sequence's chunks cut into `segments`
+    pieces whose affine maps and start states are formed first.  Covers
+    segments with several chunks and with none (a sequence of fewer chunks
+    than segments), an empty sequence, GQA, nonzero initial states and conv
+    history, with half-width CTA pairs (3, 5) and whole-row CTAs (8)."""
+    w = resized(P9B, Hk=2, Hv=4, seed=70 + segments)
+    if decay == "slow":
+        w = resized(w, A_log_range=SLOW_DECAY)
+    inp = make_prefill(w, seqlens=seqlens, with_conv_state=True)
+    bufs = run_prefill(inp, gdn.GDN_IMPL_TC_SPLIT, 64, segments=segments)
+    check_full(inp, bufs)
+
+
+def test_split_segments_agree_with_serial_chain():
+    """The same call with one serial chain and with 4 and 8 segments: the
+    results agree with each other within the parity bar and each matches
+    the oracle."""
+    w = resized(P08, Hk=4, Hv=4, seed=77, A_log_range=SLOW_DECAY)
+    inp = make_prefill(w, seqlens=(64 * 24 + 17,))
+    ref = oracle_prefill(inp)
+    outs = []
+    for seg in (1, 4, 8):
+        bufs = run_prefill(inp, gdn.GDN_IMPL_TC_SPLIT, 64, segments=seg)
+        outs.append((np64(bufs.out), np64(bufs.final_state)))
+        assert relerr(outs[-1][0], ref.out) <= PREFILL_TOL
+        assert relerr(outs[-1][1], ref.final_state) <= PREFILL_TOL
+    for o, S in outs[1:]:
+        assert relerr(o, outs[0][0]) <= PREFILL_TOL
+        assert relerr(S, outs[0][1]) <= PREFILL_TOL
+
+
+@pytest.mark.parametrize("impl,segments", [("tc", 0), ("split", 1), ("split", 4), ("split", 8)])
+def test_slow_decay_state_carry(impl, segments):
+    """Slow decay (exp(A_log) ~ 1e-3, alpha near 1) so that the state written
+    in early chunks still shapes the outputs and the final state many chunks
+    later -- the regime where the chunk-to-chunk carry, and for segmented
+    chains the segment maps and the scan, are actually exercised.  Nonzero
+    initial states, GQA, two sequences of 17 and 9 chunks."""
+    w = resized(P9B, Hk=2, Hv=4, seed=79, A_log_range=SLOW_DECAY)
+    inp = make_prefill(w, seqlens=(64 * 16 + 40, 64 * 9))
+    code, chunk = IMPLS[impl]
+    bufs = run_prefill(inp, code, chunk, segments=segments)
+    check_full(inp, bufs)
+
+
+def test_split_segments_in_place_state():
+    """final_state the same buffer as initial_state with segmented chains: the
+    state is read (by the scan) before any chain writes it back."""
+    w = resized(P9B, Hk=2, Hv=4, seed=78, A_log_range=SLOW_DECAY)
+    inp = make_prefill(w, seqlens=(64 * 9 + 3, 64 * 4))
+    dp = api.to_device(inp, chunk=64)
+    bufs = api.PrefillBuffers(dp)
+    S = dp.initial_state.clone()
+    gdn.gdn_prefill(bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b,
+                    A_log=dp.A_log, dt_bias=dp.dt_bias, z=dp.z, norm_w=dp.norm_w,
+                    cu_seqlens=dp.cu_seqlens, N=dp.N, T_tot=dp.T, chunk=64,
+                    dtype=bufs.dtype_code, out=bufs.out, workspace=bufs.workspace,
+                    workspace_bytes=bufs.ws_bytes, initial_state=S, final_state=S,
+                    impl=gdn.GDN_IMPL_TC_SPLIT, segments=4)
+    torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0
+    ref = oracle_prefill(inp)
+    assert relerr(np64(S), ref.final_state) <= PREFILL_TOL
+    assert relerr(np64(bufs.out), ref.out) <= PREFILL_TOL
 
 
 @pytest.mark.parametrize("impl", ["simt", "tc", "split"])
