@@ -641,6 +641,8 @@ extern "C" gdn_status gdn_device_error(int* code, int clear) {
   }
   const int v2 = gdn::split_error_word(clear);
   if (v2 < 0) return GDN_ERR_CUDA;
-  *code = v != 0 ? v : v2;
+  const int v3 = gdn::conv_error_word(clear);
+  if (v3 < 0) return GDN_ERR_CUDA;
+  *code = v != 0 ? v : (v2 != 0 ? v2 : v3);
   return GDN_OK;
 }

@@ -926,22 +926,31 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
 // S_start(s+1) = S_start(s) M_s + R_s for every segment s but the last (an
 // empty segment maps the state to itself).  The CTA keeps its rows
 // transposed in shared memory (sT[i][r]) and each M_s in a double buffer
-// filled by cp.async one segment ahead.  Thread (warp w, lane l) owns the 4 x
-// 4 tile rows 4 (l >> 3) .. +3, columns 4 (8 w + (l & 7)) .. +3: per index i
-// a warp reads 64 contiguous bytes of sT and 128 of M (one wavefront each)
-// for 16 FMAs.
-constexpr int SR = 16;                 // state rows per CTA
-constexpr int SCAN_THREADS = SR * 8;   // 4 x 4 outputs per thread
-constexpr uint32_t SCAN_SMEM = 2 * D * D * 4 + D * SR * 4 + 128;
+// filled by bulk copies one segment ahead; every map and R slice it will
+// read is requested into L2 at the start.  The product is split over the
+// contraction index: warp w takes i in [32 (w / 4), 32 (w / 4) + 32) and,
+// with lane l, the 4 x 4 output tile rows 4 (l / 8) .. +3, columns
+// 4 (8 (w % 4) + l % 8) .. +3 (per i a warp reads 64 contiguous bytes of sT
+// and 128 of M: one wavefront each); the four partial tiles are summed
+// through shared memory by the threads of warps 0..3, which own the rows.
+constexpr int SR = 16;                  // state rows per CTA
+constexpr int SCAN_KS = 4;              // contraction slices
+constexpr int SCAN_POS = SR * 8;        // 4 x 4 output tiles per slice
+constexpr int SCAN_THREADS = SCAN_POS * SCAN_KS;
+constexpr uint32_t SCAN_SMEM = (2 * D * D + D * SR + SCAN_KS * 16 * SCAN_POS) * 4 + 16 + 128;
 __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
   extern __shared__ uint8_t scan_raw[];
   float* Mb = reinterpret_cast<float*>(scan_raw + ((128u - (smem_u32(scan_raw) & 127u)) & 127u));
-  float* sT = Mb + 2 * D * D;  // [D][SR]
+  float* sT = Mb + 2 * D * D;   // [D][SR]
+  float* red = sT + D * SR;     // [SCAN_KS][16][SCAN_POS] partial tiles
+  const uint32_t mbar = smem_u32(red + SCAN_KS * 16 * SCAN_POS);  // two mbarriers, one per M buffer
   const int P = p.nseg;
   const int h = blockIdx.x / (D / SR), r0 = (blockIdx.x % (D / SR)) * SR;
   const int n = blockIdx.y;
   const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-  const int rr = (l >> 3) * 4, cc = (w * 8 + (l & 7)) * 4;  // this thread's tile within the CTA's rows
+  const int ks = w >> 2, pos = tid & (SCAN_POS - 1);
+  const bool owner = ks == 0;  // warps 0..3 own the rows
+  const int rr = (l >> 3) * 4, cc = ((w & 3) * 8 + (l & 7)) * 4;  // this thread's tile within the CTA's rows
   const size_t hd = (size_t)D * D;
   const size_t nh = (size_t)n * p.Hv + h;
   const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
@@ -954,18 +963,29 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     while (sg < P - 1 && !nonempty(sg)) ++sg;
     return sg;
   };
-  auto prefetch = [&](int sg, int buf) {
+  auto prefetch = [&](int sg, int buf) {  // thread 0: M_sg into buffer buf
     const float* M = map_of(sg);
-    const uint32_t dst = smem_u32(Mb + buf * D * D);
-    for (int e = tid; e < D * D / 4; e += SCAN_THREADS) cp_async16(dst + e * 16, M + e * 4, 16u);
-    cp_async_commit();
+    const uint32_t dst = smem_u32(Mb + buf * D * D), bar = mbar + 8 * buf;
+    mbar_arrive_expect_tx(bar, D * D * 4);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) bulk_load(dst + q * (D * D), M + q * (D * D / 4), D * D, bar);
   };
+  if (tid == 0) {
+    mbar_init(mbar, 1);
+    mbar_init(mbar + 8, 1);
+    fence_mbar_init();
+  }
+  if (tid < P - 1 && nonempty(tid)) {  // every map and R slice this CTA will read, into L2
+    bulk_prefetch_l2(map_of(tid), D * D * 4);
+    bulk_prefetch_l2(map_of(tid) + hd + (size_t)r0 * D, SR * D * 4);
+  }
+  __syncthreads();
   int sg_next = next_map(0);
-  int buf = 0;
-  if (sg_next < P - 1) prefetch(sg_next, buf);
+  int j = 0;  // maps applied so far: map j sits in buffer j & 1, that buffer's use j >> 1
+  if (tid == 0 && sg_next < P - 1) prefetch(sg_next, 0);
 
-  float acc[4][4];
-  {
+  float acc[4][4];  // owners: the state tile; everyone: partial products
+  if (owner) {
     const float* S0 = p.S0 ? p.S0 + nh * hd : nullptr;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -975,33 +995,45 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     }
   }
   for (int sg = 0;; ++sg) {
-    float* dst = p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd;
+    if (owner) {
+      float* dst = p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd;
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-      *reinterpret_cast<float4*>(dst + (size_t)(r0 + rr + r) * D + cc) =
-          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      for (int r = 0; r < 4; ++r)
+        *reinterpret_cast<float4*>(dst + (size_t)(r0 + rr + r) * D + cc) =
+            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
     if (sg + 1 >= P) break;
     if (sg != sg_next) continue;  // empty segment: the state passes through
-    // this segment's map: S <- S M + R
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) = make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
-    // R is added after the products, so its loads overlap them
-    const float* R = map_of(sg) + hd;
+    // this segment's map: S <- S M + R (R is added by the owners after the
+    // products, so its loads overlap them)
     float4 rv[4];
+    if (owner) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      rv[r] = __ldg(reinterpret_cast<const float4*>(R + (size_t)(r0 + rr + r) * D + cc));
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) = make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
+      const float* R = map_of(sg) + hd;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) rv[r] = __ldg(reinterpret_cast<const float4*>(R + (size_t)(r0 + rr + r) * D + cc));
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    const int buf = j & 1;
+    const uint32_t par = (uint32_t)(j >> 1) & 1u;
+    if (__syncthreads_or(!mbar_wait(mbar + 8 * buf, par))) {
+      // sT is complete but this segment's M never landed: record it, let the copy finish, stop
+      if (tid == 0) {
+        atomicExch(&g_split_error, 1);
+        mbar_wait(mbar + 8 * buf, par, 100000000ull);
+      }
+      break;
     }
-    cp_async_wait_all();
-    __syncthreads();  // sT and this segment's M are complete
     sg_next = next_map(sg + 1);
-    if (sg_next < P - 1) prefetch(sg_next, buf ^ 1);
+    if (tid == 0 && sg_next < P - 1) prefetch(sg_next, buf ^ 1);
     const float* M = Mb + buf * D * D;
 #pragma unroll 4
-    for (int i = 0; i < D; ++i) {
+    for (int i = ks * (D / SCAN_KS); i < (ks + 1) * (D / SCAN_KS); ++i) {
       const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
       const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);
       const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
@@ -1011,14 +1043,30 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(sv[r], mv[c], acc[r][c]);
     }
+    if (!owner) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      acc[r][0] += rv[r].x; acc[r][1] += rv[r].y; acc[r][2] += rv[r].z; acc[r][3] += rv[r].w;
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[((ks * 16) + r * 4 + c) * SCAN_POS + pos] = acc[r][c];
     }
-    __syncthreads();  // everyone is done with sT and this buffer
-    buf ^= 1;
+    __syncthreads();  // partial tiles written; everyone is done with sT and this buffer
+    if (owner) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float rvr[4] = {rv[r].x, rv[r].y, rv[r].z, rv[r].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v = acc[r][c] + rvr[c];
+#pragma unroll
+          for (int k2 = 1; k2 < SCAN_KS; ++k2) v += red[((k2 * 16) + r * 4 + c) * SCAN_POS + pos];
+          acc[r][c] = v;
+        }
+      }
+    }
+    ++j;
+    // the owners' reads of `red` end before its next write: two barriers
+    // (the one above sT's completion and the one after the products) lie between
   }
-  cp_async_wait_all();
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

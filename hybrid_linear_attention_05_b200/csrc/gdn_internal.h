@@ -32,6 +32,7 @@ struct ConvPrepParams {
   int tok_blocks;             // set by the launcher
 };
 cudaError_t launch_conv_prep(const ConvPrepParams& p, int d, gdn_dtype dt, cudaStream_t st);
+int conv_error_word(int clear);  // host: read (and clear) the conv kernel's device error word
 
 // Parameters of the chunked core (both implementations).
 struct ChunkParams {
