@@ -176,6 +176,27 @@ __global__ void __launch_bounds__(NTA, 2)
   const int hk = h / (p.Hv / p.Hk);
   uint8_t* rec = p.rec + ((size_t)g * p.Hv + h) * REC;
 
+  // the chunk's gates and z are requested first: their latency overlaps the
+  // barrier and TMEM set-up and the operand copies
+  float gv = 0.f, bv = 0.f;
+  if (tid < L) {
+    gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
+    bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
+  }
+  // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
+  // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
+  const bool gated = p.out != nullptr;
+  uint4 zv[4];
+  if (gated) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+      zv[k] = r < L ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.z) +
+                                                           (size_t)(c0 + r) * p.Hv * D + h * D + ch * 8))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
   if (tid == 0) {
     mbar_init(bar_load, 1);
     mbar_init(bar_m1, 1);
@@ -205,27 +226,9 @@ __global__ void __launch_bounds__(NTA, 2)
     tma_load_2d(sb + A_V, &tm_v, h * D, c0, bar_load);
     tma_load_2d(sb + A_V + TILE, &tm_v, h * D + 64, c0, bar_load);
   }
-  // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
-  // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
-  const bool gated = p.out != nullptr;
-  uint4 zv[4];
-  if (gated) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
-      zv[k] = r < L ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.z) +
-                                                           (size_t)(c0 + r) * p.Hv * D + h * D + ch * 8))
-                    : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
   if (gated && tid < D) wsm[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tid]);
   // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
-  float gv = 0.f, bv = 0.f;
   if (tid < 64) {
-    if (tid < L) {
-      gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
-      bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
-    }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float t = __shfl_up_sync(0xffffffffu, gv, o);
@@ -256,10 +259,16 @@ __global__ void __launch_bounds__(NTA, 2)
       }
       mma_commit(bar_m1);
     }
-    // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and the record's vectors
-    for (int e = tid; e < 64 * 64; e += NTA) {
-      const int i = e >> 6, j = e & 63;
-      if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gam[j]);
+    // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and
+    // the record's vectors; this thread: column j = tid % 64, rows 16 (tid / 64) .. +15
+    {
+      const int j = tid & 63, i0 = (tid >> 6) * 16;
+      const float gj = gam[j];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u;
+        if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
+      }
     }
     if (tid < 64) {
       float* vec = reinterpret_cast<float*>(rec + R_VEC);
