@@ -993,14 +993,17 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
   int j = 0;  // maps applied so far: map j sits in buffer j & 1, that buffer's use j >> 1
   if (tid == 0 && sg_next < P - 1) prefetch(sg_next, 0);
 
-  float acc[4][4];  // owners: the state tile; everyone: partial products
+  // owners: the state tile; everyone: partial products.  Column pairs as
+  // float2 for the packed fp32x2 FMA: acc[r][0] = columns cc, cc+1; acc[r][1] = cc+2, cc+3
+  float2 acc[4][2];
   if (owner) {
     const float* S0 = p.S0 ? p.S0 + nh * hd : nullptr;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float4 v = S0 ? *reinterpret_cast<const float4*>(S0 + (size_t)(r0 + rr + r) * D + cc)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
-      acc[r][0] = v.x; acc[r][1] = v.y; acc[r][2] = v.z; acc[r][3] = v.w;
+      acc[r][0] = make_float2(v.x, v.y);
+      acc[r][1] = make_float2(v.z, v.w);
     }
   }
   for (int sg = 0;; ++sg) {
@@ -1009,7 +1012,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
         *reinterpret_cast<float4*>(dst + (size_t)(r0 + rr + r) * D + cc) =
-            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
     }
     if (sg + 1 >= P) break;
     if (sg != sg_next) continue;  // empty segment: the state passes through
@@ -1018,16 +1021,18 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     float4 rv[4];
     if (owner) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) = make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
+      for (int c = 0; c < 4; ++c) {
+        const int hc = c >> 1;
+        *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) =
+            (c & 1) ? make_float4(acc[0][hc].y, acc[1][hc].y, acc[2][hc].y, acc[3][hc].y)
+                    : make_float4(acc[0][hc].x, acc[1][hc].x, acc[2][hc].x, acc[3][hc].x);
+      }
       const float* R = map_of(sg) + hd;
 #pragma unroll
       for (int r = 0; r < 4; ++r) rv[r] = __ldg(reinterpret_cast<const float4*>(R + (size_t)(r0 + rr + r) * D + cc));
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
     const int buf = j & 1;
     const uint32_t par = (uint32_t)(j >> 1) & 1u;
     if (__syncthreads_or(!mbar_wait(mbar + 8 * buf, par))) {
@@ -1046,30 +1051,35 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
       const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);
       const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-      const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+      const float2 m01 = make_float2(m4.x, m4.y), m23 = make_float2(m4.z, m4.w);
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(sv[r], mv[c], acc[r][c]);
+      for (int r = 0; r < 4; ++r) {
+        const float2 s2 = make_float2(sv[r], sv[r]);
+        acc[r][0] = __ffma2_rn(s2, m01, acc[r][0]);
+        acc[r][1] = __ffma2_rn(s2, m23, acc[r][1]);
+      }
     }
     if (!owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) red[((ks * 16) + r * 4 + c) * SCAN_POS + pos] = acc[r][c];
+        for (int c = 0; c < 4; ++c)
+          red[((ks * 16) + r * 4 + c) * SCAN_POS + pos] = (c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x;
     }
     __syncthreads();  // partial tiles written; everyone is done with sT and this buffer
     if (owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float rvr[4] = {rv[r].x, rv[r].y, rv[r].z, rv[r].w};
+        float v[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v = acc[r][c] + rvr[c];
+          v[c] = ((c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x) + rvr[c];
 #pragma unroll
-          for (int k2 = 1; k2 < SCAN_KS; ++k2) v += red[((k2 * 16) + r * 4 + c) * SCAN_POS + pos];
-          acc[r][c] = v;
+          for (int k2 = 1; k2 < SCAN_KS; ++k2) v[c] += red[((k2 * 16) + r * 4 + c) * SCAN_POS + pos];
         }
+        acc[r][0] = make_float2(v[0], v[1]);
+        acc[r][1] = make_float2(v[2], v[3]);
       }
     }
     ++j;

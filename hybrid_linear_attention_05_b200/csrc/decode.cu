@@ -45,6 +45,18 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   T* cs = static_cast<T*>(p.conv_state) + (size_t)b * Cc * 3;
   const T* cw = static_cast<const T*>(p.conv_w);
 
+  // The first value head's state rows are requested before anything else:
+  // they do not depend on the conv, so their HBM latency overlaps steps 1-2.
+  const int col = (lane % LPR) * 4;
+  auto state_of = [&](int gi) { return p.state + ((size_t)b * p.Hv + kh * G + gi) * D * D; };
+  auto row_of = [&](int s) { return warp * ROWS_PER_WARP + s * RPW + lane / LPR; };
+  float4 Sv[PASSES];
+  {
+    const float* S0 = state_of(0);
+#pragma unroll
+    for (int s = 0; s < PASSES; ++s) Sv[s] = __ldcs(reinterpret_cast<const float4*>(S0 + (size_t)row_of(s) * D + col));
+  }
+
   // 1. conv + SiLU, cache update in place (each channel read then written by one thread)
   for (int idx = tid; idx < NC; idx += NT) {
     int c;
@@ -92,10 +104,9 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   }
   __syncthreads();
 
-  // 3. state stream
+  // 3. state stream; while head gi is updated, head gi + 1's rows are requested
   const float* qv = ys;
   const float* kv = ys + D;
-  const int col = (lane % LPR) * 4;
   const float4 k4 = make_float4(kv[col], kv[col + 1], kv[col + 2], kv[col + 3]);
   const float4 q4 = make_float4(qv[col], qv[col + 1], qv[col + 2], qv[col + 3]);
   const float kq = misc[2];
@@ -103,16 +114,11 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
     const int h = kh * G + gi;
     const float alpha = misc[4 + gi], beta = misc[4 + G + gi];
     float* Sh = p.state + ((size_t)b * p.Hv + h) * D * D;
+    const float* Snext = gi + 1 < G ? state_of(gi + 1) : nullptr;
     const float* vv = ys + (2 + gi) * D;
-    float4 Sv[PASSES];
 #pragma unroll
     for (int s = 0; s < PASSES; ++s) {
-      const int r = warp * ROWS_PER_WARP + s * RPW + lane / LPR;
-      Sv[s] = *reinterpret_cast<const float4*>(Sh + (size_t)r * D + col);
-    }
-#pragma unroll
-    for (int s = 0; s < PASSES; ++s) {
-      const int r = warp * ROWS_PER_WARP + s * RPW + lane / LPR;
+      const int r = row_of(s);
       float u = Sv[s].x * k4.x + Sv[s].y * k4.y + Sv[s].z * k4.z + Sv[s].w * k4.w;
       float pp = Sv[s].x * q4.x + Sv[s].y * q4.y + Sv[s].z * q4.z + Sv[s].w * q4.w;
 #pragma unroll
@@ -126,8 +132,9 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
       sn.y = fmaf(alpha, Sv[s].y, delta * k4.y);
       sn.z = fmaf(alpha, Sv[s].z, delta * k4.z);
       sn.w = fmaf(alpha, Sv[s].w, delta * k4.w);
-      *reinterpret_cast<float4*>(Sh + (size_t)r * D + col) = sn;
+      __stcs(reinterpret_cast<float4*>(Sh + (size_t)r * D + col), sn);
       if ((lane % LPR) == 0) os[gi * D + r] = fmaf(alpha, pp, kq * delta);
+      if (Snext) Sv[s] = __ldcs(reinterpret_cast<const float4*>(Snext + (size_t)r * D + col));
     }
   }
   __syncthreads();
