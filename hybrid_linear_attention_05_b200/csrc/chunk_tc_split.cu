@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(NTA, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7, tl = tid & 127;
   const int g = blockIdx.x, h = blockIdx.y;
+  pdl_launch();
   // the sequence whose chunk owns this slot
   int lo = 0, hi = p.N - 1;
   while (lo < hi) {
@@ -176,13 +177,8 @@ __global__ void __launch_bounds__(NTA, 2)
   const int hk = h / (p.Hv / p.Hk);
   uint8_t* rec = p.rec + ((size_t)g * p.Hv + h) * REC;
 
-  // the chunk's gates and z are requested first: their latency overlaps the
-  // barrier and TMEM set-up and the operand copies
-  float gv = 0.f, bv = 0.f;
-  if (tid < L) {
-    gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
-    bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
-  }
+  // z of the chunk (an input of the call) is requested first: its latency
+  // overlaps the set-up and the wait for the conv kernel
   // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
   // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
   const bool gated = p.out != nullptr;
@@ -216,6 +212,12 @@ __global__ void __launch_bounds__(NTA, 2)
 #ifdef GDN_PHASE_TIMING
   long long t_prev = clock64();
 #endif
+  pdl_wait();  // q, k, v and the gates come from the conv kernel
+  float gv = 0.f, bv = 0.f;
+  if (tid < L) {
+    gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
+    bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
+  }
 
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_load, 6 * TILE);
@@ -545,6 +547,7 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7, tl = tid & 127;
+  pdl_launch();
   const int P = p.nseg;
   const int h = XFER ? (int)blockIdx.x >> 1 : (int)blockIdx.x / CL;
   const int vs = XFER ? 0 : (int)blockIdx.x % CL;
@@ -578,6 +581,7 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   if (nchunks == 0) {
     // empty segment; the last one is empty only for an empty sequence, whose
     // state passes through (every CTA of the cluster returns here)
+    pdl_wait();
     const float* Sin = start_state();
     float* Sfin = final_state();
     if (!XFER && Sfin)
@@ -614,6 +618,7 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
 #ifdef GDN_PHASE_TIMING
   long long t_prev = clock64();
 #endif
+  pdl_wait();  // the records, k and the start states come from the kernels before
 
   // thread LOADER streams K and the records: chunks 0 .. NST-1 up front, then
   // chunk c - 1 + NST once chunk c - 1 has released its stage
@@ -953,6 +958,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
   float* sT = Mb + 2 * D * D;   // [D][SR]
   float* red = sT + D * SR;     // [SCAN_KS][16][SCAN_POS] partial tiles
   const uint32_t mbar = smem_u32(red + SCAN_KS * 16 * SCAN_POS);  // two mbarriers, one per M buffer
+  pdl_launch();
   const int P = p.nseg;
   const int h = blockIdx.x / (D / SR), r0 = (blockIdx.x % (D / SR)) * SR;
   const int n = blockIdx.y;
@@ -984,6 +990,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     mbar_init(mbar + 8, 1);
     fence_mbar_init();
   }
+  pdl_wait();  // the maps come from the transfer chains
   if (tid < P - 1 && nonempty(tid)) {  // every map and R slice this CTA will read, into L2
     bulk_prefetch_l2(map_of(tid), D * D * 4);
     bulk_prefetch_l2(map_of(tid) + hd + (size_t)r0 * D, SR * D * 4);
@@ -1164,13 +1171,15 @@ cudaError_t launch_chain(const CUtensorMap& mk, const ChunkParams& p, cudaStream
   cfg.blockDim = dim3(XFER ? NCW : NTB, 1, 1);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = G::CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<VS, XFER>, mk, p);
 }
 
@@ -1195,9 +1204,18 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(chunk_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)A_SMEM);
     if (e != cudaSuccess) return e;
-    dim3 ga((unsigned)record_slots(p.N, p.T), p.Hv);
-    chunk_keys_kernel<<<ga, NTA, A_SMEM, st>>>(mq, mk, mv, p);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)record_slots(p.N, p.T), (unsigned)p.Hv, 1);
+    cfg.blockDim = dim3(NTA, 1, 1);
+    cfg.dynamicSmemBytes = A_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, chunk_keys_kernel, mq, mk, mv, p);
     if (e != cudaSuccess) return e;
   }
   const int P = p.nseg;
@@ -1207,8 +1225,18 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCAN_SMEM);
     if (e != cudaSuccess) return e;
-    seg_scan_kernel<<<dim3((unsigned)(p.Hv * (D / SR)), (unsigned)p.N), SCAN_THREADS, SCAN_SMEM, st>>>(p);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(p.Hv * (D / SR)), (unsigned)p.N, 1);
+    cfg.blockDim = dim3(SCAN_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SCAN_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, seg_scan_kernel, p);
     if (e != cudaSuccess) return e;
   }
   // Half-width value slices (two CTAs per chain) while that still fits the

@@ -245,6 +245,8 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
   const int n_ct = Cc / D;  // head segments
   const __nv_bfloat16* __restrict__ x = static_cast<const __nv_bfloat16*>(p.x);
   const __nv_bfloat16* __restrict__ hist_all = static_cast<const __nv_bfloat16*>(p.conv_state_in);
+  // the key-side kernel may be scheduled now; it waits for this grid to finish
+  ptx::pdl_launch();
 
   if ((int)blockIdx.x >= main_ctas) {
     // ------------------------------------------------------ conv tails

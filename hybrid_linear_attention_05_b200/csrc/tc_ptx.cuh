@@ -149,6 +149,17 @@ __device__ __forceinline__ bool bar_named_or(int id, int n, bool pred) {
   return r != 0;
 }
 
+// ------------------------------------------------- programmatic launch
+
+// Wait until the grid this one was launched after (as a programmatic
+// dependent) has completed and its memory is visible; a no-op for an
+// ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next grid on the stream, if it was launched as a programmatic
+// dependent, be scheduled once every CTA of this grid has issued this (or
+// exited); it still waits in pdl_wait for this grid to complete.
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------ TMA
 
 // 2-D tile load global -> shared, completion counted in bytes on `bar`.
