@@ -216,8 +216,8 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
 // 2-D TMA box brings its 67 input rows -- the 64 tokens and the 3 before
 // them, which the conv window needs; rows before token 0 read as zeros --
 // into shared memory, 256 B per row.  Persistent CTAs of 128 threads walk
-// the tiles with a three-buffer ring, so the next two tiles' boxes are in
-// flight while this one is computed.  Thread (tg = tid / 16, cg = tid % 16) takes channels
+// the tiles with a two-buffer ring, so the next tile's box is in flight while
+// this one is computed; the head's conv taps (1 KiB) arrive with each box.  Thread (tg = tid / 16, cg = tid % 16) takes channels
 // 8 cg .. 8 cg + 7 of tokens 8 tg .. 8 tg + 7: the 16 threads of a token
 // group hold one whole head and reduce the L2 norm with shuffles.  Window
 // rows before a sequence's first token come from its conv history (or are
@@ -226,8 +226,9 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
 constexpr int KT = 64;              // tokens per tile
 constexpr int KR = KT + 3;          // rows per box
 constexpr int KNT = 128;            // threads per CTA
-constexpr uint32_t KBUF = 17408;    // one box (67 x 256 B), rounded up to 1 KiB
-constexpr int KST = 3;               // boxes in flight per CTA
+constexpr uint32_t KW = KR * 256;   // the head's conv taps (128 x 4 bf16) follow the box
+constexpr uint32_t KBUF = 18432;    // one box (67 x 256 B) and the taps (1 KiB), rounded up to 1 KiB
+constexpr int KST = 2;               // boxes in flight per CTA
 constexpr uint32_t KSMEM = KST * KBUF + 64 + 1024;
 constexpr int KCTAS_PER_SM = 4;
 
@@ -288,8 +289,9 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
   auto issue = [&](int tile, int buf) {
     const int ct = tile % n_ct, tt = tile / n_ct;
     const uint32_t bar = bar0 + 8 * buf;
-    ptx::mbar_arrive_expect_tx(bar, (uint32_t)(KR * 256));
+    ptx::mbar_arrive_expect_tx(bar, (uint32_t)(KR * 256 + 1024));
     ptx::tma_load_2d(sb + buf * KBUF, &tm_x, ct * D, tt * KT - 3, bar);
+    ptx::bulk_load(sb + buf * KBUF + KW, static_cast<const __nv_bfloat16*>(p.conv_w) + (size_t)ct * D * 4, 1024, bar);
   };
 
   const int cg = tid & 15, tg = tid >> 4;
@@ -306,17 +308,20 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
     const int c0 = ct * D + cg * 8;
     const int t0 = tt * KT + tg * 8;
     const bool is_qk = ct < 2 * p.Hk, is_q = ct < p.Hk;
-    // conv taps as channel pairs: wv[tap][pair] = (w[2 pair][tap], w[2 pair + 1][tap])
-    float2 wv[4][4];
-    {
-      const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(p.conv_w) + (size_t)c0 * 4;
-      float tmp[32];
+    // gate inputs of this thread's tokens (first thread of a value head's
+    // token group), requested before the wait so that their latency overlaps it
+    const bool gates = !is_qk && cg == 0;
+    const int hh = ct - 2 * p.Hk;
+    float av[8], bv[8];
+    if (gates) {
+      const __nv_bfloat16* ap = static_cast<const __nv_bfloat16*>(p.a);
+      const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) load8(wp + r * 8, tmp + r * 8);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int tap = 0; tap < 4; ++tap) wv[tap][q] = make_float2(tmp[(2 * q) * 4 + tap], tmp[(2 * q + 1) * 4 + tap]);
+      for (int kk = 0; kk < 8; ++kk) {
+        const int t = min(t0 + kk, p.T - 1);
+        av[kk] = ld_f(ap + (size_t)t * p.Hv + hh);
+        bv[kk] = ld_f(bp + (size_t)t * p.Hv + hh);
+      }
     }
     int n = seq_of_token(p.cu_seqlens, p.N, min(t0, p.T - 1));
     int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
@@ -333,6 +338,18 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
       break;
     }
     const uint8_t* rows = smem + buf * KBUF + cg * 16;  // box row r of this thread at rows + 256 r
+    // conv taps as channel pairs: wv[tap][pair] = (w[2 pair][tap], w[2 pair + 1][tap])
+    float2 wv[4][4];
+    {
+      const __nv_bfloat16* wsm = reinterpret_cast<const __nv_bfloat16*>(smem + buf * KBUF + KW) + cg * 32;
+      float tmp[32];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) load8(wsm + r * 8, tmp + r * 8);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int tap = 0; tap < 4; ++tap) wv[tap][q] = make_float2(tmp[(2 * q) * 4 + tap], tmp[(2 * q + 1) * 4 + tap]);
+    }
     auto row2 = [&](int r, float2* f) {  // eight bf16 of box row r as four channel pairs
       const uint4 u = *reinterpret_cast<const uint4*>(rows + 256 * r);
       const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -433,20 +450,15 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
       store(t, y0, f0);
       if (has1) store(t + 1, y1, f1);
     }
-    if (!is_qk && cg == 0) {
+    if (gates) {
       // gates of value head hh for this thread's tokens
-      const int hh = ct - 2 * p.Hk;
       const float eA = expf(__ldg(p.A_log + hh)), db = __ldg(p.dt_bias + hh);
-      const __nv_bfloat16* ap = static_cast<const __nv_bfloat16*>(p.a);
-      const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int t = t0 + kk;
         if (t >= p.T) break;
-        const float av = ld_f(ap + (size_t)t * p.Hv + hh);
-        const float bv = ld_f(bp + (size_t)t * p.Hv + hh);
-        p.g[(size_t)hh * p.T + t] = -eA * softplus_f(av + db);
-        p.beta[(size_t)hh * p.T + t] = sigmoid_f(bv);
+        p.g[(size_t)hh * p.T + t] = -eA * softplus_f(av[kk] + db);
+        p.beta[(size_t)hh * p.T + t] = sigmoid_f(bv[kk]);
       }
     }
     __syncthreads();  // this buffer is read; the next iteration's prefetch may refill it
