@@ -159,7 +159,9 @@ __global__ void __launch_bounds__(NTA, 2)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7, tl = tid & 127;
-  const int g = blockIdx.x, h = blockIdx.y;
+  // heads vary fastest and chunk slots run from the last down, so that the
+  // records the chains read first are the most recently written (in L2)
+  const int g = (int)(gridDim.y - 1 - blockIdx.y), h = blockIdx.x;
   pdl_launch();
   // the sequence whose chunk owns this slot
   int lo = 0, hi = p.N - 1;
@@ -827,9 +829,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         // O = D + Pt V, back into TMEM, and its sum of squares over this CTA's columns
         ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;  // the stage's copies are seen here too
         ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
-        // start once the state update of this chunk is under way: the new-value
-        // threads' TMEM reads come first
-        ok = mbar_wait(bar_s + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
         tc_fence_after();
         GDN_SPLIT_MARK(16);
 #pragma unroll 1
@@ -1206,7 +1205,7 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)record_slots(p.N, p.T), (unsigned)p.Hv, 1);
+    cfg.gridDim = dim3((unsigned)p.Hv, (unsigned)record_slots(p.N, p.T), 1);
     cfg.blockDim = dim3(NTA, 1, 1);
     cfg.dynamicSmemBytes = A_SMEM;
     cfg.stream = st;
