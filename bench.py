@@ -117,11 +117,11 @@ def prefill_counts(inp, chunk):
                 call_flops=core_flops)
 
 
-def decode_counts(inp):
+def decode_counts(inp, state_bytes=4):
     w = inp.w
     B, Hv, d = inp.mixed_qkv.shape[0], w.Hv, w.d
     e = 2 if w.dtype == "bf16" else 4
-    state = 2 * B * Hv * d * d * 4
+    state = 2 * B * Hv * d * d * state_bytes
     conv = 2 * B * w.Cc * 3 * e
     io = B * (w.Cc * e + 2 * Hv * e + Hv * d * e + Hv * d * e)
     return dict(bytes=state + conv + io, flops=B * Hv * 6 * d * d)
@@ -401,31 +401,36 @@ def run_ours(args, rank, world, local_rank):
            "pipelined": "two buffer sets; copy-in, compute and copy-out streams"}
     del host, h_out, h_S, slots
 
-    # ---------------- decode half of the metric
+    # ---------------- decode half of the metric (fp32 state; then a bf16 state)
     wd = WORKLOADS[args.decode_workload]
     dinp = make_decode(wd)
-    dd = api.decode_to_device(dinp, device=dev)
-    dout = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dev)
-    for _ in range(args.warmup):
-        api.decode(dd, out=dout)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    dev_ms = []
-    for i in range(args.steps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        api.decode(dd, out=dout)
-        b.record(stream)
-        dev_ms.append((a, b))
-    torch.cuda.synchronize()
-    d_ms = [a.elapsed_time(b) for a, b in dev_ms]
-    d_total = max_over_ranks(sum(d_ms), dev)
+
+    def time_decode(state_dtype):
+        dd = api.decode_to_device(dinp, device=dev, state_dtype=state_dtype)
+        dout = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dev)
+        for _ in range(args.warmup):
+            api.decode(dd, out=dout)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        dev_ms = []
+        for i in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            api.decode(dd, out=dout)
+            b.record(stream)
+            dev_ms.append((a, b))
+        torch.cuda.synchronize()
+        d_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in dev_ms), dev)
+        state_mib = dd.state.numel() * dd.state.element_size() >> 20
+        del dd
+        return d_total / args.steps * 1e-3, state_mib
+
+    d_step_s, state_mib = time_decode(torch.float32)
     dcnt = decode_counts(dinp)
-    d_step_s = d_total / args.steps * 1e-3
     decode = {
         "metric": "GDN decode tokens/s per layer", "unit": "tokens/s",
-        "value": job_throughput(dd.B, world, d_step_s), "ms_per_step": d_step_s * 1e3,
+        "value": job_throughput(dinp.mixed_qkv.shape[0], world, d_step_s), "ms_per_step": d_step_s * 1e3,
         "workload": args.decode_workload,
         "roofline": {"kernel": "gdn_decode", "bound": "hbm",
                      "achieved": dcnt["bytes"] / d_step_s / 1e9, "peak": hbm, "unit": "GB/s",
@@ -433,9 +438,20 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": args.decode_traffic if args.decode_traffic is not None else
                                 profiled_traffic("decode.cu", args.decode_workload),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": dcnt["bytes"]},
-        "l2": "state (%d MiB) larger than L2" % (dd.state.numel() * 4 >> 20),
+        "l2": "state (%d MiB) larger than L2" % state_mib,
     }
-    del dd
+    # the same step with the recurrent state held in bf16 (half the state bytes)
+    b_step_s, b_state_mib = time_decode(torch.bfloat16)
+    bcnt = decode_counts(dinp, state_bytes=2)
+    decode["bf16_state"] = {
+        "value": job_throughput(dinp.mixed_qkv.shape[0], world, b_step_s), "unit": "tokens/s",
+        "ms_per_step": b_step_s * 1e3,
+        "roofline": {"kernel": "gdn_decode (bf16 state)", "bound": "hbm",
+                     "achieved": bcnt["bytes"] / b_step_s / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": bcnt["bytes"] / b_step_s / 1e9 / hbm, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": bcnt["bytes"]},
+        "l2": "state (%d MiB) larger than L2" % b_state_mib,
+    }
 
     result = {
         "metric": "GDN prefill tokens/s per layer (decode tokens/s under 'decode')",

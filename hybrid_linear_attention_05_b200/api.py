@@ -123,7 +123,10 @@ class DeviceDecode:
     conv_state: torch.Tensor
 
 
-def decode_to_device(inp: DecodeInputs, device="cuda") -> DeviceDecode:
+def decode_to_device(inp: DecodeInputs, device="cuda", state_dtype=torch.float32) -> DeviceDecode:
+    """The decode inputs on the device; the state in `state_dtype` (fp32, or
+    bf16 for the bf16-state step -- the caller rounds the state beforehand if
+    it wants the device to hold exactly the values it has)."""
     w = inp.w
     dt = _torch_dtype(w.dtype)
 
@@ -134,7 +137,7 @@ def decode_to_device(inp: DecodeInputs, device="cuda") -> DeviceDecode:
         Hk=w.Hk, Hv=w.Hv, d=w.d, scale=w.scale, B=inp.mixed_qkv.shape[0],
         mixed_qkv=t(inp.mixed_qkv), conv_w=t(inp.conv_w), a=t(inp.a), b=t(inp.b),
         A_log=t(inp.A_log, torch.float32), dt_bias=t(inp.dt_bias, torch.float32), z=t(inp.z),
-        norm_w=t(inp.norm_w), state=t(inp.state, torch.float32), conv_state=t(inp.conv_state))
+        norm_w=t(inp.norm_w), state=t(inp.state, state_dtype), conv_state=t(inp.conv_state))
 
 
 def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -145,5 +148,5 @@ def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None) -> torch.Tensor
     gdn.gdn_decode(dims, mixed_qkv=dd.mixed_qkv, conv_w=dd.conv_w, a=dd.a, b=dd.b,
                    A_log=dd.A_log, dt_bias=dd.dt_bias, z=dd.z, norm_w=dd.norm_w, state=dd.state,
                    conv_state=dd.conv_state, out=out, B=dd.B,
-                   dtype=gdn.dtype_code(dd.mixed_qkv))
+                   dtype=gdn.dtype_code(dd.mixed_qkv), state_dtype=gdn.dtype_code(dd.state))
     return out

@@ -13,17 +13,45 @@
 //   4. gated RMSNorm of o with z.
 // The state rows are spread over the warps with each lane holding a float4 of
 // a row; row dot products are shuffle reductions over the lanes of the row.
-// HBM traffic is dominated by the fp32 state: 2 * Hv * dk * dv * 4 bytes per
-// token ("Qwen3.5", HF model doc, Usage tips: the single-token recurrence is
-// memory-bandwidth-bound).
+// HBM traffic is dominated by the state: 2 * Hv * dk * dv * 4 bytes per
+// token in fp32, half that with a bf16 state ("Qwen3.5", HF model doc, Usage
+// tips: the single-token recurrence is memory-bandwidth-bound).  A bf16
+// state is widened to fp32 on load and rounded to nearest on store; all
+// arithmetic is fp32.
 #include "gdn_internal.h"
 
 namespace gdn {
 
 namespace {
 
-template <typename T, int D>
+// Four consecutive state entries (one lane's share of a row) in the state's
+// storage type, widened to / narrowed from fp32.
+template <typename S> struct State4;
+template <> struct State4<float> {
+  using Raw = float4;
+  static __device__ __forceinline__ Raw load(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ float4 widen(Raw r) { return r; }
+  static __device__ __forceinline__ void store(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+};
+template <> struct State4<__nv_bfloat16> {
+  using Raw = uint2;
+  static __device__ __forceinline__ Raw load(const __nv_bfloat16* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+  static __device__ __forceinline__ float4 widen(Raw r) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float4 v) {
+    uint2 r;
+    *reinterpret_cast<__nv_bfloat162*>(&r.x) = __floats2bfloat162_rn(v.x, v.y);
+    *reinterpret_cast<__nv_bfloat162*>(&r.y) = __floats2bfloat162_rn(v.z, v.w);
+    __stcs(reinterpret_cast<uint2*>(p), r);
+  }
+};
+
+template <typename T, typename SD, int D>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
+  using SV = State4<SD>;
   constexpr int NT = 256, NW = NT / 32;
   constexpr int LPR = D / 4;            // lanes per state row
   constexpr int RPW = 32 / LPR;         // rows per warp per pass
@@ -48,13 +76,14 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   // The first value head's state rows are requested before anything else:
   // they do not depend on the conv, so their HBM latency overlaps steps 1-2.
   const int col = (lane % LPR) * 4;
-  auto state_of = [&](int gi) { return p.state + ((size_t)b * p.Hv + kh * G + gi) * D * D; };
+  SD* const state = static_cast<SD*>(p.state);
+  auto state_of = [&](int gi) { return state + ((size_t)b * p.Hv + kh * G + gi) * D * D; };
   auto row_of = [&](int s) { return warp * ROWS_PER_WARP + s * RPW + lane / LPR; };
-  float4 Sv[PASSES];
+  typename SV::Raw Sv[PASSES];
   {
-    const float* S0 = state_of(0);
+    const SD* S0 = state_of(0);
 #pragma unroll
-    for (int s = 0; s < PASSES; ++s) Sv[s] = __ldcs(reinterpret_cast<const float4*>(S0 + (size_t)row_of(s) * D + col));
+    for (int s = 0; s < PASSES; ++s) Sv[s] = SV::load(S0 + (size_t)row_of(s) * D + col);
   }
 
   // 1. conv + SiLU, cache update in place (each channel read then written by one thread)
@@ -113,14 +142,15 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   for (int gi = 0; gi < G; ++gi) {
     const int h = kh * G + gi;
     const float alpha = misc[4 + gi], beta = misc[4 + G + gi];
-    float* Sh = p.state + ((size_t)b * p.Hv + h) * D * D;
-    const float* Snext = gi + 1 < G ? state_of(gi + 1) : nullptr;
+    SD* Sh = state + ((size_t)b * p.Hv + h) * D * D;
+    const SD* Snext = gi + 1 < G ? state_of(gi + 1) : nullptr;
     const float* vv = ys + (2 + gi) * D;
 #pragma unroll
     for (int s = 0; s < PASSES; ++s) {
       const int r = row_of(s);
-      float u = Sv[s].x * k4.x + Sv[s].y * k4.y + Sv[s].z * k4.z + Sv[s].w * k4.w;
-      float pp = Sv[s].x * q4.x + Sv[s].y * q4.y + Sv[s].z * q4.z + Sv[s].w * q4.w;
+      const float4 sv = SV::widen(Sv[s]);
+      float u = sv.x * k4.x + sv.y * k4.y + sv.z * k4.z + sv.w * k4.w;
+      float pp = sv.x * q4.x + sv.y * q4.y + sv.z * q4.z + sv.w * q4.w;
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) {
         u += __shfl_xor_sync(0xffffffffu, u, o, 32);
@@ -128,13 +158,13 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
       }
       const float delta = beta * (vv[r] - alpha * u);
       float4 sn;
-      sn.x = fmaf(alpha, Sv[s].x, delta * k4.x);
-      sn.y = fmaf(alpha, Sv[s].y, delta * k4.y);
-      sn.z = fmaf(alpha, Sv[s].z, delta * k4.z);
-      sn.w = fmaf(alpha, Sv[s].w, delta * k4.w);
-      __stcs(reinterpret_cast<float4*>(Sh + (size_t)r * D + col), sn);
+      sn.x = fmaf(alpha, sv.x, delta * k4.x);
+      sn.y = fmaf(alpha, sv.y, delta * k4.y);
+      sn.z = fmaf(alpha, sv.z, delta * k4.z);
+      sn.w = fmaf(alpha, sv.w, delta * k4.w);
+      SV::store(Sh + (size_t)r * D + col, sn);
       if ((lane % LPR) == 0) os[gi * D + r] = fmaf(alpha, pp, kq * delta);
-      if (Snext) Sv[s] = __ldcs(reinterpret_cast<const float4*>(Snext + (size_t)r * D + col));
+      if (Snext) Sv[s] = SV::load(Snext + (size_t)r * D + col);
     }
   }
   __syncthreads();
@@ -154,17 +184,21 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
+template <typename T, typename SD, int D>
+cudaError_t launch_ts(const DecodeParams& p, cudaStream_t st) {
   const int G = p.Hv / p.Hk;
   const size_t smem = ((size_t)(2 + G) * D + (size_t)G * D + 4 + 2 * G) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, SD, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  decode_kernel<T, D><<<p.B * p.Hk, 256, smem, st>>>(p);
+  decode_kernel<T, SD, D><<<p.B * p.Hk, 256, smem, st>>>(p);
   return cudaGetLastError();
+}
+template <typename T, int D>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
+  return p.state_bf16 ? launch_ts<T, __nv_bfloat16, D>(p, st) : launch_ts<T, float, D>(p, st);
 }
 
 }  // namespace

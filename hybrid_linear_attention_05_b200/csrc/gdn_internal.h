@@ -98,11 +98,12 @@ struct DecodeParams {
   const float* dt_bias;
   const void* z;              // [B, Hv*d]
   const void* norm_w;         // [d]
-  float* state;               // [B, Hv, d, d]
+  void* state;                // [B, Hv, d, d] fp32 or bf16 (state_bf16)
   void* conv_state;           // [B, Cc, 3]
   void* out;                  // [B, Hv, d]
   int B, Hk, Hv, Cc;
   float scale, eps_l2, eps_norm;
+  bool state_bf16;
 };
 cudaError_t launch_decode(const DecodeParams& p, int d, gdn_dtype dt, cudaStream_t st);
 

@@ -213,6 +213,13 @@ gdn_status gdn_prefill_noalloc(const gdn_dims* dims, const gdn_prefill_args* arg
 /* ------------------------------------------------------------------- decode
  * One token for each of B independent sequences.  state and conv_state are
  * read and overwritten in place with the values after this token.
+ *
+ * The recurrent state is fp32 by default.  With state_dtype = GDN_BF16 it is
+ * held in bf16 ([B, Hv, dv, dk], 2 bytes per entry), which halves the HBM
+ * bytes of this bandwidth-bound step ("Qwen3.5", HF model doc, Usage tips: the
+ * single-token recurrence is memory-bandwidth-bound): the step reads the bf16
+ * state, computes in fp32 and writes the new state rounded to the nearest
+ * bf16; out is computed from the unrounded fp32 state.
  */
 typedef struct {
   const void* mixed_qkv;       /* device [B, Cc]          dtype                     */
@@ -223,11 +230,12 @@ typedef struct {
   const float* dt_bias;        /* device [Hv]             fp32                      */
   const void* z;               /* device [B, Hv*dv]       dtype                     */
   const void* norm_w;          /* device [dv]             dtype                     */
-  float* state;                /* device [B, Hv, dv, dk]  fp32, in place            */
+  void* state;                 /* device [B, Hv, dv, dk]  state_dtype, in place     */
   void* conv_state;            /* device [B, Cc, 3]       dtype, in place           */
   void* out;                   /* device [B, Hv, dv]      dtype                     */
   int B;                       /* batch (>= 0)                                      */
   gdn_dtype dtype;
+  gdn_dtype state_dtype;       /* GDN_F32 (0, the default) or GDN_BF16             */
 } gdn_decode_args;
 
 gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* args, void* stream);

@@ -147,6 +147,8 @@ def decode_kwargs(**over):
     (dict(out=FAKE + 2), gdn.GDN_ERR_ALIGN),
     (dict(B=-1), gdn.GDN_ERR_DIMS),
     (dict(B=0), gdn.GDN_OK),
+    (dict(state_dtype=7), gdn.GDN_ERR_DIMS),
+    (dict(state_dtype=gdn.GDN_F16), gdn.GDN_ERR_DIMS),
 ])
 def test_decode_rejects_bad_args(L, over, status):
     assert gdn.gdn_decode(gdn.make_dims(2, 4, 128), **decode_kwargs(**over)) == status

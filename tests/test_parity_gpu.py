@@ -308,6 +308,50 @@ def test_decode_fp32(d, Hk, Hv):
     np.testing.assert_array_equal(np64(dd.conv_state), ref_cs)
 
 
+def test_decode_bf16_state_full_batch():
+    """The decode workload with its recurrent state held in bf16 (256 MiB):
+    the step widens the state to fp32, updates it and rounds it back.  The
+    oracle runs in fp64 from the same bf16 values; the new state and out
+    must match beyond their own bf16 rounding."""
+    import dataclasses
+    from hybrid_linear_attention_05_b200.workloads import bf16_round
+    inp = make_decode(D9B)
+    inp = dataclasses.replace(inp, state=bf16_round(inp.state))
+    dd = api.decode_to_device(inp, state_dtype=torch.bfloat16)
+    out = api.decode(dd)
+    torch.cuda.synchronize()
+    ref_out, ref_S, ref_cs = oracle_decode(inp)
+    assert relerr_beyond_bf16(np64(dd.state), ref_S) <= DECODE_TOL
+    assert relerr_beyond_bf16(np64(out), ref_out) <= DECODE_TOL
+    np.testing.assert_array_equal(np64(dd.conv_state), ref_cs)
+
+
+@pytest.mark.parametrize("d,Hk,Hv,dtype", [(32, 2, 2, "f32"), (64, 2, 8, "bf16"), (128, 4, 16, "f32")])
+def test_decode_bf16_state_shapes(d, Hk, Hv, dtype):
+    """bf16 state at every head width, with fp32 and bf16 token inputs, over
+    three steps in a row (each step reads the state the previous one rounded)."""
+    import dataclasses
+    from hybrid_linear_attention_05_b200.workloads import bf16_round
+    w = resized(D9B, Hk=Hk, Hv=Hv, d=d, dtype=dtype, seed=90 + d)
+    inp = make_decode(w, batch=5)
+    inp = dataclasses.replace(inp, state=bf16_round(inp.state))
+    dd = api.decode_to_device(inp, state_dtype=torch.bfloat16)
+    state, conv = inp.state, inp.conv_state
+    for step in range(3):
+        out = api.decode(dd)
+        torch.cuda.synchronize()
+        cur = dataclasses.replace(inp, state=state, conv_state=conv)
+        ref_out, ref_S, ref_cs = oracle_decode(cur)
+        got_S = np64(dd.state)
+        assert relerr_beyond_bf16(got_S, ref_S) <= DECODE_TOL, step
+        if dtype == "f32":
+            assert relerr(np64(out), ref_out) <= DECODE_TOL, step
+        else:
+            assert relerr_beyond_bf16(np64(out), ref_out) <= DECODE_TOL, step
+        np.testing.assert_array_equal(np64(dd.conv_state), ref_cs)
+        state, conv = got_S.astype(np.float32), ref_cs.astype(np.float32)
+
+
 def test_prefill_then_decode_composition():
     """prefill of T tokens followed by a decode of token T+1 equals the
     oracle's prefill of T+1 tokens (state and last output)."""
