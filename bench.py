@@ -117,13 +117,15 @@ def prefill_counts(inp, chunk):
                 call_flops=core_flops)
 
 
-def decode_counts(inp, state_bytes=4):
+def decode_counts(inp, state_bytes=4, T=1):
+    """Algorithmic bytes of one decode step of T tokens for each of the
+    workload's sequences (the token rows of `inp` are T per sequence)."""
     w = inp.w
-    B, Hv, d = inp.mixed_qkv.shape[0], w.Hv, w.d
+    B, Hv, d = inp.mixed_qkv.shape[0] // T, w.Hv, w.d
     e = 2 if w.dtype == "bf16" else 4
     state = 2 * B * Hv * d * d * state_bytes
     conv = 2 * B * w.Cc * 3 * e
-    io = B * (w.Cc * e + 2 * Hv * e + Hv * d * e + Hv * d * e)
+    io = B * T * (w.Cc * e + 2 * Hv * e + Hv * d * e + Hv * d * e)
     return dict(bytes=state + conv + io, flops=B * Hv * 6 * d * d)
 
 
@@ -405,11 +407,18 @@ def run_ours(args, rank, world, local_rank):
     wd = WORKLOADS[args.decode_workload]
     dinp = make_decode(wd)
 
-    def time_decode(state_dtype):
-        dd = api.decode_to_device(dinp, device=dev, state_dtype=state_dtype)
-        dout = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dev)
+    def time_decode(state_dtype, T=1, src=None):
+        dd = api.decode_to_device(src or dinp, device=dev, state_dtype=state_dtype)
+        if T > 1:  # token rows b * T + t; the state and conv cache of the first B rows
+            B = dd.B // T
+            dd = api.DeviceDecode(Hk=dd.Hk, Hv=dd.Hv, d=dd.d, scale=dd.scale, B=B, mixed_qkv=dd.mixed_qkv,
+                                  conv_w=dd.conv_w, a=dd.a, b=dd.b, A_log=dd.A_log, dt_bias=dd.dt_bias,
+                                  z=dd.z, norm_w=dd.norm_w, state=dd.state[:B].contiguous(),
+                                  conv_state=dd.conv_state[:B].contiguous())
+        shape = (dd.B, dd.Hv, dd.d) if T == 1 else (dd.B, T, dd.Hv, dd.d)
+        dout = torch.empty(shape, dtype=dd.mixed_qkv.dtype, device=dev)
         for _ in range(args.warmup):
-            api.decode(dd, out=dout)
+            api.decode(dd, out=dout, T=T)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -417,7 +426,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.steps):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            api.decode(dd, out=dout)
+            api.decode(dd, out=dout, T=T)
             b.record(stream)
             dev_ms.append((a, b))
         torch.cuda.synchronize()
@@ -451,6 +460,20 @@ def run_ours(args, rank, world, local_rank):
                      "frac": bcnt["bytes"] / b_step_s / 1e9 / hbm, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": bcnt["bytes"]},
         "l2": "state (%d MiB) larger than L2" % b_state_mib,
+    }
+    # short multi-token decode: T = 4 tokens per sequence and step (fp32 state)
+    T_mt = 4
+    mt_inp = make_decode(wd, batch=dinp.mixed_qkv.shape[0] * T_mt)
+    m_step_s, _ = time_decode(torch.float32, T=T_mt, src=mt_inp)
+    mcnt = decode_counts(mt_inp, T=T_mt)
+    decode["multi_token"] = {
+        "tokens_per_sequence": T_mt,
+        "value": job_throughput(dinp.mixed_qkv.shape[0] * T_mt, world, m_step_s), "unit": "tokens/s",
+        "ms_per_step": m_step_s * 1e3,
+        "roofline": {"kernel": "gdn_decode (T = 4)", "bound": "hbm",
+                     "achieved": mcnt["bytes"] / m_step_s / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": mcnt["bytes"] / m_step_s / 1e9 / hbm, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": mcnt["bytes"]},
     }
 
     result = {

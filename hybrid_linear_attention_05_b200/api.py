@@ -140,13 +140,15 @@ def decode_to_device(inp: DecodeInputs, device="cuda", state_dtype=torch.float32
         norm_w=t(inp.norm_w), state=t(inp.state, state_dtype), conv_state=t(inp.conv_state))
 
 
-def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """One step; dd.state and dd.conv_state are updated in place."""
+def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None, T: int = 1) -> torch.Tensor:
+    """One step of T tokens per sequence (token inputs [B, T, ...] when T > 1);
+    dd.state and dd.conv_state are updated in place."""
     if out is None:
-        out = torch.empty((dd.B, dd.Hv, dd.d), dtype=dd.mixed_qkv.dtype, device=dd.mixed_qkv.device)
+        shape = (dd.B, dd.Hv, dd.d) if T == 1 else (dd.B, T, dd.Hv, dd.d)
+        out = torch.empty(shape, dtype=dd.mixed_qkv.dtype, device=dd.mixed_qkv.device)
     dims = gdn.make_dims(dd.Hk, dd.Hv, dd.d, scale=dd.scale)
     gdn.gdn_decode(dims, mixed_qkv=dd.mixed_qkv, conv_w=dd.conv_w, a=dd.a, b=dd.b,
                    A_log=dd.A_log, dt_bias=dd.dt_bias, z=dd.z, norm_w=dd.norm_w, state=dd.state,
                    conv_state=dd.conv_state, out=out, B=dd.B,
-                   dtype=gdn.dtype_code(dd.mixed_qkv), state_dtype=gdn.dtype_code(dd.state))
+                   dtype=gdn.dtype_code(dd.mixed_qkv), state_dtype=gdn.dtype_code(dd.state), T=T)
     return out

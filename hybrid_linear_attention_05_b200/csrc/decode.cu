@@ -3,14 +3,17 @@
 // One CTA per (sequence, key head) owns the G = Hv/Hk value heads that read
 // that key head, so the conv-cache channels it updates in place (its q and k
 // head, and its G value heads) belong to no other CTA.
-//   1. conv over (cache[0..2], new input) + SiLU for those channels, cache
-//      shifted left with the new raw input appended;
+//   1. conv over (cache[0..2], the new inputs) + SiLU for those channels,
+//      cache shifted left with the new raw inputs appended;
 //   2. L2 norm of q and k, gates alpha = exp(-exp(A_log) softplus(a+dt_bias)),
 //      beta = sigmoid(b);
 //   3. each state row S[r, :] (dk floats) is read once from HBM and written
 //      once: u = S k, p = S q, delta = beta (v - alpha u),
 //      S' = alpha S + delta k^T, o = alpha p + (k.q) delta   (= S' q);
 //   4. gated RMSNorm of o with z.
+// A step may carry T = 1..8 tokens per sequence (short multi-token decode,
+// e.g. verifying drafted tokens): each state row then takes the T updates in
+// turn while it is in registers, so the state is still read and written once.
 // The state rows are spread over the warps with each lane holding a float4 of
 // a row; row dot products are shuffle reductions over the lanes of the row.
 // HBM traffic is dominated by the state: 2 * Hv * dk * dv * 4 bytes per
@@ -184,16 +187,185 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   }
 }
 
+// The same step for p.T = 2..8 tokens per sequence (short multi-token
+// decode): each state row takes the T tokens' updates in turn while it is in
+// registers, so the state is still read and written once per step.
+template <typename T, typename SD, int D>
+__global__ void __launch_bounds__(256, 2) decode_multi_kernel(DecodeParams p) {
+  using SV = State4<SD>;
+  constexpr int NT = 256, NW = NT / 32;
+  constexpr int LPR = D / 4;            // lanes per state row
+  constexpr int RPW = 32 / LPR;         // rows per warp per pass
+  constexpr int ROWS_PER_WARP = D / NW; // rows of one head handled by a warp
+  constexpr int PASSES = ROWS_PER_WARP / RPW;
+  static_assert(PASSES >= 1, "decode layout");
+
+  extern __shared__ float sm[];
+  const int G = p.Hv / p.Hk;
+  const int TK = p.T;             // tokens of every sequence in this step
+  const int NC = (2 + G) * D;     // channels of this CTA
+  const int MS = 4 + 2 * G;
+  float* ys = sm;                 // [TK][NC] q | k | v of each token
+  float* os = ys + TK * NC;       // [TK][G * D] core outputs
+  float* misc = os + TK * G * D;  // [TK][MS]: rq, rk, kq, -, alpha[G], beta[G]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x / p.Hk, kh = blockIdx.x % p.Hk;
+  const int Cc = p.Cc;
+  const T* xb = static_cast<const T*>(p.x) + (size_t)b * TK * Cc;  // token t at xb + t Cc
+  T* cs = static_cast<T*>(p.conv_state) + (size_t)b * Cc * 3;
+  const T* cw = static_cast<const T*>(p.conv_w);
+
+  // A thread's rows of a head are taken RG at a time (a "group"); the first
+  // group is requested before anything else, each next one while the current
+  // one is updated, so the state latency overlaps the conv and the updates.
+  constexpr int RG = PASSES < 8 ? PASSES : 8;
+  constexpr int NGH = PASSES / RG;  // groups per head
+  const int col = (lane % LPR) * 4;
+  SD* const state = static_cast<SD*>(p.state);
+  auto row_of = [&](int s) { return warp * ROWS_PER_WARP + s * RPW + lane / LPR; };
+  // group q: head q / NGH, passes (q % NGH) RG .. + RG - 1
+  auto group_ptr = [&](int q, int j) {
+    return state + ((size_t)b * p.Hv + kh * G + q / NGH) * D * D + (size_t)row_of((q % NGH) * RG + j) * D + col;
+  };
+  typename SV::Raw Sv[RG];
+#pragma unroll
+  for (int j = 0; j < RG; ++j) Sv[j] = SV::load(group_ptr(0, j));
+
+  // 1. conv + SiLU over [cache, x_0 .. x_{TK-1}]; the cache keeps the last
+  //    three raw inputs (each channel read then written by one thread)
+  for (int idx = tid; idx < NC; idx += NT) {
+    int c;
+    if (idx < D) c = kh * D + idx;
+    else if (idx < 2 * D) c = p.Hk * D + kh * D + (idx - D);
+    else c = 2 * p.Hk * D + kh * G * D + (idx - 2 * D);
+    const float w0 = ld_f(cw + (size_t)c * 4 + 0), w1 = ld_f(cw + (size_t)c * 4 + 1);
+    const float w2 = ld_f(cw + (size_t)c * 4 + 2), w3 = ld_f(cw + (size_t)c * 4 + 3);
+    float h0 = ld_f(cs + (size_t)c * 3 + 0);
+    float h1 = ld_f(cs + (size_t)c * 3 + 1);
+    float h2 = ld_f(cs + (size_t)c * 3 + 2);
+    for (int t = 0; t < TK; ++t) {
+      const float xn = ld_f(xb + (size_t)t * Cc + c);
+      float y = w0 * h0;
+      y = fmaf(w1, h1, y);
+      y = fmaf(w2, h2, y);
+      y = fmaf(w3, xn, y);
+      ys[t * NC + idx] = silu_f(y);
+      h0 = h1;
+      h1 = h2;
+      h2 = xn;
+    }
+    st_f(cs + (size_t)c * 3 + 0, h0);
+    st_f(cs + (size_t)c * 3 + 1, h1);
+    st_f(cs + (size_t)c * 3 + 2, h2);
+  }
+  __syncthreads();
+  // 2. norms and gates of every token
+  for (int job = warp; job < 2 * TK; job += NW) {  // the q (even) and k (odd) norms
+    const int t = job >> 1, which = job & 1;
+    const float* y = ys + t * NC + which * D;
+    float ss = 0.f;
+    for (int i = lane; i < D; i += 32) ss = fmaf(y[i], y[i], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) misc[t * MS + which] = rsqrtf(ss + p.eps_l2) * (which == 0 ? p.scale : 1.0f);
+  }
+  for (int j = tid; j < TK * G; j += NT) {
+    const int t = j / G, gi = j % G, h = kh * G + gi;
+    const size_t row = (size_t)b * TK + t;
+    const float av = ld_f(static_cast<const T*>(p.a) + row * p.Hv + h);
+    const float bv = ld_f(static_cast<const T*>(p.b) + row * p.Hv + h);
+    const float gg = -expf(__ldg(p.A_log + h)) * softplus_f(av + __ldg(p.dt_bias + h));
+    misc[t * MS + 4 + gi] = expf(gg);
+    misc[t * MS + 4 + G + gi] = sigmoid_f(bv);
+  }
+  __syncthreads();
+  for (int i = tid; i < TK * 2 * D; i += NT) {
+    const int t = i / (2 * D), j = i % (2 * D);
+    ys[t * NC + j] *= misc[t * MS + (j < D ? 0 : 1)];
+  }
+  __syncthreads();
+  for (int t = warp; t < TK; t += NW) {
+    const float* q = ys + t * NC;
+    float kq = 0.f;
+    for (int i = lane; i < D; i += 32) kq = fmaf(q[i], q[D + i], kq);
+    kq = warp_sum(kq);
+    if (lane == 0) misc[t * MS + 2] = kq;
+  }
+  __syncthreads();
+
+  // 3. state stream: a group of this thread's rows stays in registers while
+  //    the TK tokens update it in turn; the rows of one token are
+  //    independent, so their row reductions overlap.
+  for (int q = 0; q < G * NGH; ++q) {
+    const int gi = q / NGH;
+    float4 sv[RG];
+#pragma unroll
+    for (int j = 0; j < RG; ++j) sv[j] = SV::widen(Sv[j]);
+    if (q + 1 < G * NGH) {
+#pragma unroll
+      for (int j = 0; j < RG; ++j) Sv[j] = SV::load(group_ptr(q + 1, j));
+    }
+    for (int t = 0; t < TK; ++t) {
+      const float* qt = ys + t * NC;
+      const float4 q4 = *reinterpret_cast<const float4*>(qt + col);
+      const float4 k4 = *reinterpret_cast<const float4*>(qt + D + col);
+      const float alpha = misc[t * MS + 4 + gi], beta = misc[t * MS + 4 + G + gi], kq = misc[t * MS + 2];
+      float u[RG], pp[RG];
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        u[j] = sv[j].x * k4.x + sv[j].y * k4.y + sv[j].z * k4.z + sv[j].w * k4.w;
+        pp[j] = sv[j].x * q4.x + sv[j].y * q4.y + sv[j].z * q4.z + sv[j].w * q4.w;
+      }
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1)
+#pragma unroll
+        for (int j = 0; j < RG; ++j) {
+          u[j] += __shfl_xor_sync(0xffffffffu, u[j], o, 32);
+          pp[j] += __shfl_xor_sync(0xffffffffu, pp[j], o, 32);
+        }
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        const int r = row_of((q % NGH) * RG + j);
+        const float delta = beta * (qt[(2 + gi) * D + r] - alpha * u[j]);
+        sv[j].x = fmaf(alpha, sv[j].x, delta * k4.x);
+        sv[j].y = fmaf(alpha, sv[j].y, delta * k4.y);
+        sv[j].z = fmaf(alpha, sv[j].z, delta * k4.z);
+        sv[j].w = fmaf(alpha, sv[j].w, delta * k4.w);
+        if ((lane % LPR) == 0) os[(t * G + gi) * D + r] = fmaf(alpha, pp[j], kq * delta);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < RG; ++j) SV::store(group_ptr(q, j), sv[j]);
+  }
+  __syncthreads();
+
+  // 4. gated RMSNorm, one warp per (token, value head)
+  for (int job = warp; job < TK * G; job += NW) {
+    const int t = job / G, gi = job % G, h = kh * G + gi;
+    const float* o = os + (t * G + gi) * D;
+    float ss = 0.f;
+    for (int r = lane; r < D; r += 32) ss = fmaf(o[r], o[r], ss);
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / D + p.eps_norm);
+    const size_t row = ((size_t)b * TK + t) * p.Hv + h;
+    const T* zz = static_cast<const T*>(p.z) + row * D;
+    T* oo = static_cast<T*>(p.out) + row * D;
+    const T* ww = static_cast<const T*>(p.norm_w);
+    for (int r = lane; r < D; r += 32) st_f(oo + r, o[r] * inv * ld_f(ww + r) * silu_f(ld_f(zz + r)));
+  }
+}
+
 template <typename T, typename SD, int D>
 cudaError_t launch_ts(const DecodeParams& p, cudaStream_t st) {
   const int G = p.Hv / p.Hk;
-  const size_t smem = ((size_t)(2 + G) * D + (size_t)G * D + 4 + 2 * G) * sizeof(float);
+  const size_t smem = (size_t)p.T * ((size_t)(2 + G) * D + (size_t)G * D + 4 + 2 * G) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, SD, D>,
+    cudaError_t e = cudaFuncSetAttribute(p.T == 1 ? decode_kernel<T, SD, D> : decode_multi_kernel<T, SD, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  decode_kernel<T, SD, D><<<p.B * p.Hk, 256, smem, st>>>(p);
+  if (p.T == 1) decode_kernel<T, SD, D><<<p.B * p.Hk, 256, smem, st>>>(p);
+  else decode_multi_kernel<T, SD, D><<<p.B * p.Hk, 256, smem, st>>>(p);
   return cudaGetLastError();
 }
 template <typename T, int D>

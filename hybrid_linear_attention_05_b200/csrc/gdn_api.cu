@@ -185,6 +185,8 @@ gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* a, void* stre
   if (s != GDN_OK) return s;
   if (!a) return GDN_ERR_NULL;
   if (a->B < 0 || !dtype_ok(a->dtype) || !dtype_ok(a->state_dtype)) return GDN_ERR_DIMS;
+  if (a->T < 0) return GDN_ERR_DIMS;
+  if (a->T > 8) return GDN_ERR_UNSUPPORTED;
   if (a->B == 0) return GDN_OK;
   if (!a->mixed_qkv || !a->conv_w || !a->a || !a->b || !a->A_log || !a->dt_bias || !a->z ||
       !a->norm_w || !a->state || !a->conv_state || !a->out)
@@ -201,6 +203,7 @@ gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* a, void* stre
   p.B = a->B; p.Hk = dims->Hk; p.Hv = dims->Hv; p.Cc = 2 * dims->Hk * d + dims->Hv * d;
   p.scale = dims->scale; p.eps_l2 = dims->eps_l2; p.eps_norm = dims->eps_norm;
   p.state_bf16 = a->state_dtype == GDN_BF16;
+  p.T = a->T > 0 ? a->T : 1;
   return from_cuda(launch_decode(p, d, a->dtype, static_cast<cudaStream_t>(stream)));
 }
 

@@ -102,6 +102,7 @@ struct DecodeParams {
   void* conv_state;           // [B, Cc, 3]
   void* out;                  // [B, Hv, d]
   int B, Hk, Hv, Cc;
+  int T;                      // tokens per sequence in this step (1..8)
   float scale, eps_l2, eps_norm;
   bool state_bf16;
 };

@@ -65,7 +65,7 @@ class gdn_decode_args(ctypes.Structure):
     _fields_ = [("mixed_qkv", _vp), ("conv_w", _vp), ("a", _vp), ("b", _vp), ("A_log", _vp),
                 ("dt_bias", _vp), ("z", _vp), ("norm_w", _vp), ("state", _vp),
                 ("conv_state", _vp), ("out", _vp), ("B", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("state_dtype", ctypes.c_int)]
+                ("state_dtype", ctypes.c_int), ("T", ctypes.c_int)]
 
 
 class gdn_core_args(ctypes.Structure):
@@ -206,11 +206,11 @@ def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bi
 
 
 def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w, state,
-               conv_state, out, B, dtype, state_dtype=GDN_F32, stream=None,
+               conv_state, out, B, dtype, state_dtype=GDN_F32, T=1, stream=None,
                raise_on_error=True) -> int:
     args = gdn_decode_args(ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log),
                            ptr(dt_bias), ptr(z), ptr(norm_w), ptr(state), ptr(conv_state),
-                           ptr(out), int(B), int(dtype), int(state_dtype))
+                           ptr(out), int(B), int(dtype), int(state_dtype), int(T))
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_decode(ctypes.byref(dims), ctypes.byref(args), s), "gdn_decode",
                   raise_on_error)

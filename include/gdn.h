@@ -236,6 +236,14 @@ typedef struct {
   int B;                       /* batch (>= 0)                                      */
   gdn_dtype dtype;
   gdn_dtype state_dtype;       /* GDN_F32 (0, the default) or GDN_BF16             */
+  int T;                       /* tokens per sequence in this step: 1..8 (0 = 1).
+                                  With T > 1 the token inputs are [B, T, ...]
+                                  (mixed_qkv [B, T, Cc], a, b [B, T, Hv], z
+                                  [B, T, Hv*dv]) and out is [B, T, Hv, dv]; the
+                                  step equals T one-token steps (short
+                                  multi-token decode, e.g. verifying drafted
+                                  tokens), with the state read and written once.
+                                  T > 8 returns GDN_ERR_UNSUPPORTED.             */
 } gdn_decode_args;
 
 gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* args, void* stream);

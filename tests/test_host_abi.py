@@ -149,6 +149,8 @@ def decode_kwargs(**over):
     (dict(B=0), gdn.GDN_OK),
     (dict(state_dtype=7), gdn.GDN_ERR_DIMS),
     (dict(state_dtype=gdn.GDN_F16), gdn.GDN_ERR_DIMS),
+    (dict(T=-1), gdn.GDN_ERR_DIMS),
+    (dict(T=9), gdn.GDN_ERR_UNSUPPORTED),
 ])
 def test_decode_rejects_bad_args(L, over, status):
     assert gdn.gdn_decode(gdn.make_dims(2, 4, 128), **decode_kwargs(**over)) == status

@@ -352,6 +352,39 @@ def test_decode_bf16_state_shapes(d, Hk, Hv, dtype):
         state, conv = got_S.astype(np.float32), ref_cs.astype(np.float32)
 
 
+@pytest.mark.parametrize("T,state_dtype,d,Hk,Hv", [
+    (2, "f32", 128, 16, 32), (3, "f32", 32, 2, 2), (4, "f32", 64, 2, 8), (8, "bf16", 128, 4, 16)])
+def test_decode_multi_token(T, state_dtype, d, Hk, Hv):
+    """Short multi-token decode: one gdn_decode step of T tokens per sequence
+    equals the fp64 oracle's prefill of those T tokens from the same state and
+    conv history (out, final state, conv cache)."""
+    from hybrid_linear_attention_05_b200.workloads import bf16_round
+    w = resized(D9B, Hk=Hk, Hv=Hv, d=d, seed=100 + T)
+    B = 6
+    tok = make_decode(w, batch=B * T)  # row b * T + t: token t of sequence b
+    state = tok.state[:B].copy()
+    if state_dtype == "bf16":
+        state = bf16_round(state)
+    cs = tok.conv_state[:B].copy()
+    t = lambda x, dt=torch.bfloat16: torch.from_numpy(np.ascontiguousarray(x)).cuda().to(dt)  # noqa: E731
+    dd = api.DeviceDecode(
+        Hk=w.Hk, Hv=w.Hv, d=w.d, scale=w.scale, B=B, mixed_qkv=t(tok.mixed_qkv), conv_w=t(tok.conv_w),
+        a=t(tok.a), b=t(tok.b), A_log=t(tok.A_log, torch.float32), dt_bias=t(tok.dt_bias, torch.float32),
+        z=t(tok.z), norm_w=t(tok.norm_w),
+        state=t(state, torch.float32 if state_dtype == "f32" else torch.bfloat16), conv_state=t(cs))
+    out = api.decode(dd, T=T)
+    torch.cuda.synchronize()
+    cu = np.arange(B + 1, dtype=np.int32) * T
+    ref = oracle.prefill(w.Hk, w.Hv, w.d, w.d, cu, tok.mixed_qkv, tok.conv_w, tok.a, tok.b, tok.A_log,
+                         tok.dt_bias, tok.z, tok.norm_w, state, cs, scale=w.scale)
+    assert relerr_beyond_bf16(np64(out).reshape(B * T, w.Hv, w.d), ref.out) <= DECODE_TOL
+    if state_dtype == "f32":
+        assert relerr(np64(dd.state), ref.final_state) <= DECODE_TOL
+    else:
+        assert relerr_beyond_bf16(np64(dd.state), ref.final_state) <= DECODE_TOL
+    np.testing.assert_array_equal(np64(dd.conv_state), ref.conv_state_out)
+
+
 def test_prefill_then_decode_composition():
     """prefill of T tokens followed by a decode of token T+1 equals the
     oracle's prefill of T+1 tokens (state and last output)."""
