@@ -568,8 +568,10 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   const size_t nh = (size_t)n * p.Hv + h;
   // the state this CTA starts from (null: zero; transfer chains build theirs)
   // and where its last state goes (null: nowhere)
+  // (the R chain of segment 0 starts from S0 itself, so it leaves the state
+  // at the start of segment 1 and segment 0 needs no map M)
   auto start_state = [&]() -> const float* {
-    if (XFER) return nullptr;
+    if (XFER) return sg == 0 && p.S0 ? p.S0 + nh * hd + slice : nullptr;
     if (P == 1) return p.S0 ? p.S0 + nh * hd + slice : nullptr;
     return p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd + slice;
   };
@@ -580,6 +582,7 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   const bool norm_out = !XFER && p.out != nullptr;
   const bool want_u = !XFER || role == 1;  // the chain adds U to its new values
 
+  if (XFER && sg == 0 && role == 0) return;  // segment 0's map M is not needed
   if (nchunks == 0) {
     // empty segment; the last one is empty only for an empty sequence, whose
     // state passes through (every CTA of the cluster returns here)
@@ -668,7 +671,7 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
       float r[CW];
 #pragma unroll
       for (int j = 0; j < CW; ++j)
-        r[j] = XFER ? (role == 0 && col + j == tl ? 1.f : 0.f) : (Sin ? Sin[(size_t)(col + j) * D + tl] : 0.f);
+        r[j] = XFER && role == 0 ? (col + j == tl ? 1.f : 0.f) : (Sin ? Sin[(size_t)(col + j) * D + tl] : 0.f);
       tmem_stw<CW>(lane_base + G::TM_S + col, r);
       tmem_wait_st();
     }
@@ -972,8 +975,10 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
   const int nch = (eos - bos + C - 1) / C;
   auto nonempty = [&](int sg) { return seg_lo(nch, sg + 1, P) > seg_lo(nch, sg, P); };
   auto map_of = [&](int sg) { return p.seg_mr + ((((size_t)n * (P - 1) + sg) * p.Hv + h) * 2) * hd; };
-  // next non-empty segment at or after sg that has a map (sg < P - 1), or P - 1
+  // next non-empty segment at or after sg that has a map M (1 <= sg < P - 1;
+  // segment 0 has none: its R slot holds the state at the start of segment 1), or P - 1
   auto next_map = [&](int sg) {
+    if (sg < 1) sg = 1;
     while (sg < P - 1 && !nonempty(sg)) ++sg;
     return sg;
   };
@@ -991,7 +996,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
   }
   pdl_wait();  // the maps come from the transfer chains
   if (tid < P - 1 && nonempty(tid)) {  // every map and R slice this CTA will read, into L2
-    bulk_prefetch_l2(map_of(tid), D * D * 4);
+    if (tid > 0) bulk_prefetch_l2(map_of(tid), D * D * 4);
     bulk_prefetch_l2(map_of(tid) + hd + (size_t)r0 * D, SR * D * 4);
   }
   __syncthreads();
@@ -1021,6 +1026,18 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
             make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
     }
     if (sg + 1 >= P) break;
+    if (sg == 0) {  // segment 0: its R is the next start state (or, if it is empty, S0 passes)
+      if (owner && nonempty(0)) {
+        const float* R = map_of(0) + hd;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(R + (size_t)(r0 + rr + r) * D + cc));
+          acc[r][0] = make_float2(v.x, v.y);
+          acc[r][1] = make_float2(v.z, v.w);
+        }
+      }
+      continue;
+    }
     if (sg != sg_next) continue;  // empty segment: the state passes through
     // this segment's map: S <- S M + R (R is added by the owners after the
     // products, so its loads overlap them)
@@ -1247,9 +1264,10 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
 
 // Segments per sequence for the chain: the count that minimises an estimate
 // of the serial chain steps -- ceil(chunks / P) steps for the transfer chains
-// (per wave of them) plus as many for the output chains, about two per scan
-// step and two for the extra launches -- among those whose output chains fit
-// the SMs in one wave.  One serial chain takes `chunks` steps.
+// (per wave of them: 2 (P - 1) - 1 CTAs per chain, segment 0 needing no map)
+// plus as many for the output chains, about two per scan step (P - 2) and two
+// for the extra launches -- among those whose output chains fit the SMs in
+// one wave.  One serial chain takes `chunks` steps.
 int chunk_tc_split_auto_segments(int N, int T, int Hv) {
   const long chains = (long)N * Hv;
   if (N <= 0 || chains > kSegMaxChains) return 1;
@@ -1260,9 +1278,9 @@ int chunk_tc_split_auto_segments(int N, int T, int Hv) {
   for (int P = 3; P <= kSegMax; ++P) {
     if (chains * P > sms) break;
     const double seg = ceil(nch / P);
-    const double waves = ceil(2.0 * chains * (P - 1) / sms);
+    const double waves = ceil((double)chains * (2 * (P - 1) - 1) / sms);
     const double out_step = 2 * chains * P <= sms ? 1.0 : 1.15;  // whole-row chains are a little slower
-    const double cost = seg * waves + seg * out_step + 2.0 * (P - 1) + 2.0;
+    const double cost = seg * waves + seg * out_step + 2.0 * (P - 2) + 2.0;
     if (cost < best_cost) {
       best_cost = cost;
       best = P;
