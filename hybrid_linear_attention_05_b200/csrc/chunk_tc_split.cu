@@ -413,9 +413,11 @@ __global__ void __launch_bounds__(NTA, 2)
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
     // The record is assembled in shared memory regions the MMAs no longer
-    // read, then leaves in three bulk copies: [-W; Qt] over AW, [U; Pt V]
-    // over [K; Q], w * silu(z) over [Tb; Pt].
-    // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.
+    // read: [-W; Qt] over AW, [U; Pt V] over [K; Q], w * silu(z) over [Tb; Pt].
+    // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.  Each
+    // warpgroup's part leaves by bulk copy as soon as that warpgroup has
+    // written it (a named barrier per warpgroup), overlapping the rest.
+    const bool wg_lead = tl == 0;
     float x[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -425,11 +427,20 @@ __global__ void __launch_bounds__(NTA, 2)
 #pragma unroll
       for (int q = 0; q < 4; ++q) st_half8(smem + A_AW + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
     }
+    fence_proxy_async();
+    bar_named(1 + wg, 128);
+    if (wg_lead) bulk_store(rec + R_WQ + wg * 16384, sb + A_AW + wg * 16384, 16384);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       tmem_ld32(lane_base + A_TM_D4 + wg * 64 + hh * 32, x);
 #pragma unroll
       for (int q = 0; q < 4; ++q) st_half8(smem + A_KQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+    }
+    fence_proxy_async();
+    bar_named(1 + wg, 128);
+    if (wg_lead) {
+      bulk_store(rec + R_UO + wg * 16384, sb + A_KQ + wg * 16384, 16384);
+      bulk_commit();
     }
     // w * silu(z) in the chain's tile layout (value block ch / 8, row r, swizzled chunk)
     if (gated) {
@@ -446,16 +457,14 @@ __global__ void __launch_bounds__(NTA, 2)
         }
         *reinterpret_cast<uint4*>(smem + A_TBP + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
       }
+      fence_proxy_async();
+      __syncthreads();
+      if (tid == 0) {
+        bulk_store(rec + R_ZW, sb + A_TBP, 16384);
+        bulk_commit();
+      }
     }
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_store(rec + R_WQ, sb + A_AW, 32768);
-      bulk_store(rec + R_UO, sb + A_KQ, 32768);
-      if (gated) bulk_store(rec + R_ZW, sb + A_TBP, 16384);
-      bulk_commit();
-      bulk_wait_read();  // shared memory stays valid until the copies have read it
-    }
+    if (wg_lead) bulk_wait_read();  // shared memory stays valid until the copies have read it
   } else if (tid == 0) {
     atomicExch(&g_split_error, 1);
     mbar_wait(bar_load, 0, 100000000ull);
