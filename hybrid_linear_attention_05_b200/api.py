@@ -104,6 +104,31 @@ def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[Pre
     return PrefillOut(bufs.out, bufs.final_state, bufs.conv_state_out)
 
 
+def state_map(dp: DevicePrefill, bufs: Optional[PrefillBuffers] = None, segments: int = 0,
+              conv_state_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """(M, R) of every sequence of dp as [N, Hv, 2, d, d] fp32: a start state S
+    gives the final state S @ M + R (the initial state of dp is not used)."""
+    bufs = bufs or PrefillBuffers(dp)
+    maps = torch.empty((dp.N, dp.Hv, 2, dp.d, dp.d), dtype=torch.float32, device=dp.mixed_qkv.device)
+    gdn.gdn_prefill_state_map(
+        bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b, A_log=dp.A_log,
+        dt_bias=dp.dt_bias, cu_seqlens=dp.cu_seqlens, N=dp.N, T_tot=dp.T, chunk=dp.chunk,
+        dtype=bufs.dtype_code, map_out=maps, workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
+        conv_state_in=dp.conv_state_in, conv_state_out=conv_state_out, segments=segments)
+    return maps
+
+
+def state_fold(maps: torch.Tensor, S_first: Optional[torch.Tensor], Hk: int, Hv: int, d: int,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Fold of maps [count, N, Hv, 2, d, d] from S_first [N, Hv, d, d] (None: zeros)."""
+    count, N = int(maps.shape[0]), int(maps.shape[1])
+    if out is None:
+        out = torch.empty((N, Hv, d, d), dtype=torch.float32, device=maps.device)
+    gdn.gdn_state_fold(gdn.make_dims(Hk, Hv, d), N=N, count=count, maps=maps.contiguous(),
+                       S_out=out, S_first=S_first)
+    return out
+
+
 @dataclass
 class DeviceDecode:
     Hk: int

@@ -563,8 +563,11 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   const int h = XFER ? (int)blockIdx.x >> 1 : (int)blockIdx.x / CL;
   const int vs = XFER ? 0 : (int)blockIdx.x % CL;
   const int role = XFER ? (int)blockIdx.x & 1 : 1;  // 0: the map M (from S = I, U = 0)
-  const int n = XFER ? (int)blockIdx.y / (P - 1) : (int)blockIdx.y / P;
-  const int sg = XFER ? (int)blockIdx.y % (P - 1) : (int)blockIdx.y % P;
+  // transfer chains: the maps of segments 0 .. P-2, or of all P in state-map mode
+  const bool map_all = XFER && p.map_out != nullptr;
+  const int NM = XFER ? (map_all ? P : P - 1) : P;
+  const int n = (int)blockIdx.y / NM;
+  const int sg = (int)blockIdx.y % NM;
   const int hk = h / (p.Hv / p.Hk);
   const int bos0 = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
   const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos0, p.T);
@@ -580,26 +583,29 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   // (the R chain of segment 0 starts from S0 itself, so it leaves the state
   // at the start of segment 1 and segment 0 needs no map M)
   auto start_state = [&]() -> const float* {
-    if (XFER) return sg == 0 && p.S0 ? p.S0 + nh * hd + slice : nullptr;
+    if (XFER) return sg == 0 && p.S0 && !map_all ? p.S0 + nh * hd + slice : nullptr;
     if (P == 1) return p.S0 ? p.S0 + nh * hd + slice : nullptr;
     return p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd + slice;
   };
   auto final_state = [&]() -> float* {
-    if (XFER) return p.seg_mr + ((((size_t)n * (P - 1) + sg) * p.Hv + h) * 2 + role) * hd;
+    if (XFER) return p.seg_mr + ((((size_t)n * NM + sg) * p.Hv + h) * 2 + role) * hd;
     return sg == P - 1 && p.S_out ? p.S_out + nh * hd + slice : nullptr;
   };
   const bool norm_out = !XFER && p.out != nullptr;
   const bool want_u = !XFER || role == 1;  // the chain adds U to its new values
 
-  if (XFER && sg == 0 && role == 0) return;  // segment 0's map M is not needed
+  if (XFER && sg == 0 && role == 0 && !map_all) return;  // segment 0's map M is not needed
   if (nchunks == 0) {
     // empty segment; the last one is empty only for an empty sequence, whose
-    // state passes through (every CTA of the cluster returns here)
+    // state passes through (every CTA of the cluster returns here).  In
+    // state-map mode an empty segment's map is the identity: M = I, R = 0.
     pdl_wait();
     const float* Sin = start_state();
     float* Sfin = final_state();
     if (!XFER && Sfin)
       for (int idx = tid; idx < VS * D; idx += NTB) Sfin[idx] = Sin ? Sin[idx] : 0.f;
+    if (map_all)
+      for (int idx = tid; idx < D * D; idx += NCW) Sfin[idx] = role == 0 && idx / D == idx % D ? 1.f : 0.f;
     return;
   }
   const int slot0 = slot_start(p.cu_seqlens, n, p.T) + cb;
@@ -1154,6 +1160,142 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
 
 size_t record_slots(int N, int T) { return (size_t)(T / C) + (size_t)N + 1; }
 
+// ========================================================== affine fold
+// X <- X M_s (+ R_s on rows >= r_add) for s = 0 .. nmaps-1, in fp32 on the
+// CUDA cores, SR rows of one (sequence, head) per CTA (the products split as
+// in seg_scan_kernel: four contraction slices, 4 x 4 output tiles, slice 0
+// owning the rows).  M_s arrives by bulk copies into a double buffer one map
+// ahead.  Used to compose the segment maps of the state-map mode and to fold
+// the maps of consecutive parts of a sequence into a start state.
+constexpr int FOLD_KS = 4;
+constexpr int FOLD_POS = SR * 8;
+constexpr int FOLD_THREADS = FOLD_POS * FOLD_KS;
+constexpr uint32_t FOLD_SMEM = (2 * D * D + D * SR + (FOLD_KS - 1) * 16 * FOLD_POS) * 4 + 16 + 128;
+__global__ void __launch_bounds__(FOLD_THREADS) state_fold_kernel(FoldParams p) {
+  extern __shared__ uint8_t fold_raw[];
+  float* Mb = reinterpret_cast<float*>(fold_raw + ((128u - (smem_u32(fold_raw) & 127u)) & 127u));
+  float* sT = Mb + 2 * D * D;  // [D][SR]: this CTA's rows, transposed
+  float* red = sT + D * SR;    // [FOLD_KS - 1][16][FOLD_POS]: partial tiles of slices 1..
+  const uint32_t mbar = smem_u32(red + (FOLD_KS - 1) * 16 * FOLD_POS);
+  pdl_launch();
+  const int per = p.rows / SR;
+  const int h = (int)blockIdx.x / per, r0 = ((int)blockIdx.x % per) * SR;
+  const int n = (int)blockIdx.y;
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int ks = w >> 2, pos = tid & (FOLD_POS - 1);
+  const bool owner = ks == 0;
+  const int rr = (l >> 3) * 4, cc = ((w & 3) * 8 + (l & 7)) * 4;
+  const size_t dd = (size_t)D * D;
+  const bool add_r = r0 >= p.r_add;  // a CTA's rows lie on one side of r_add (a multiple of SR)
+  auto map_of = [&](int s) { return p.maps + (size_t)s * p.map_s + (size_t)n * p.map_n + (size_t)h * 2 * dd; };
+  auto prefetch = [&](int s, int buf) {  // thread 0: M_s into buffer buf
+    const float* M = map_of(s);
+    const uint32_t dst = smem_u32(Mb + buf * D * D), bar = mbar + 8 * buf;
+    mbar_arrive_expect_tx(bar, D * D * 4);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) bulk_load(dst + q * (D * D), M + q * (D * D / 4), D * D, bar);
+  };
+  if (tid == 0) {
+    mbar_init(mbar, 1);
+    mbar_init(mbar + 8, 1);
+    fence_mbar_init();
+  }
+  pdl_wait();  // the maps may come from the kernel before
+  if (tid < p.nmaps) {  // every map (and R slice) this CTA reads, into L2
+    bulk_prefetch_l2(map_of(tid), D * D * 4);
+    if (add_r) bulk_prefetch_l2(map_of(tid) + dd + (size_t)(r0 - p.r_add) * D, SR * D * 4);
+  }
+  __syncthreads();
+  if (tid == 0 && p.nmaps > 0) prefetch(0, 0);
+  float2 acc[4][2];
+  if (owner) {
+    const float* X0 = p.x0 ? p.x0 + (size_t)n * p.x0_n + (size_t)h * p.x0_h : nullptr;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 v = X0 ? *reinterpret_cast<const float4*>(X0 + (size_t)(r0 + rr + r) * D + cc)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[r][0] = make_float2(v.x, v.y);
+      acc[r][1] = make_float2(v.z, v.w);
+    }
+  }
+  bool ok = true;
+  for (int s = 0; s < p.nmaps; ++s) {
+    float4 rv[4];
+    if (owner) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int hc = c >> 1;
+        *reinterpret_cast<float4*>(sT + (cc + c) * SR + rr) =
+            (c & 1) ? make_float4(acc[0][hc].y, acc[1][hc].y, acc[2][hc].y, acc[3][hc].y)
+                    : make_float4(acc[0][hc].x, acc[1][hc].x, acc[2][hc].x, acc[3][hc].x);
+      }
+      const float* R = map_of(s) + dd + (size_t)(r0 - p.r_add) * D;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        rv[r] = add_r ? __ldg(reinterpret_cast<const float4*>(R + (size_t)(rr + r) * D + cc))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
+    const int buf = s & 1;
+    const uint32_t par = (uint32_t)(s >> 1) & 1u;
+    if (__syncthreads_or(!mbar_wait(mbar + 8 * buf, par))) {
+      if (tid == 0) {  // the copy never landed: record it, let it finish, stop
+        atomicExch(&g_split_error, 1);
+        mbar_wait(mbar + 8 * buf, par, 100000000ull);
+      }
+      ok = false;
+      break;
+    }
+    if (tid == 0 && s + 1 < p.nmaps) prefetch(s + 1, buf ^ 1);
+    const float* M = Mb + buf * D * D;
+#pragma unroll 4
+    for (int i = ks * (D / FOLD_KS); i < (ks + 1) * (D / FOLD_KS); ++i) {
+      const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
+      const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+      const float2 m01 = make_float2(m4.x, m4.y), m23 = make_float2(m4.z, m4.w);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float2 s2 = make_float2(sv[r], sv[r]);
+        acc[r][0] = __ffma2_rn(s2, m01, acc[r][0]);
+        acc[r][1] = __ffma2_rn(s2, m23, acc[r][1]);
+      }
+    }
+    if (!owner) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          red[(((ks - 1) * 16) + r * 4 + c) * FOLD_POS + pos] = (c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x;
+    }
+    __syncthreads();  // partial tiles written; sT and this buffer are free again
+    if (owner) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float rvr[4] = {rv[r].x, rv[r].y, rv[r].z, rv[r].w};
+        float v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          v[c] = ((c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x) + rvr[c];
+#pragma unroll
+          for (int k2 = 1; k2 < FOLD_KS; ++k2) v[c] += red[(((k2 - 1) * 16) + r * 4 + c) * FOLD_POS + pos];
+        }
+        acc[r][0] = make_float2(v[0], v[1]);
+        acc[r][1] = make_float2(v[2], v[3]);
+      }
+    }
+  }
+  if (owner && ok) {
+    float* dst = p.out + ((size_t)n * p.Hv + h) * p.rows * D;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      *reinterpret_cast<float4*>(dst + (size_t)(r0 + rr + r) * D + cc) =
+          make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+  }
+}
+
+
 }  // namespace
 
 size_t chunk_tc_split_record_bytes(int N, int T, int Hv) {
@@ -1191,7 +1333,7 @@ cudaError_t launch_chain(const CUtensorMap& mk, const ChunkParams& p, cudaStream
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = XFER ? dim3((unsigned)(2 * p.Hv), (unsigned)(p.N * (p.nseg - 1)), 1)
+  cfg.gridDim = XFER ? dim3((unsigned)(2 * p.Hv), (unsigned)(p.N * (p.map_out ? p.nseg : p.nseg - 1)), 1)
                      : dim3((unsigned)(G::CL * p.Hv), (unsigned)(p.N * p.nseg), 1);
   cfg.blockDim = dim3(XFER ? NCW : NTB, 1, 1);
   cfg.dynamicSmemBytes = G::SMEM;
@@ -1244,6 +1386,27 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   const int P = p.nseg;
+  if (p.map_out) {
+    // state-map mode: the maps of all P segments, then their composition
+    if (!p.seg_mr || P > kSegMax - 1 || (P == 1 && p.seg_mr != p.map_out)) return cudaErrorInvalidValue;
+    cudaError_t e = launch_chain<D, true>(mk, p, st);
+    if (e != cudaSuccess || P == 1) return e;
+    const size_t dd = (size_t)D * D;
+    FoldParams f{};
+    f.x0 = p.seg_mr;  // segment 0's [M; R]
+    f.x0_n = (size_t)P * p.Hv * 2 * dd;
+    f.x0_h = 2 * dd;
+    f.maps = p.seg_mr + (size_t)p.Hv * 2 * dd;  // segments 1 .. P-1
+    f.map_s = (size_t)p.Hv * 2 * dd;
+    f.map_n = (size_t)P * p.Hv * 2 * dd;
+    f.nmaps = P - 1;
+    f.rows = 2 * D;
+    f.r_add = D;
+    f.out = p.map_out;
+    f.N = p.N;
+    f.Hv = p.Hv;
+    return launch_state_fold(f, st);
+  }
   if (P > 1) {
     if (!p.seg_mr || !p.seg_start || P > kSegMax) return cudaErrorInvalidValue;
     cudaError_t e = launch_chain<D, true>(mk, p, st);
@@ -1277,6 +1440,36 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
 // plus as many for the output chains, about two per scan step (P - 2) and two
 // for the extra launches -- among those whose output chains fit the SMs in
 // one wave.  One serial chain takes `chunks` steps.
+cudaError_t launch_state_fold(const FoldParams& p, cudaStream_t st) {
+  if (p.N == 0 || p.Hv == 0) return cudaSuccess;
+  if (p.rows != D && p.rows != 2 * D) return cudaErrorInvalidValue;
+  if (p.r_add != 0 && p.r_add != D) return cudaErrorInvalidValue;
+  if (p.nmaps < 0 || (p.nmaps > 0 && !p.maps) || !p.out) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(state_fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FOLD_SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(p.Hv * (p.rows / SR)), (unsigned)p.N, 1);
+  cfg.blockDim = dim3(FOLD_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = FOLD_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, state_fold_kernel, p);
+}
+
+// State-map mode: as many segments as fill the SMs with the transfer chains
+// (both roles of every segment) in one wave.
+int chunk_tc_split_map_segments(int N, int Hv) {
+  const long chains = (long)N * Hv;
+  if (N <= 0 || chains > kSegMaxChains) return 1;
+  const long P = sm_count() / (2 * chains);
+  return (int)(P < 1 ? 1 : P > kSegMax - 1 ? kSegMax - 1 : P);
+}
+
 int chunk_tc_split_auto_segments(int N, int T, int Hv) {
   const long chains = (long)N * Hv;
   if (N <= 0 || chains > kSegMaxChains) return 1;

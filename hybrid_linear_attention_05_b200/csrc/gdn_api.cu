@@ -180,6 +180,88 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   return GDN_OK;
 }
 
+gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* a, float* map, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (!a || !map) return GDN_ERR_NULL;
+  if (a->N < 0 || a->T_tot < 0) return GDN_ERR_DIMS;
+  if (!dtype_ok(a->dtype)) return GDN_ERR_DIMS;
+  if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (a->segments < 0 || a->segments > kSegMax - 1) return GDN_ERR_UNSUPPORTED;
+  if (a->segments > 1 && (long)a->N * dims->Hv > kSegMaxChains) return GDN_ERR_UNSUPPORTED;
+  if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
+  const int d = dims->dk;
+  if (!chunk_tc_supported(d, a->chunk, mid_dtype(a->dtype)) || dims->dv != d) return GDN_ERR_UNSUPPORTED;
+  const int Cc = 2 * dims->Hk * d + dims->Hv * d;
+  const size_t full = carve(dims, a->T_tot, a->dtype, nullptr, a->N).bytes;
+  if (!a->workspace || a->workspace_bytes < full) return GDN_ERR_WORKSPACE;
+  if (!a->cu_seqlens || !a->conv_w || !a->A_log || !a->dt_bias) return GDN_ERR_NULL;
+  if (a->T_tot > 0 && (!a->mixed_qkv || !a->a || !a->b)) return GDN_ERR_NULL;
+  const void* ptrs[] = {a->mixed_qkv, a->conv_w, a->a, a->b, a->A_log, a->dt_bias, a->cu_seqlens,
+                        a->conv_state_in, a->conv_state_out, a->workspace, map};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const size_t cs_bytes = (size_t)a->N * Cc * 3 * esize(a->dtype);
+  if (overlap(a->conv_state_in, cs_bytes, a->conv_state_out, cs_bytes)) return GDN_ERR_ALIAS;
+  const size_t map_bytes = (size_t)a->N * dims->Hv * 2 * d * d * sizeof(float);
+  if (overlap(map, map_bytes, a->workspace, a->workspace_bytes)) return GDN_ERR_ALIAS;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Workspace ws = carve(dims, a->T_tot, a->dtype, a->workspace, a->N);
+  ConvPrepParams cp{};
+  cp.x = a->mixed_qkv; cp.conv_w = a->conv_w; cp.a = a->a; cp.b = a->b;
+  cp.A_log = a->A_log; cp.dt_bias = a->dt_bias; cp.cu_seqlens = a->cu_seqlens;
+  cp.conv_state_in = a->conv_state_in; cp.conv_state_out = a->conv_state_out;
+  cp.q = ws.q; cp.k = ws.k; cp.v = ws.v; cp.g = ws.g; cp.beta = ws.beta;
+  cp.T = a->T_tot; cp.N = a->N; cp.Hk = dims->Hk; cp.Hv = dims->Hv; cp.Cc = Cc;
+  cp.scale = dims->scale; cp.eps_l2 = dims->eps_l2;
+  s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
+  if (s != GDN_OK) return s;
+
+  ChunkParams ch{};
+  ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
+  ch.cu_seqlens = a->cu_seqlens; ch.S0 = nullptr; ch.S_out = nullptr;
+  ch.z = nullptr; ch.norm_w = nullptr; ch.out = nullptr; ch.o_raw = nullptr;
+  ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
+  ch.eps_norm = dims->eps_norm;
+  ch.rec = ws.rec;
+  ch.map_out = map;
+  ch.nseg = ws.seg_mr ? (a->segments > 0 ? a->segments : chunk_tc_split_map_segments(a->N, dims->Hv)) : 1;
+  ch.seg_mr = ch.nseg > 1 ? ws.seg_mr : map;
+  ch.seg_start = nullptr;
+  return from_cuda(launch_chunk_tc_split(ch, st));
+}
+
+gdn_status gdn_state_fold(const gdn_dims* dims, int N, int count, const float* maps, const float* S_first,
+                          float* S_out, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (N < 0 || count < 0) return GDN_ERR_DIMS;
+  if (dims->dk != 128 || dims->dv != 128) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!S_out || (count > 0 && !maps)) return GDN_ERR_NULL;
+  if (!aligned16(maps) || !aligned16(S_first) || !aligned16(S_out)) return GDN_ERR_ALIGN;
+  const size_t dd = (size_t)dims->dk * dims->dk;
+  const size_t st_bytes = (size_t)N * dims->Hv * dd * sizeof(float);
+  const size_t map_bytes = (size_t)count * N * dims->Hv * 2 * dd * sizeof(float);
+  if (overlap(maps, map_bytes, S_out, st_bytes)) return GDN_ERR_ALIAS;
+  if (S_first != S_out && overlap(S_first, st_bytes, S_out, st_bytes)) return GDN_ERR_ALIAS;
+  FoldParams f{};
+  f.x0 = S_first;
+  f.x0_n = (size_t)dims->Hv * dd;
+  f.x0_h = dd;
+  f.maps = maps;
+  f.map_s = (size_t)N * dims->Hv * 2 * dd;
+  f.map_n = (size_t)dims->Hv * 2 * dd;
+  f.nmaps = count;
+  f.rows = dims->dk;
+  f.r_add = 0;
+  f.out = S_out;
+  f.N = N;
+  f.Hv = dims->Hv;
+  return from_cuda(launch_state_fold(f, static_cast<cudaStream_t>(stream)));
+}
+
 gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* a, void* stream) {
   gdn_status s = check_dims(dims);
   if (s != GDN_OK) return s;

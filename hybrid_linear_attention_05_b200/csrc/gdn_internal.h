@@ -59,6 +59,11 @@ struct ChunkParams {
   int nseg;
   float* seg_mr;
   float* seg_start;
+  // state-map mode (map_out != null): no outputs; every one of the nseg
+  // segments gets its map, in seg_mr as [N][nseg][Hv][2][d][d] (role 1 from a
+  // zero state), and the maps of each (sequence, head), composed in segment
+  // order, go to map_out [N][Hv][2][d][d].  With nseg == 1, seg_mr == map_out.
+  float* map_out;
 };
 
 // chunk_simt.cu: fp32 CUDA-core chunked core.  Supported (d, chunk) pairs:
@@ -87,6 +92,29 @@ size_t chunk_tc_split_seg_bytes(int N, int Hv);
 int chunk_tc_split_auto_segments(int N, int T, int Hv);
 cudaError_t launch_chunk_tc_split(const ChunkParams& p, cudaStream_t st);
 int split_error_word(int clear);  // host: read (and clear) that path's device error word
+// Segments of the state-map mode for N sequences of Hv heads (1 when the
+// segment buffers do not exist for these sizes).
+int chunk_tc_split_map_segments(int N, int Hv);
+
+// Affine fold, d = 128: for every (sequence n, head h), the rows X (rows x d,
+// fp32) start from x0 (zeros when null) and go through the maps s = 0 ..
+// nmaps-1 in order, X <- X M_s, and rows r >= r_add also take row r - r_add
+// of R_s.  With rows = d and r_add = 0, X is a state and the fold is the
+// state after consecutive parts; with rows = 2d and r_add = d, X is a stacked
+// map [M; R] and the fold composes maps.  out may be x0 (each row is read
+// before it is written, by the same CTA).
+struct FoldParams {
+  const float* x0;        // rows of (n, h) at x0 + n * x0_n + h * x0_h, or null
+  size_t x0_n, x0_h;
+  const float* maps;      // map s of (n, h) at maps + s * map_s + n * map_n + h * 2 d d: M then R
+  size_t map_s, map_n;
+  int nmaps;
+  int rows;               // d or 2 d
+  int r_add;              // 0 or d
+  float* out;             // [N][Hv][rows][d]
+  int N, Hv;
+};
+cudaError_t launch_state_fold(const FoldParams& p, cudaStream_t st);
 
 // decode.cu
 struct DecodeParams {

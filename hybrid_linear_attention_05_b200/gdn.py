@@ -34,7 +34,8 @@ GDN_IMPL_TC = 2
 GDN_IMPL_TC_SPLIT = 3
 
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
-            "gdn_prefill_auto_segments", "gdn_prefill_noalloc", "gdn_decode", "gdn_chunk_core",
+            "gdn_prefill_auto_segments", "gdn_prefill_noalloc", "gdn_prefill_state_map",
+            "gdn_state_fold", "gdn_decode", "gdn_chunk_core",
             "gdn_device_error", "gdn_status_string", "gdn_version"]
 
 # Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
@@ -99,6 +100,11 @@ def lib():
         L.gdn_prefill_noalloc.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
                                           _vp]
         L.gdn_prefill_noalloc.restype = ctypes.c_int
+        L.gdn_prefill_state_map.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
+                                            _vp, _vp]
+        L.gdn_prefill_state_map.restype = ctypes.c_int
+        L.gdn_state_fold.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp]
+        L.gdn_state_fold.restype = ctypes.c_int
         L.gdn_decode.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_decode_args), _vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_chunk_core.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_core_args), _vp]
@@ -203,6 +209,28 @@ def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bi
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill_noalloc(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_prefill_noalloc", raise_on_error)
+
+
+def gdn_prefill_state_map(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, cu_seqlens, N,
+                          T_tot, chunk, dtype, map_out, workspace, workspace_bytes, conv_state_in=None,
+                          conv_state_out=None, segments=0, stream=None, raise_on_error=True) -> int:
+    """(M, R) of every sequence: final state = initial state @ M + R (gdn.h)."""
+    args = gdn_prefill_args(
+        ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), None, None,
+        ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(GDN_IMPL_TC_SPLIT), None,
+        None, ptr(conv_state_in), ptr(conv_state_out), None, ptr(workspace), int(workspace_bytes),
+        None, None, int(segments))
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_prefill_state_map(ctypes.byref(dims), ctypes.byref(args), ptr(map_out), s),
+                  "gdn_prefill_state_map", raise_on_error)
+
+
+def gdn_state_fold(dims: gdn_dims, *, N, count, maps, S_out, S_first=None, stream=None,
+                   raise_on_error=True) -> int:
+    """S_out = fold of `count` consecutive maps [count, N, Hv, 2, d, d] from S_first."""
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_state_fold(ctypes.byref(dims), int(N), int(count), ptr(maps), ptr(S_first),
+                                       ptr(S_out), s), "gdn_state_fold", raise_on_error)
 
 
 def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w, state,

@@ -179,6 +179,50 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* args, void*
  * states.  0 when the sizes are invalid. */
 int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot);
 
+/* ------------------------------------------------ context-parallel prefill
+ * One long sequence cut into consecutive parts, e.g. one part per GPU (the
+ * family is built for long contexts: "Qwen/Qwen3.5-9B", config table:
+ * max_position_embeddings 262144; "Qwen3.5-397B-A17B", specification table:
+ * context length 256K tokens).  Step 4 is linear in the state, so over a
+ * part of the sequence the state after it is an affine function of the state
+ * before it:
+ *     S_after = S_before M + R,
+ *     M = prod over the part's tokens, in order, of alpha_t (I - beta_t k_t k_t^T)
+ *         (dk x dk),
+ *     R = the state after the part when it starts from zero (dv x dk).
+ * The parts' (M, R) are independent of one another; the start state of part
+ * j is the fold S_j = (...((S_0 M_0 + R_0) M_1 + R_1) ...) M_{j-1} + R_{j-1}.
+ * A context-parallel prefill therefore computes every part's map at once,
+ * gathers the maps (an exchange of 2 * Hv * d * d * 4 bytes per part and
+ * sequence), folds them, and runs gdn_prefill on each part from its start
+ * state, with the last three raw inputs before the part as conv_state_in.
+ *
+ * gdn_prefill_state_map: (M, R) of every sequence of the call.
+ *   map   device [N, Hv, 2, dv, dk] fp32, written: map[n][h][0] = M (dk x dk,
+ *         dv = dk), map[n][h][1] = R.  Must not overlap the workspace.
+ *   args  as for gdn_prefill; mixed_qkv, conv_w, a, b, A_log, dt_bias,
+ *         cu_seqlens and conv_state_in are read, conv_state_out is written
+ *         when given; initial_state, final_state, z, norm_w and out are not
+ *         used.  segments: 0 = chosen from the sizes, 1 = one serial chain,
+ *         2..7 = that many segments per sequence, composed in fp32 (more than
+ *         1 only when N*Hv <= 64).
+ *   Supported: bf16, dk = dv = 128, chunk 64 (the tensor-core shapes), with
+ *   gdn_prefill_workspace_size_n bytes of workspace; GDN_ERR_UNSUPPORTED /
+ *   GDN_ERR_WORKSPACE otherwise.  An empty sequence gives M = I, R = 0.
+ *
+ * gdn_state_fold: S_out = the fold of `count` consecutive maps from S_first.
+ *   maps    device [count, N, Hv, 2, dv, dk] fp32 (e.g. the maps of parts
+ *           0 .. count-1 gathered from their ranks, in part order)
+ *   S_first device [N, Hv, dv, dk] fp32, or NULL for zeros
+ *   S_out   device [N, Hv, dv, dk] fp32; may be S_first (in place), must not
+ *           overlap maps.  count = 0 copies S_first (or zeros).
+ *   Supported: dk = dv = 128.
+ */
+gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* args, float* map,
+                                 void* stream);
+gdn_status gdn_state_fold(const gdn_dims* dims, int N, int count, const float* maps,
+                          const float* S_first, float* S_out, void* stream);
+
 /* ------------------------------------------------ prefill without workspace
  * No counterpart on the pages: this is an addition of this library for
  * callers that cannot hand gdn_prefill a workspace -- e.g. an operator plugin

@@ -118,6 +118,34 @@ def prefill(Hk, Hv, dk, dv, cu_seqlens, mixed_qkv, conv_w, a, b, A_log, dt_bias,
     return res
 
 
+def state_map(Hk, Hv, dk, dv, mixed_qkv, conv_w, a, b, A_log, dt_bias, conv_state_in=None, scale=None,
+              eps_l2=1e-6, nthreads=None):
+    """The affine state map of one sequence: final state = S0 @ M + R.
+
+    The delta rule S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+    ("Qwen (text & vision-language)", Architecture notes) is linear in S, so
+      M = prod over t, in token order, of alpha_t (I - beta_t k_t k_t^T)  [Hv, dk, dk]
+      R = the final state from S0 = 0                                     [Hv, dv, dk]
+    k, alpha, beta are the prepared values of ``prefill`` (conv from
+    conv_state_in, L2 norm, gates); M is accumulated token by token here.
+    """
+    Cc = 2 * Hk * dk + Hv * dv
+    x = _d(mixed_qkv).reshape(-1, Cc)
+    T = x.shape[0]
+    res = prefill(Hk, Hv, dk, dv, [0, T], x, conv_w, a, b, A_log, dt_bias,
+                  np.zeros((T, Hv * dv)), np.ones(dv), initial_state=None,
+                  conv_state_in=conv_state_in, scale=scale, eps_l2=eps_l2, nthreads=nthreads)
+    G = Hv // Hk
+    M = np.zeros((Hv, dk, dk))
+    for h in range(Hv):
+        Mh = np.eye(dk)
+        for t in range(T):
+            k = res.k[t, h // G]
+            Mh = np.exp(res.g[t, h]) * (Mh - res.beta[t, h] * np.outer(Mh @ k, k))
+        M[h] = Mh
+    return M, res.final_state[0].copy()
+
+
 def decode(Hk, Hv, dk, dv, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w, state,
            conv_state, scale=None, eps_l2=1e-6, eps_norm=1e-6, nthreads=None):
     """One recurrent step for B sequences.  Returns (out, new_state, new_conv_state)."""

@@ -163,3 +163,45 @@ def test_core_rejects_bad_args(L):
     assert gdn.gdn_chunk_core(dims, **{**kw, "o": None}) == gdn.GDN_ERR_NULL
     assert gdn.gdn_chunk_core(dims, **{**kw, "beta": FAKE + 4}) == gdn.GDN_ERR_ALIGN
     assert gdn.gdn_chunk_core(dims, **{**kw, "chunk": 8}) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def map_kwargs(**over):
+    kw = dict(mixed_qkv=FAKE, conv_w=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, cu_seqlens=FAKE,
+              N=1, T_tot=16, chunk=64, dtype=gdn.GDN_BF16, map_out=FAKE + (1 << 30),
+              workspace=FAKE, workspace_bytes=1 << 29, stream=0, raise_on_error=False)
+    kw.update(over)
+    return kw
+
+
+@pytest.mark.parametrize("dims,over,status", [
+    (gdn.make_dims(2, 4, 64), {}, gdn.GDN_ERR_UNSUPPORTED),          # the tensor-core width only
+    (gdn.make_dims(2, 4, 128), dict(chunk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128), dict(dtype=gdn.GDN_F32), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128), dict(map_out=None), gdn.GDN_ERR_NULL),
+    (gdn.make_dims(2, 4, 128), dict(map_out=FAKE + (1 << 30) + 8), gdn.GDN_ERR_ALIGN),
+    (gdn.make_dims(2, 4, 128), dict(map_out=FAKE + 4096), gdn.GDN_ERR_ALIAS),  # inside the workspace
+    (gdn.make_dims(2, 4, 128), dict(workspace_bytes=1 << 20), gdn.GDN_ERR_WORKSPACE),
+    (gdn.make_dims(2, 4, 128), dict(workspace=None), gdn.GDN_ERR_WORKSPACE),
+    (gdn.make_dims(2, 4, 128), dict(segments=8), gdn.GDN_ERR_UNSUPPORTED),   # at most 7 in map mode
+    (gdn.make_dims(2, 4, 128), dict(segments=2, N=17, T_tot=17), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128), dict(mixed_qkv=None), gdn.GDN_ERR_NULL),
+    (gdn.make_dims(2, 4, 128), dict(N=0, T_tot=0), gdn.GDN_OK),
+])
+def test_state_map_rejects_bad_args(L, dims, over, status):
+    assert gdn.gdn_prefill_state_map(dims, **map_kwargs(**over)) == status
+
+
+@pytest.mark.parametrize("dims,over,status", [
+    (gdn.make_dims(2, 4, 64), {}, gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.make_dims(2, 4, 128), dict(S_out=None), gdn.GDN_ERR_NULL),
+    (gdn.make_dims(2, 4, 128), dict(maps=None), gdn.GDN_ERR_NULL),
+    (gdn.make_dims(2, 4, 128), dict(count=0, maps=None, N=0), gdn.GDN_OK),
+    (gdn.make_dims(2, 4, 128), dict(S_out=FAKE + 8), gdn.GDN_ERR_ALIGN),
+    (gdn.make_dims(2, 4, 128), dict(S_out=FAKE + 4096), gdn.GDN_ERR_ALIAS),   # overlaps the maps
+    (gdn.make_dims(2, 4, 128), dict(S_first=FAKE + (1 << 28) + 4096), gdn.GDN_ERR_ALIAS),
+    (gdn.make_dims(2, 4, 128), dict(count=-1), gdn.GDN_ERR_DIMS),
+])
+def test_state_fold_rejects_bad_args(L, dims, over, status):
+    kw = dict(N=1, count=3, maps=FAKE, S_out=FAKE + (1 << 28), S_first=None, stream=0, raise_on_error=False)
+    kw.update(over)
+    assert gdn.gdn_state_fold(dims, **kw) == status

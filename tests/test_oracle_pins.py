@@ -390,3 +390,86 @@ def test_397b_state_size():
     per_key_head = kv_tok * ctx + gdn_layers * Hk * d * d * 2 + conv
     assert "%.2fGiB" % (per_value_head / 2 ** 30) == gold["kv_cache_plus_state_256k_bf16"]
     assert "%.2fGiB" % (per_key_head / 2 ** 30) != gold["kv_cache_plus_state_256k_bf16"]
+
+
+# ----------------------------------------- affine state maps (context parallel)
+# The delta rule is linear in the state, so over a stretch of tokens the state
+# after it is S0 @ M + R ("Qwen (text & vision-language)", Architecture notes:
+# S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T).
+
+
+def _map(oracle_mod, Hk, Hv, d, inp, sl=slice(None), hist=None):
+    return oracle_mod.state_map(Hk, Hv, d, d, inp["mixed_qkv"][sl], inp["conv_w"], inp["a"][sl],
+                                inp["b"][sl], inp["A_log"], inp["dt_bias"], conv_state_in=hist)
+
+
+def test_state_map_affine_in_start_state(oracle_mod):
+    """The final state from any S0 equals S0 @ M + R: the C++ recurrence of
+    ``prefill`` against the map that ``state_map`` accumulates token by token
+    in numpy.  Slow decay, so that S0 @ M is not negligible."""
+    rng = np.random.default_rng(21)
+    Hk, Hv, d = 2, 4, 8
+    inp = mixer_inputs(rng, [37], Hk, Hv, d)
+    inp["A_log"] = rng.uniform(-7.0, -5.0, Hv)
+    M, R = _map(oracle_mod, Hk, Hv, d, inp, hist=inp["conv_state_in"])
+    assert np.max(np.abs(M)) > 0.1
+    for _ in range(3):
+        S0 = rng.standard_normal((1, Hv, d, d))
+        r = oracle_mod.prefill(Hk, Hv, d, d, **dict(inp, initial_state=S0))
+        assert rel(r.final_state[0], S0[0] @ M + R) < 1e-12
+
+
+def test_state_map_one_token_closed_form(oracle_mod):
+    """One token: M = alpha (I - beta k k^T) and R = beta v k^T, from the
+    prepared k, v, g, beta of ``prefill``."""
+    rng = np.random.default_rng(23)
+    Hk, Hv, d = 1, 2, 6
+    inp = mixer_inputs(rng, [1], Hk, Hv, d)
+    r = oracle_mod.prefill(Hk, Hv, d, d, **dict(inp, initial_state=None))
+    M, R = _map(oracle_mod, Hk, Hv, d, inp, hist=inp["conv_state_in"])
+    for h in range(Hv):
+        k, v = r.k[0, h // (Hv // Hk)], r.v[0, h]
+        al, be = math.exp(r.g[0, h]), r.beta[0, h]
+        assert rel(M[h], al * (np.eye(d) - be * np.outer(k, k))) < 1e-13
+        assert rel(R[h], be * np.outer(v, k)) < 1e-13
+
+
+def test_state_map_empty_is_identity(oracle_mod):
+    rng = np.random.default_rng(24)
+    Hk, Hv, d = 1, 2, 4
+    inp = mixer_inputs(rng, [5], Hk, Hv, d)
+    M, R = _map(oracle_mod, Hk, Hv, d, inp, sl=slice(0, 0), hist=inp["conv_state_in"])
+    np.testing.assert_array_equal(M, np.broadcast_to(np.eye(d), (Hv, d, d)))
+    np.testing.assert_array_equal(R, 0.0)
+
+
+def test_parts_fold_to_the_whole_sequence(oracle_mod):
+    """A sequence cut into consecutive parts, some shorter than the conv
+    window and one empty.  Each part's conv history is the three raw inputs
+    before it, its start state the fold of the earlier parts' maps from S0;
+    run from there, the parts give the whole sequence's outputs, and the
+    fold of all maps its final state."""
+    rng = np.random.default_rng(22)
+    Hk, Hv, d = 2, 4, 8
+    lens = [2, 17, 0, 1, 25]
+    T = sum(lens)
+    inp = mixer_inputs(rng, [T], Hk, Hv, d)
+    inp["A_log"] = rng.uniform(-7.0, -5.0, Hv)
+    whole = oracle_mod.prefill(Hk, Hv, d, d, **inp)
+    raw = np.concatenate([inp["conv_state_in"][0].T, inp["mixed_qkv"]], axis=0)  # row j = token j - 3
+    S = inp["initial_state"][0]
+    outs, t0 = [], 0
+    for L in lens:
+        sl = slice(t0, t0 + L)
+        hist = raw[t0:t0 + 3].T[None]
+        part = dict(inp, cu_seqlens=[0, L], mixed_qkv=inp["mixed_qkv"][sl], a=inp["a"][sl],
+                    b=inp["b"][sl], z=inp["z"][sl], conv_state_in=hist, initial_state=S[None])
+        r = oracle_mod.prefill(Hk, Hv, d, d, **part)
+        outs.append(r.out)
+        M, R = _map(oracle_mod, Hk, Hv, d, inp, sl=sl, hist=hist)
+        S_next = S @ M + R
+        assert rel(S_next, r.final_state[0]) < 1e-12
+        S = S_next
+        t0 += L
+    assert rel(np.concatenate(outs), whole.out) < 1e-12
+    assert rel(S, whole.final_state[0]) < 1e-12
