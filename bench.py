@@ -403,6 +403,49 @@ def run_ours(args, rank, world, local_rank):
            "pipelined": "two buffer sets; copy-in, compute and copy-out streams"}
     del host, h_out, h_S, slots
 
+    # ---------------- context-parallel pieces: the kernels one rank runs for its
+    # part of a long sequence (the map of the part, the fold of the earlier
+    # parts' maps, the part's prefill), timed on this GPU with the L2 flushed
+    # before each call.  Only on a single-GPU run: the exchange between ranks
+    # (one all-gather of the maps) is not part of these numbers.
+    context_parallel = None
+    if world == 1 and inp.N == 1 and wp.d == 128 and wp.dtype == "bf16":
+        W_cp = 8
+        maps = api.state_map(dp, bufs)
+        gathered = maps.expand(W_cp - 1, *maps.shape).contiguous()
+        S_buf = torch.empty((1, wp.Hv, wp.d, wp.d), dtype=torch.float32, device=dev)
+
+        def timed(fn):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                tot += a.elapsed_time(b)
+            return tot / args.steps * 1e3  # us
+
+        map_us = timed(lambda: api.state_map(dp, bufs))
+        fold_us = timed(lambda: api.state_fold(gathered, None, wp.Hk, wp.Hv, wp.d, out=S_buf))
+        # the part's prefill on the workspace its map left (conv and key-side kernels skipped)
+        part_us = timed(lambda: api.prefill(dp, bufs=bufs, reuse_workspace=True))
+        rank_us = map_us + fold_us + part_us
+        context_parallel = {
+            "parts": W_cp, "tokens_per_part": inp.T,
+            "map_us": map_us, "fold_us": fold_us, "fold_maps": W_cp - 1,
+            "prefill_after_map_us": part_us, "rank_us": rank_us,
+            "rank_tokens_per_s": inp.T / (rank_us * 1e-6),
+            "exchange_bytes_per_part": int(maps.numel() * 4),
+            "note": "kernels of the last rank of a context-parallel prefill of one sequence of "
+                    "%d x %d tokens, on one GPU; the all-gather of the maps is not included" % (W_cp, inp.T),
+        }
+        del maps, gathered, S_buf
+
     # ---------------- decode half of the metric (fp32 state; then a bf16 state)
     wd = WORKLOADS[args.decode_workload]
     dinp = make_decode(wd)
@@ -487,6 +530,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "flushed before every timed step (256 MiB write)"},
         "roofline": roofline,
         "decode": decode,
+        "context_parallel": context_parallel,
         "e2e": e2e,
         # conv_prep + the core's launches per prefill step
         "gpu_launches": (1 + core_launches) * args.steps,

@@ -89,7 +89,9 @@ class PrefillBuffers:
 
 
 def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[PrefillBuffers] = None,
-            core_events=None, segments: int = 0) -> PrefillOut:
+            core_events=None, segments: int = 0, reuse_workspace: bool = False) -> PrefillOut:
+    """reuse_workspace: bufs.workspace holds a ``state_map`` of the same inputs
+    (the conv and key-side kernels are skipped, conv_state_out is not written)."""
     bufs = bufs or PrefillBuffers(dp)
     ev0, ev1 = (None, None) if core_events is None else (core_events[0].cuda_event,
                                                          core_events[1].cuda_event)
@@ -99,22 +101,25 @@ def prefill(dp: DevicePrefill, impl: int = gdn.GDN_IMPL_AUTO, bufs: Optional[Pre
         T_tot=dp.T, chunk=dp.chunk, dtype=bufs.dtype_code, out=bufs.out,
         workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
         initial_state=dp.initial_state, final_state=bufs.final_state,
-        conv_state_in=dp.conv_state_in, conv_state_out=bufs.conv_state_out, impl=impl,
-        core_event_begin=ev0, core_event_end=ev1, segments=segments)
+        conv_state_in=dp.conv_state_in, conv_state_out=None if reuse_workspace else bufs.conv_state_out,
+        impl=gdn.GDN_IMPL_TC_SPLIT if reuse_workspace else impl, core_event_begin=ev0, core_event_end=ev1,
+        segments=segments, reuse_workspace=int(reuse_workspace))
     return PrefillOut(bufs.out, bufs.final_state, bufs.conv_state_out)
 
 
 def state_map(dp: DevicePrefill, bufs: Optional[PrefillBuffers] = None, segments: int = 0,
               conv_state_out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """(M, R) of every sequence of dp as [N, Hv, 2, d, d] fp32: a start state S
-    gives the final state S @ M + R (the initial state of dp is not used)."""
+    gives the final state S @ M + R (the initial state of dp is not used).
+    bufs.workspace is left ready for ``prefill(dp, bufs=bufs, reuse_workspace=True)``."""
     bufs = bufs or PrefillBuffers(dp)
     maps = torch.empty((dp.N, dp.Hv, 2, dp.d, dp.d), dtype=torch.float32, device=dp.mixed_qkv.device)
     gdn.gdn_prefill_state_map(
         bufs.dims, mixed_qkv=dp.mixed_qkv, conv_w=dp.conv_w, a=dp.a, b=dp.b, A_log=dp.A_log,
         dt_bias=dp.dt_bias, cu_seqlens=dp.cu_seqlens, N=dp.N, T_tot=dp.T, chunk=dp.chunk,
         dtype=bufs.dtype_code, map_out=maps, workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
-        conv_state_in=dp.conv_state_in, conv_state_out=conv_state_out, segments=segments)
+        conv_state_in=dp.conv_state_in, conv_state_out=conv_state_out, z=dp.z, norm_w=dp.norm_w,
+        segments=segments)
     return maps
 
 

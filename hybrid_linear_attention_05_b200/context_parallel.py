@@ -45,19 +45,34 @@ class PartResult:
 
 
 class LibraryCompute:
-    """The three calls on the CUDA library (parts are ``api.DevicePrefill``)."""
+    """The three calls on the CUDA library (parts are ``api.DevicePrefill``).
 
-    def __init__(self, segments: int = 0):
+    A part's workspace is kept from its map to its prefill, which then skips
+    the conv and the key-side kernel (``reuse_workspace``)."""
+
+    def __init__(self, segments: int = 0, reuse: bool = True):
         self.segments = segments
+        self.reuse = reuse
+        self._bufs = {}
+
+    @staticmethod
+    def _key(part):
+        return (part.mixed_qkv.data_ptr(), part.T)
 
     def state_map(self, part: api.DevicePrefill) -> torch.Tensor:
-        return api.state_map(part, segments=self.segments)
+        bufs = api.PrefillBuffers(part)
+        self._bufs[self._key(part)] = bufs
+        return api.state_map(part, bufs, segments=self.segments)
 
     def fold(self, maps: torch.Tensor, S_first: Optional[torch.Tensor], part: api.DevicePrefill) -> torch.Tensor:
         return api.state_fold(maps, S_first, part.Hk, part.Hv, part.d)
 
     def prefill(self, part: api.DevicePrefill):
-        r = api.prefill(part)
+        bufs = self._bufs.pop(self._key(part), None)
+        if self.reuse and bufs is not None and part.T > 0:
+            r = api.prefill(part, bufs=bufs, reuse_workspace=True)
+        else:
+            r = api.prefill(part)
         return r.out.clone(), r.final_state.clone()
 
 

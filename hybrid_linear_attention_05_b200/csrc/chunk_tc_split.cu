@@ -62,6 +62,16 @@ __device__ int g_split_error = 0;  // nonzero: a bounded wait in a kernel of thi
 // Development aid (off by default): SM cycles spent by chain-kernel thread 0
 // in each phase of the chunk loop, summed over all CTAs.
 __device__ unsigned long long g_split_phase[32];
+// seg_scan_kernel, thread 0 of every CTA: cycles per phase, summed
+__device__ unsigned long long g_scan_phase[8];
+#define GDN_SCAN_MARK(k)                                                \
+  do {                                                                  \
+    if (tid == 0) {                                                     \
+      const long long t_ = clock64();                                   \
+      atomicAdd(&g_scan_phase[k], (unsigned long long)(t_ - t_prev));   \
+      t_prev = t_;                                                      \
+    }                                                                   \
+  } while (0)
 #define GDN_SPLIT_MARK(k)                                               \
   do {                                                                  \
     if (tid == NCW + 64) {                                              \
@@ -95,6 +105,9 @@ __device__ unsigned long long g_split_phase[32];
   } while (0)
 #define GDN_SPLIT_MARK(k) \
   do {                    \
+  } while (0)
+#define GDN_SCAN_MARK(k) \
+  do {                   \
   } while (0)
 #endif
 
@@ -183,7 +196,7 @@ __global__ void __launch_bounds__(NTA, 2)
   // overlaps the set-up and the wait for the conv kernel
   // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
   // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
-  const bool gated = p.out != nullptr;
+  const bool gated = p.z != nullptr;  // w * silu(z) into the record (the gated norm's factor)
   uint4 zv[4];
   if (gated) {
 #pragma unroll
@@ -1004,12 +1017,16 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) bulk_load(dst + q * (D * D), M + q * (D * D / 4), D * D, bar);
   };
+#ifdef GDN_PHASE_TIMING
+  long long t_prev = clock64();
+#endif
   if (tid == 0) {
     mbar_init(mbar, 1);
     mbar_init(mbar + 8, 1);
     fence_mbar_init();
   }
   pdl_wait();  // the maps come from the transfer chains
+  GDN_SCAN_MARK(0);
   if (tid < P - 1 && nonempty(tid)) {  // every map and R slice this CTA will read, into L2
     if (tid > 0) bulk_prefetch_l2(map_of(tid), D * D * 4);
     bulk_prefetch_l2(map_of(tid) + hd + (size_t)r0 * D, SR * D * 4);
@@ -1032,6 +1049,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       acc[r][1] = make_float2(v.z, v.w);
     }
   }
+  GDN_SCAN_MARK(1);
   for (int sg = 0;; ++sg) {
     if (owner) {
       float* dst = p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd;
@@ -1073,6 +1091,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
     const int buf = j & 1;
     const uint32_t par = (uint32_t)(j >> 1) & 1u;
+    GDN_SCAN_MARK(2);
     if (__syncthreads_or(!mbar_wait(mbar + 8 * buf, par))) {
       // sT is complete but this segment's M never landed: record it, let the copy finish, stop
       if (tid == 0) {
@@ -1081,6 +1100,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       }
       break;
     }
+    GDN_SCAN_MARK(3);
     sg_next = next_map(sg + 1);
     if (tid == 0 && sg_next < P - 1) prefetch(sg_next, buf ^ 1);
     const float* M = Mb + buf * D * D;
@@ -1097,6 +1117,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
         acc[r][1] = __ffma2_rn(s2, m23, acc[r][1]);
       }
     }
+    GDN_SCAN_MARK(4);
     if (!owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
@@ -1105,6 +1126,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
           red[((ks * 16) + r * 4 + c) * SCAN_POS + pos] = (c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x;
     }
     __syncthreads();  // partial tiles written; everyone is done with sT and this buffer
+    GDN_SCAN_MARK(5);
     if (owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
@@ -1121,6 +1143,10 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       }
     }
     ++j;
+    GDN_SCAN_MARK(6);
+#ifdef GDN_PHASE_TIMING
+    if (tid == 0) atomicAdd(&g_scan_phase[7], 1ull);
+#endif
     // the owners' reads of `red` end before its next write: two barriers
     // (the one above sT's completion and the one after the products) lie between
   }
@@ -1368,6 +1394,8 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
         !make_map(&mk, p.k, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
         !make_map(&mv, p.v, (uint64_t)p.T, (uint64_t)p.Hv * D, f16, sw))
       return cudaErrorInvalidValue;
+  }
+  if (p.T > 0 && !p.reuse_records) {
     cudaError_t e = cudaFuncSetAttribute(chunk_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)A_SMEM);
     if (e != cudaSuccess) return e;
@@ -1492,6 +1520,15 @@ int chunk_tc_split_auto_segments(int N, int T, int Hv) {
 }
 
 #ifdef GDN_PHASE_TIMING
+extern "C" int gdn_debug_phase_cycles_scan(unsigned long long* out, int clear) {
+  cudaDeviceSynchronize();
+  if (cudaMemcpyFromSymbol(out, g_scan_phase, sizeof(unsigned long long) * 8) != cudaSuccess) return -1;
+  if (clear) {
+    unsigned long long z[8] = {0};
+    cudaMemcpyToSymbol(g_scan_phase, z, sizeof(z));
+  }
+  return 0;
+}
 extern "C" int gdn_debug_phase_cycles_split(unsigned long long* out, int clear) {
   cudaDeviceSynchronize();
   if (cudaMemcpyFromSymbol(out, g_split_phase, sizeof(unsigned long long) * 32) != cudaSuccess) return -1;

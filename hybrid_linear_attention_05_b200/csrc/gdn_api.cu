@@ -127,6 +127,7 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype), records);
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
   if (path == Path::TcSplit && !records) return GDN_ERR_WORKSPACE;
+  if (a->reuse_workspace != 0 && (a->reuse_workspace != 1 || path != Path::TcSplit)) return GDN_ERR_UNSUPPORTED;
   if (!a->cu_seqlens || !a->conv_w || !a->A_log || !a->dt_bias || !a->norm_w) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->mixed_qkv || !a->a || !a->b || !a->z || !a->out || !a->workspace))
     return GDN_ERR_NULL;
@@ -153,13 +154,16 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   cp.q = ws.q; cp.k = ws.k; cp.v = ws.v; cp.g = ws.g; cp.beta = ws.beta;
   cp.T = a->T_tot; cp.N = a->N; cp.Hk = dims->Hk; cp.Hv = dims->Hv; cp.Cc = Cc;
   cp.scale = dims->scale; cp.eps_l2 = dims->eps_l2;
-  s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
-  if (s != GDN_OK) return s;
+  if (!a->reuse_workspace) {
+    s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
+    if (s != GDN_OK) return s;
+  }
 
   ChunkParams ch{};
   ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
   ch.cu_seqlens = a->cu_seqlens; ch.S0 = a->initial_state; ch.S_out = a->final_state;
   ch.z = a->z; ch.norm_w = a->norm_w; ch.out = a->out; ch.o_raw = nullptr;
+  ch.reuse_records = a->reuse_workspace;
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
   ch.eps_norm = dims->eps_norm;
   ch.rec = ws.rec;
@@ -197,8 +201,9 @@ gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* a
   if (!a->workspace || a->workspace_bytes < full) return GDN_ERR_WORKSPACE;
   if (!a->cu_seqlens || !a->conv_w || !a->A_log || !a->dt_bias) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->mixed_qkv || !a->a || !a->b)) return GDN_ERR_NULL;
+  if (a->T_tot > 0 && (a->z == nullptr) != (a->norm_w == nullptr)) return GDN_ERR_NULL;
   const void* ptrs[] = {a->mixed_qkv, a->conv_w, a->a, a->b, a->A_log, a->dt_bias, a->cu_seqlens,
-                        a->conv_state_in, a->conv_state_out, a->workspace, map};
+                        a->conv_state_in, a->conv_state_out, a->workspace, map, a->z, a->norm_w};
   for (const void* p : ptrs)
     if (!aligned16(p)) return GDN_ERR_ALIGN;
   const size_t cs_bytes = (size_t)a->N * Cc * 3 * esize(a->dtype);
@@ -221,7 +226,7 @@ gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* a
   ChunkParams ch{};
   ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
   ch.cu_seqlens = a->cu_seqlens; ch.S0 = nullptr; ch.S_out = nullptr;
-  ch.z = nullptr; ch.norm_w = nullptr; ch.out = nullptr; ch.o_raw = nullptr;
+  ch.z = a->T_tot > 0 ? a->z : nullptr; ch.norm_w = a->norm_w; ch.out = nullptr; ch.o_raw = nullptr;
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
   ch.eps_norm = dims->eps_norm;
   ch.rec = ws.rec;

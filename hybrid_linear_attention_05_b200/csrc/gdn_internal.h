@@ -64,6 +64,9 @@ struct ChunkParams {
   // zero state), and the maps of each (sequence, head), composed in segment
   // order, go to map_out [N][Hv][2][d][d].  With nseg == 1, seg_mr == map_out.
   float* map_out;
+  // the workspace already holds q, k, v, the gates and the records (of a
+  // state-map call on the same inputs): the key-side kernel is not launched
+  int reuse_records;
 };
 
 // chunk_simt.cu: fp32 CUDA-core chunked core.  Supported (d, chunk) pairs:

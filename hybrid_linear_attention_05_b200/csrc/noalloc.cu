@@ -46,6 +46,7 @@ void* scratch_on_current_device() {
 extern "C" gdn_status gdn_prefill_noalloc(const gdn_dims* dims, const gdn_prefill_args* args,
                                           void* stream) {
   if (!dims || !args) return GDN_ERR_NULL;
+  if (args->reuse_workspace) return GDN_ERR_UNSUPPORTED;  // the scratch holds no state map's records
   const size_t need = gdn_prefill_workspace_size(dims, args->T_tot, args->dtype);
   if (args->T_tot > 0 && need == 0) return gdn_prefill(dims, args, stream);  // reports the bad size
   if (need > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;

@@ -59,7 +59,7 @@ class gdn_prefill_args(ctypes.Structure):
                 ("initial_state", _vp), ("final_state", _vp), ("conv_state_in", _vp),
                 ("conv_state_out", _vp), ("out", _vp), ("workspace", _vp),
                 ("workspace_bytes", ctypes.c_size_t), ("core_event_begin", _vp),
-                ("core_event_end", _vp), ("segments", ctypes.c_int)]
+                ("core_event_end", _vp), ("segments", ctypes.c_int), ("reuse_workspace", ctypes.c_int)]
 
 
 class gdn_decode_args(ctypes.Structure):
@@ -183,12 +183,13 @@ def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, n
                 cu_seqlens, N, T_tot, chunk, dtype, out, workspace, workspace_bytes,
                 initial_state=None, final_state=None, conv_state_in=None, conv_state_out=None,
                 impl=GDN_IMPL_AUTO, core_event_begin=None, core_event_end=None, segments=0,
-                stream=None, raise_on_error=True) -> int:
+                reuse_workspace=0, stream=None, raise_on_error=True) -> int:
     args = gdn_prefill_args(
         ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
         ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
         ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
-        ptr(workspace), int(workspace_bytes), core_event_begin, core_event_end, int(segments))
+        ptr(workspace), int(workspace_bytes), core_event_begin, core_event_end, int(segments),
+        int(reuse_workspace))
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill(ctypes.byref(dims), ctypes.byref(args), s), "gdn_prefill",
                   raise_on_error)
@@ -197,7 +198,7 @@ def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, n
 def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,
                         cu_seqlens, N, T_tot, chunk, dtype, out, initial_state=None,
                         final_state=None, conv_state_in=None, conv_state_out=None,
-                        impl=GDN_IMPL_AUTO, stream=None, raise_on_error=True) -> int:
+                        impl=GDN_IMPL_AUTO, reuse_workspace=0, stream=None, raise_on_error=True) -> int:
     """gdn_prefill on the library's own scratch: for callers that have no way
     to allocate a workspace (see gdn.h).  Calls that overlap on the GPU race
     on the shared scratch."""
@@ -205,7 +206,7 @@ def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bi
         ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z),
         ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(impl),
         ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out), ptr(out),
-        None, 0, None, None, 0)
+        None, 0, None, None, 0, int(reuse_workspace))
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_prefill_noalloc(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_prefill_noalloc", raise_on_error)
@@ -213,10 +214,11 @@ def gdn_prefill_noalloc(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bi
 
 def gdn_prefill_state_map(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, cu_seqlens, N,
                           T_tot, chunk, dtype, map_out, workspace, workspace_bytes, conv_state_in=None,
-                          conv_state_out=None, segments=0, stream=None, raise_on_error=True) -> int:
+                          conv_state_out=None, z=None, norm_w=None, segments=0, stream=None,
+                          raise_on_error=True) -> int:
     """(M, R) of every sequence: final state = initial state @ M + R (gdn.h)."""
     args = gdn_prefill_args(
-        ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), None, None,
+        ptr(mixed_qkv), ptr(conv_w), ptr(a), ptr(b), ptr(A_log), ptr(dt_bias), ptr(z), ptr(norm_w),
         ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(dtype), int(GDN_IMPL_TC_SPLIT), None,
         None, ptr(conv_state_in), ptr(conv_state_out), None, ptr(workspace), int(workspace_bytes),
         None, None, int(segments))

@@ -148,6 +148,21 @@ typedef struct {
                                   when N*Hv > 64, return GDN_ERR_UNSUPPORTED.
                                   Every choice computes the same result up to
                                   rounding.                                      */
+  int reuse_workspace;         /* 1: the workspace already holds what this call
+                                  would compute before its state chains -- left
+                                  there by gdn_prefill_state_map on the same
+                                  dims, dtype, inputs (mixed_qkv, conv_w, a, b,
+                                  A_log, dt_bias, cu_seqlens, conv_state_in, and
+                                  z and norm_w, which that call must then have
+                                  been given), N, T_tot and chunk -- so the conv
+                                  and the key-side kernel are skipped and
+                                  conv_state_out is not written.  Two-kernel
+                                  tensor-core path only (GDN_ERR_UNSUPPORTED
+                                  otherwise).  0: compute everything.  A
+                                  context-parallel rank maps its part, folds the
+                                  gathered maps into its start state and then
+                                  runs its part from there without repeating the
+                                  key-side work.                                  */
 } gdn_prefill_args;
 
 /* Bytes of device workspace gdn_prefill needs for these sizes (0 when the
@@ -202,8 +217,11 @@ int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot);
  *         dv = dk), map[n][h][1] = R.  Must not overlap the workspace.
  *   args  as for gdn_prefill; mixed_qkv, conv_w, a, b, A_log, dt_bias,
  *         cu_seqlens and conv_state_in are read, conv_state_out is written
- *         when given; initial_state, final_state, z, norm_w and out are not
- *         used.  segments: 0 = chosen from the sizes, 1 = one serial chain,
+ *         when given; initial_state, final_state and out are not used.  z and
+ *         norm_w are optional (both or neither when T_tot > 0, else
+ *         GDN_ERR_NULL): with them
+ *         the workspace is left ready for gdn_prefill with reuse_workspace = 1
+ *         on the same inputs.  segments: 0 = chosen from the sizes, 1 = one serial chain,
  *         2..7 = that many segments per sequence, composed in fp32 (more than
  *         1 only when N*Hv <= 64).
  *   Supported: bf16, dk = dv = 128, chunk 64 (the tensor-core shapes), with
@@ -236,7 +254,8 @@ gdn_status gdn_state_fold(const gdn_dims* dims, int N, int count, const float* m
  * memory, held on every device that loads the library until the process
  * exits).  It allocates nothing.
  *   - args->workspace and args->workspace_bytes are ignored; every other
- *     argument means what it means for gdn_prefill, with the same checks.
+ *     argument means what it means for gdn_prefill, with the same checks,
+ *     except reuse_workspace, which must be 0 (GDN_ERR_UNSUPPORTED).
  *   - Returns GDN_ERR_WORKSPACE, launching nothing, when the workspace these
  *     sizes need (gdn_prefill_workspace_size) exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES -- about 5400 tokens at 16 key / 16 value

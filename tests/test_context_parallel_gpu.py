@@ -123,3 +123,21 @@ def test_context_parallel_parts_on_one_device(lens):
     whole = api.prefill(dp)
     assert relerr(np64(out), np64(whole.out)) <= PREFILL_TOL
     assert relerr(np64(res[-1].final_state), np64(whole.final_state)) <= PREFILL_TOL
+
+
+def test_prefill_on_a_state_maps_workspace_is_the_full_prefill():
+    """gdn_prefill with reuse_workspace after gdn_prefill_state_map on the same
+    inputs skips the conv and key-side kernels and gives exactly the result
+    of the full call (same records, same chains)."""
+    w = resized(P9B, Hk=2, Hv=4, seed=98, A_log_range=SLOW_DECAY, s0_std=0.02)
+    inp = make_prefill(w, seqlens=(64 * 7 + 5, 64 * 2), with_conv_state=True)
+    dp = api.to_device(inp, chunk=64)
+    full = api.prefill(dp)
+    out, S = full.out.clone(), full.final_state.clone()
+    bufs = api.PrefillBuffers(dp)
+    api.state_map(dp, bufs)
+    r = api.prefill(dp, bufs=bufs, reuse_workspace=True)
+    torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0
+    assert torch.equal(r.out, out)
+    assert torch.equal(r.final_state, S)

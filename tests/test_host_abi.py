@@ -205,3 +205,25 @@ def test_state_fold_rejects_bad_args(L, dims, over, status):
     kw = dict(N=1, count=3, maps=FAKE, S_out=FAKE + (1 << 28), S_first=None, stream=0, raise_on_error=False)
     kw.update(over)
     assert gdn.gdn_state_fold(dims, **kw) == status
+
+
+@pytest.mark.parametrize("over", [dict(reuse_workspace=1, impl=gdn.GDN_IMPL_SIMT),
+                                  dict(reuse_workspace=1, impl=gdn.GDN_IMPL_TC, chunk=64),
+                                  dict(reuse_workspace=2, impl=gdn.GDN_IMPL_TC_SPLIT, chunk=64)])
+def test_reuse_workspace_only_on_the_two_kernel_path(L, over):
+    dims = gdn.make_dims(2, 4, 128)
+    assert gdn.gdn_prefill(dims, **prefill_kwargs(**over)) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_reuse_workspace_rejected_without_workspace(L):
+    dims = gdn.make_dims(2, 4, 128)
+    assert gdn.gdn_prefill_noalloc(dims, mixed_qkv=FAKE, conv_w=FAKE, a=FAKE, b=FAKE, A_log=FAKE,
+                                   dt_bias=FAKE, z=FAKE, norm_w=FAKE, cu_seqlens=FAKE, N=1, T_tot=16,
+                                   chunk=64, dtype=gdn.GDN_BF16, out=FAKE, reuse_workspace=1, stream=0,
+                                   raise_on_error=False) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_state_map_gate_inputs_both_or_neither(L):
+    dims = gdn.make_dims(2, 4, 128)
+    assert gdn.gdn_prefill_state_map(dims, **map_kwargs(z=FAKE)) == gdn.GDN_ERR_NULL
+    assert gdn.gdn_prefill_state_map(dims, **map_kwargs(norm_w=FAKE)) == gdn.GDN_ERR_NULL
