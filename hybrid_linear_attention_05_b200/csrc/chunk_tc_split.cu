@@ -1104,7 +1104,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     sg_next = next_map(sg + 1);
     if (tid == 0 && sg_next < P - 1) prefetch(sg_next, buf ^ 1);
     const float* M = Mb + buf * D * D;
-#pragma unroll 4
+#pragma unroll 8
     for (int i = ks * (D / SCAN_KS); i < (ks + 1) * (D / SCAN_KS); ++i) {
       const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
       const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);
@@ -1275,7 +1275,7 @@ __global__ void __launch_bounds__(FOLD_THREADS) state_fold_kernel(FoldParams p) 
     }
     if (tid == 0 && s + 1 < p.nmaps) prefetch(s + 1, buf ^ 1);
     const float* M = Mb + buf * D * D;
-#pragma unroll 4
+#pragma unroll 8
     for (int i = ks * (D / FOLD_KS); i < (ks + 1) * (D / FOLD_KS); ++i) {
       const float4 s4 = *reinterpret_cast<const float4*>(sT + i * SR + rr);
       const float4 m4 = *reinterpret_cast<const float4*>(M + i * D + cc);

@@ -172,44 +172,15 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
   const float4 k4 = make_float4(kv[col], kv[col + 1], kv[col + 2], kv[col + 3]);
   const float4 q4 = make_float4(qv[col], qv[col + 1], qv[col + 2], qv[col + 3]);
   const float kq = misc[2];
-  // fp32 state: the row sums of RG passes at a time are reduced together
-  // (rows_sum_transposed); bf16 state: one pass at a time, each row's sums
-  // reduced on their own (measured faster there: 106 against 130 us at batch
-  // 256, 16/32 heads of width 128)
-  constexpr int RG = PASSES < 8 ? PASSES : 8;
+  // the row sums of RG passes at a time are reduced together
+  // (rows_sum_transposed): 8 for an fp32 state, 4 for a bf16 one (measured at
+  // batch 256, 16/32 heads of width 128: 102 us against 106 us with each
+  // row's sums reduced on their own and 130 us with 8)
+  constexpr int RG = std::is_same<SD, float>::value ? (PASSES < 8 ? PASSES : 8) : (PASSES < 4 ? PASSES : 4);
   static_assert(RG <= LPR && PASSES % RG == 0, "decode layout");
   const int jr = (lane % LPR) / (LPR / RG);  // the pass of a group whose sums this lane ends with
   const int src0 = lane - lane % LPR;        // first lane of this lane's row group
-  if constexpr (!std::is_same<SD, float>::value) {
-    for (int gi = 0; gi < G; ++gi) {
-      const int h = kh * G + gi;
-      const float alpha = misc[4 + gi], beta = misc[4 + G + gi];
-      SD* Sh = state + ((size_t)b * p.Hv + h) * D * D;
-      const SD* Snext = gi + 1 < G ? state_of(gi + 1) : nullptr;
-      const float* vv = ys + (2 + gi) * D;
-#pragma unroll
-      for (int s = 0; s < PASSES; ++s) {
-        const int r = row_of(s);
-        const float4 sv = SV::widen(Sv[s]);
-        float u = sv.x * k4.x + sv.y * k4.y + sv.z * k4.z + sv.w * k4.w;
-        float pp = sv.x * q4.x + sv.y * q4.y + sv.z * q4.z + sv.w * q4.w;
-#pragma unroll
-        for (int o = LPR / 2; o > 0; o >>= 1) {
-          u += __shfl_xor_sync(0xffffffffu, u, o, 32);
-          pp += __shfl_xor_sync(0xffffffffu, pp, o, 32);
-        }
-        const float delta = beta * (vv[r] - alpha * u);
-        float4 sn;
-        sn.x = fmaf(alpha, sv.x, delta * k4.x);
-        sn.y = fmaf(alpha, sv.y, delta * k4.y);
-        sn.z = fmaf(alpha, sv.z, delta * k4.z);
-        sn.w = fmaf(alpha, sv.w, delta * k4.w);
-        SV::store(Sh + (size_t)r * D + col, sn);
-        if ((lane % LPR) == 0) os[gi * D + r] = fmaf(alpha, pp, kq * delta);
-        if (Snext) Sv[s] = SV::load(Snext + (size_t)r * D + col);
-      }
-    }
-  } else for (int gi = 0; gi < G; ++gi) {
+  for (int gi = 0; gi < G; ++gi) {
     const int h = kh * G + gi;
     const float alpha = misc[4 + gi], beta = misc[4 + G + gi];
     SD* Sh = state + ((size_t)b * p.Hv + h) * D * D;
