@@ -217,13 +217,13 @@ int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot);
  *         dv = dk), map[n][h][1] = R.  Must not overlap the workspace.
  *   args  as for gdn_prefill; mixed_qkv, conv_w, a, b, A_log, dt_bias,
  *         cu_seqlens and conv_state_in are read, conv_state_out is written
- *         when given; initial_state, final_state and out are not used.  z and
- *         norm_w are optional (both or neither when T_tot > 0, else
- *         GDN_ERR_NULL): with them
- *         the workspace is left ready for gdn_prefill with reuse_workspace = 1
- *         on the same inputs.  segments: 0 = chosen from the sizes, 1 = one serial chain,
- *         2..7 = that many segments per sequence, composed in fp32 (more than
- *         1 only when N*Hv <= 64).
+ *         when given; initial_state, final_state and out are not used.
+ *         z and norm_w are optional (both or neither when T_tot > 0, else
+ *         GDN_ERR_NULL): with them the workspace is left ready for
+ *         gdn_prefill with reuse_workspace = 1 on the same inputs.
+ *         segments: 0 = chosen from the sizes, 1 = one serial chain, 2..7 =
+ *         that many segments per sequence, composed in fp32 (more than 1
+ *         only when N*Hv <= 64).
  *   Supported: bf16, dk = dv = 128, chunk 64 (the tensor-core shapes), with
  *   gdn_prefill_workspace_size_n bytes of workspace; GDN_ERR_UNSUPPORTED /
  *   GDN_ERR_WORKSPACE otherwise.  An empty sequence gives M = I, R = 0.
