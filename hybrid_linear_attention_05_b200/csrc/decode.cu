@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
 // decode): each state row takes the T tokens' updates in turn while it is in
 // registers, so the state is still read and written once per step.
 template <typename T, typename SD, int D>
-__global__ void __launch_bounds__(256, 2) decode_multi_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(256, 3) decode_multi_kernel(DecodeParams p) {
   using SV = State4<SD>;
   constexpr int NT = 256, NW = NT / 32;
   constexpr int LPR = D / 4;            // lanes per state row
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(256, 2) decode_multi_kernel(DecodeParams p) {
   // A thread's rows of a head are taken RG at a time (a "group"); the first
   // group is requested before anything else, each next one while the current
   // one is updated, so the state latency overlaps the conv and the updates.
-  constexpr int RG = PASSES < 8 ? PASSES : 8;
+  constexpr int RG = PASSES < 4 ? PASSES : 4;
   constexpr int NGH = PASSES / RG;  // groups per head
   static_assert(RG <= LPR, "decode layout");
   const int col = (lane % LPR) * 4;
