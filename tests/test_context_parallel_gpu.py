@@ -76,7 +76,24 @@ def test_state_map_matches_oracle(segments, seqlens):
     np.testing.assert_array_equal(np64(cs_out), oracle_prefill(inp).conv_state_out)
 
 
-@pytest.mark.parametrize("count,with_first,in_place", [(0, True, False), (1, False, False),
+def test_state_map_many_chains():
+    """17 sequences x 4 value heads (68 chains, past the segment buffers): one
+    serial chain per (sequence, head) writes its maps straight into the
+    caller's array."""
+    w = resized(P9B, Hk=2, Hv=4, seed=96, A_log_range=SLOW_DECAY)
+    rng = np.random.default_rng(96)
+    seqlens = tuple(int(x) for x in rng.integers(1, 200, 17))
+    inp = make_prefill(w, seqlens=seqlens, with_conv_state=True)
+    dp = api.to_device(inp, chunk=64)
+    maps = api.state_map(dp)
+    torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0
+    for n, (M, R) in enumerate(oracle_maps(inp)):
+        assert relerr(np64(maps[n, :, 0]), M) <= PREFILL_TOL
+        assert relerr(np64(maps[n, :, 1]), R) <= PREFILL_TOL
+
+
+@pytest.mark.parametrize("count,with_first,in_place", [(0, True, False), (0, False, False), (1, False, False),
                                                         (3, True, False), (5, True, True)])
 def test_state_fold_matches_fp64(count, with_first, in_place):
     """S <- S M_s + R_s over `count` maps of two sequences and three heads."""
@@ -95,8 +112,8 @@ def test_state_fold_matches_fp64(count, with_first, in_place):
     got = api.state_fold(dev_maps, first, Hk=1, Hv=Hv, d=d, out=out)
     torch.cuda.synchronize()
     assert gdn.gdn_device_error(True) == 0
-    if count == 0 and S0 is not None:
-        np.testing.assert_array_equal(np64(got), S0)
+    if count == 0:
+        np.testing.assert_array_equal(np64(got), 0.0 if S0 is None else S0)
     else:
         assert relerr(np64(got), ref) <= FOLD_TOL
 
