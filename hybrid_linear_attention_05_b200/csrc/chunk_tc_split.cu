@@ -44,6 +44,12 @@
 //     leaves the segment's M) and from S = 0 (its R).  seg_scan_kernel then
 //     walks the segments, S_start(s+1) = S_start(s) M_s + R_s in fp32, and the
 //     output chains run all segments at once from their start states.
+//  4. State-map mode (gdn_prefill_state_map, for context-parallel prefill):
+//     the transfer chains run every segment, both maps of segment 0 too and
+//     R from a zero state, and state_fold_kernel composes the segments' maps
+//     in order into the map of the whole sequence; no output chain runs.
+//     state_fold_kernel also folds gathered maps into a start state
+//     (gdn_state_fold).
 // The algebra is the chunked (WY / UT transform) form of the recurrence, exact
 // in real arithmetic ("Qwen (text & vision-language)", Verified parity).
 // No TMA multicast is used.
