@@ -6,7 +6,6 @@ the fold order, the final state from the last rank) runs here on gloo ranks,
 with the three compute calls answered by the fp64 oracle instead of the CUDA
 library.  The result must be the oracle's own prefill of the whole sequence.
 """
-import math
 import os
 import socket
 import sys
@@ -170,3 +169,23 @@ def test_context_parallel_gloo_ranks(lens):
     assert rel(np.concatenate([g[1] for g in got]), whole.out) < 1e-12
     for g in got:  # every rank holds the sequence's final state
         assert rel(g[2], whole.final_state) < 1e-12
+
+
+def test_split_sequence_and_tails():
+    """Parts are consecutive slices with their own cu_seqlens; a part's tail
+    is its last min(3, T) rows, right-aligned in zeros."""
+    inp = _inputs(10, 7)
+    dp = _device_prefill(inp, 0, 10)
+    parts = cp.split_sequence(dp, [4, 0, 1, 5])
+    assert [p.T for p in parts] == [4, 0, 1, 5]
+    got = torch.cat([p.mixed_qkv for p in parts]).numpy()
+    np.testing.assert_array_equal(got, inp["mixed_qkv"])
+    for p in parts:
+        assert p.cu_seqlens.tolist() == [0, p.T] and p.N == 1
+        assert p.initial_state is None and p.conv_state_in is None
+        t = cp._tail(p.mixed_qkv).numpy()
+        take = min(3, p.T)
+        np.testing.assert_array_equal(t[:3 - take], 0.0)
+        np.testing.assert_array_equal(t[3 - take:], p.mixed_qkv.numpy()[p.T - take:])
+    with pytest.raises(AssertionError):
+        cp.split_sequence(dp, [4, 5])  # lengths must cover the sequence
