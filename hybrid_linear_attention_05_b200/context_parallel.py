@@ -108,8 +108,8 @@ def prefill_context_parallel(part: api.DevicePrefill, group=None, compute=None,
     token order.  initial_state [1, Hv, d, d] / conv_state_in [1, Cc, 3]: the
     sequence's own, the same on every rank (None: zeros); part.initial_state
     and part.conv_state_in are ignored.  Every rank calls this with its part;
-    the collectives are: one all-gather of the tails and lengths, one of the
-    maps, one broadcast of the final state."""
+    the collectives, in this order on every rank: an all-gather of the tails,
+    one of the lengths, one of the maps, and a broadcast of the final state."""
     compute = compute or LibraryCompute()
     W = dist.get_world_size(group)
     r = dist.get_rank(group)
