@@ -396,4 +396,16 @@ int gdn_oracle_core(int Hk, int Hv, int dk, int dv, int N, const int64_t* cu_seq
   return run_core(D, N, cu_seqlens, q, k, v, g, beta, S0, o, S_final, chunk, nthreads);
 }
 
+// The element-wise pieces on their own, so that the tests can pin them at
+// hand-evaluated points: y[i] = silu(x[i]) (step 2), and step 6 over `rows`
+// independent (token, value head) rows of width dv with one dv-wide weight.
+void gdn_oracle_silu(int n, const double* x, double* y) {
+  for (int i = 0; i < n; ++i) y[i] = silu(x[i]);
+}
+void gdn_oracle_gated_rmsnorm(int rows, int dv, double eps, const double* o, const double* z,
+                              const double* w, double* out) {
+  for (int r = 0; r < rows; ++r)
+    gated_rmsnorm(dv, eps, o + (size_t)r * dv, z + (size_t)r * dv, w, out + (size_t)r * dv);
+}
+
 }  // extern "C"

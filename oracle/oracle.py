@@ -47,6 +47,10 @@ def _load():
         _lib.gdn_oracle_decode.restype = i
         _lib.gdn_oracle_core.argtypes = [i, i, i, i, i, lp] + [dp] * 6 + [dp, dp, i, i]
         _lib.gdn_oracle_core.restype = i
+        _lib.gdn_oracle_silu.argtypes = [i, dp, dp]
+        _lib.gdn_oracle_silu.restype = None
+        _lib.gdn_oracle_gated_rmsnorm.argtypes = [i, i, d, dp, dp, dp, dp]
+        _lib.gdn_oracle_gated_rmsnorm.restype = None
     return _lib
 
 
@@ -192,3 +196,25 @@ def core(Hk, Hv, dk, dv, cu_seqlens, q, k, v, g, beta, initial_state=None, chunk
     if rc != 0:
         raise ValueError("oracle rejected the dimensions")
     return o, S
+
+
+def silu(x):
+    """The oracle's SiLU (step 2 of the mixer), element-wise."""
+    lib = _load()
+    x = _d(x)
+    y = np.zeros_like(x)
+    lib.gdn_oracle_silu(int(x.size), _ptr(x), _ptr(y))
+    return y
+
+
+def gated_rmsnorm(o, z, w, eps=1e-6):
+    """The oracle's gated RMSNorm (step 6) over the last axis of o and z, with
+    the one weight vector w shared by every row."""
+    lib = _load()
+    o, z, w = _d(o), _d(z), _d(w)
+    dv = int(o.shape[-1])
+    assert z.shape == o.shape and w.shape == (dv,)
+    out = np.zeros_like(o)
+    lib.gdn_oracle_gated_rmsnorm(int(o.size // max(dv, 1)), dv, float(eps), _ptr(o), _ptr(z), _ptr(w),
+                                 _ptr(out))
+    return out

@@ -197,6 +197,50 @@ def test_golden_gates(oracle_mod):
     np.testing.assert_allclose(r.beta[0], rows[:, 5], rtol=1e-12, atol=0)
 
 
+def _golden_rows(name, tag):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line.startswith(tag + " "):
+                rows.append([float(x) for x in line.split()[1:]])
+    return np.array(rows)
+
+
+def test_golden_silu(oracle_mod):
+    """SiLU at hand-evaluated points (tests/golden/silu_norm.txt): a dropped
+    factor x, a sign slip in the sigmoid or a swapped argument fails a row."""
+    rows = _golden_rows("silu_norm.txt", "silu")
+    assert rows.shape == (6, 2)
+    y = oracle_mod.silu(rows[:, 0])
+    np.testing.assert_allclose(y, rows[:, 1], rtol=2e-15, atol=0)
+
+
+def test_golden_gated_rmsnorm(oracle_mod):
+    """The gated RMSNorm at hand-evaluated rows (tests/golden/silu_norm.txt):
+    eps near, above and below mean(o^2), per-channel weights and gates, a
+    mean (not a sum) over the row, and eps = 0."""
+    rows = _golden_rows("silu_norm.txt", "norm")
+    assert rows.shape == (5, 17)
+    for r in rows:
+        eps, o, z, w, expect = r[0], r[1:5], r[5:9], r[9:13], r[13:17]
+        out = oracle_mod.gated_rmsnorm(o[None], z[None], w, eps=eps)[0]
+        np.testing.assert_allclose(out, expect, rtol=2e-15, atol=1e-300)
+
+
+def test_mixer_uses_the_pinned_silu_and_norm(oracle_mod):
+    """The whole mixer applies exactly the pinned pieces: v is silu of the conv
+    output, and out is the gated RMSNorm of the core output o."""
+    rng = np.random.default_rng(21)
+    Hk, Hv, d = 1, 2, 8
+    inp = mixer_inputs(rng, [5, 3], Hk, Hv, d)
+    r = oracle_mod.prefill(Hk, Hv, d, d, **inp)
+    T = r.o.shape[0]
+    np.testing.assert_array_equal(r.v.reshape(T, Hv * d), oracle_mod.silu(r.y_pre[:, 2 * Hk * d:]))
+    out = oracle_mod.gated_rmsnorm(r.o, inp["z"].reshape(T, Hv, d), inp["norm_w"], eps=1e-6)
+    np.testing.assert_array_equal(r.out, out)
+
+
 def test_conv_impulse_and_history(oracle_mod):
     """Single-tap conv weights reproduce the input shifted by (3 - tap); the
     positions before the sequence start come from the conv history, oldest
