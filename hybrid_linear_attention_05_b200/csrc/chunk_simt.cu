@@ -73,6 +73,10 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(ChunkParams p) {
         kv = ld_f(kg + (t * p.Hk + hk) * D + l);
         qv = ld_f(qg + (t * p.Hk + hk) * D + l);
         vv = ld_f(vg + (t * p.Hv + h) * D + l);
+        if (p.k_lo) {  // fp16 q, k plus their rounding residuals
+          kv += ld_f(static_cast<const TM*>(p.k_lo) + (t * p.Hk + hk) * D + l);
+          qv += ld_f(static_cast<const TM*>(p.q_lo) + (t * p.Hk + hk) * D + l);
+        }
       }
       Ks[i * DP + l] = kv; Qs[i * DP + l] = qv; Vs[i * DP + l] = vv;
     }

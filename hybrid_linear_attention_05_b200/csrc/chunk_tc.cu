@@ -33,24 +33,6 @@ namespace gdn {
 
 __device__ int g_tc_error = 0;  // nonzero: a bounded wait in a kernel gave up
 
-#ifdef GDN_PHASE_TIMING
-// Development aid (off by default): SM cycles spent by CTA thread 0 in each
-// phase of the chunk loop, summed over all CTAs.
-__device__ unsigned long long g_phase_cycles[16];
-#define GDN_PHASE(k)                                             \
-  do {                                                           \
-    if (tid == 0) {                                              \
-      const long long t_ = clock64();                            \
-      atomicAdd(&g_phase_cycles[k], (unsigned long long)(t_ - t_prev)); \
-      t_prev = t_;                                               \
-    }                                                            \
-  } while (0)
-#else
-#define GDN_PHASE(k) \
-  do {               \
-  } while (0)
-#endif
-
 namespace {
 
 using namespace ptx;
@@ -81,7 +63,7 @@ constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;     // fp32 T [64][AS]; before
 constexpr uint32_t OFF_RS = OFF_TF + 64 * AS * 4;     // fp32 scratch of the inverse, 1024 floats
 constexpr uint32_t OFF_MISC = OFF_RS + 1024 * 4;      // gamma, e^gamma, beta, rms, e^{gamma_L - gamma}, scan
 constexpr uint32_t OFF_BAR = OFF_MISC + 5 * 64 * 4 + 64;
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t SMEM_USED = OFF_BAR + 80;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(OFF_AF + 64 * 128 * 4 <= OFF_RS, "epilogue staging overlaps the scratch");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -96,6 +78,7 @@ constexpr uint32_t STAGE_TX = 6 * TILE_BYTES;       // K, Q (2 halves each), V (
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
+                    const __grid_constant__ CUtensorMap tm_ql, const __grid_constant__ CUtensorMap tm_kl,
                     ChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -116,7 +99,13 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t bar_load0 = sb + OFF_BAR, bar_z = sb + OFF_BAR + 16;
   const uint32_t bar_m1 = sb + OFF_BAR + 24, bar_w = sb + OFF_BAR + 32, bar_v = sb + OFF_BAR + 40,
                  bar_o = sb + OFF_BAR + 48;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 56);
+  const uint32_t bar_lo = sb + OFF_BAR + 56;  // the chunk's [K_lo; Q_lo] tiles
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 64);
+  // With the rounding residuals of q and k, D1 also takes [K_lo; Q_lo] K^T and
+  // [K; Q] K_lo^T.  Their dk halves (laid out like [K; Q]) land in OFF_TB (the
+  // TB and TBE tiles) and OFF_VTS at the top of each chunk: the previous
+  // chunk's last MMAs, which read those regions, have completed by then.
+  const bool has_lo = p.k_lo != nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7;     // warpgroup: which column quarter of a TMEM row this thread handles
@@ -143,6 +132,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(bar_w, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_lo, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -197,9 +187,6 @@ __global__ void __launch_bounds__(NT, 1)
 
   bool ok = true;
   int c = 0;
-#ifdef GDN_PHASE_TIMING
-  long long t_prev = clock64();
-#endif
   for (; c < nchunks; ++c) {
     const int s = c & 1;
     const int c0 = bos + c * C;
@@ -209,6 +196,13 @@ __global__ void __launch_bounds__(NT, 1)
     uint8_t* wt_ptr = smem + (s ? OFF_V1 : OFF_V0);  // -W^T reuses the consumed V tile
 
     if (tid == 0) {
+      if (has_lo) {
+        mbar_arrive_expect_tx(bar_lo, 4 * TILE_BYTES);
+        tma_load_2d(sb + OFF_TB, &tm_kl, hk * D, c0, bar_lo);
+        tma_load_2d(sb + OFF_VTS, &tm_kl, hk * D + 64, c0, bar_lo);
+        tma_load_2d(sb + OFF_TB + 8192, &tm_ql, hk * D, c0, bar_lo);
+        tma_load_2d(sb + OFF_VTS + 8192, &tm_ql, hk * D + 64, c0, bar_lo);
+      }
       if (c + 1 < nchunks) issue_loads(c + 1, s ^ 1);
       if (norm_out) {
         mbar_arrive_expect_tx(bar_z, 2 * TILE_BYTES);
@@ -237,18 +231,24 @@ __global__ void __launch_bounds__(NT, 1)
     }
 
     // ---- D1 = [K; Q] K^T
-    ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
-    if (__syncthreads_or(!ok)) break;
-    GDN_PHASE(0);
     const uint32_t par = (uint32_t)c & 1u;  // phase parity of the once-per-chunk barriers
+    ok = mbar_wait(bar_load0 + 8 * s, (uint32_t)(c >> 1) & 1u);
+    if (has_lo) ok = mbar_wait(bar_lo, par) && ok;
+    if (__syncthreads_or(!ok)) break;
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, false, false);
+      const uint32_t lo_half[2] = {sb + OFF_TB, sb + OFF_VTS};
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + TM_D1, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
-                kk > 0);
+        const uint64_t dh = sdesc_sw128(kq + off, 16, 1024);
+        mma_f16(tmem + TM_D1, dh, dh, id, kk > 0);
+        if (has_lo) {
+          const uint64_t lw = sdesc_sw128(lo_half[kk >> 2] + (kk & 3) * 32, 16, 1024);
+          mma_f16(tmem + TM_D1, lw, dh, id, 1);
+          mma_f16(tmem + TM_D1, dh, lw, id, 1);
+        }
       }
       mma_commit(bar_m1);
     }
@@ -279,7 +279,6 @@ __global__ void __launch_bounds__(NT, 1)
     ok = mbar_wait(bar_m1, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    GDN_PHASE(1);
 
     // ---- A (rows 0..63) and P (rows 64..127); this thread: columns wg*CW .. wg*CW+CW-1
     {
@@ -316,11 +315,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
     __syncthreads();
-    GDN_PHASE(2);
 
     // ---- T = (I + A)^-1, then the B operands T diag(beta) and T diag(beta e^gamma)
     solve_unit_lower<NT>(Af, Tf, Xs, tid);
-    GDN_PHASE(3);
     {
       const int i = tid >> 3, qt = tid & 7;  // row i, 8 columns (one 16-byte chunk) per thread
       uint8_t* Tb = smem + OFF_TB;
@@ -367,7 +364,6 @@ __global__ void __launch_bounds__(NT, 1)
     ok = mbar_wait(bar_w, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    GDN_PHASE(4);
 
     // ---- -W^T as the MN-major B operand (row l = tl, tokens wg*CW .. wg*CW+CW-1)
     {
@@ -405,7 +401,6 @@ __global__ void __launch_bounds__(NT, 1)
     ok = mbar_wait(bar_v, par);
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    GDN_PHASE(5);
 
     // ---- Vn^T rows: plain (A of D5) and decayed to the chunk end (A of the state update)
     {
@@ -457,7 +452,6 @@ __global__ void __launch_bounds__(NT, 1)
     ok = mbar_wait(bar_o, par) && ok;
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    GDN_PHASE(6);
 
     // ---- epilogue: O^T = D4 diag(e^gamma) + D5 for tokens wg*CW .. +CW-1, staged as O [token][v]
     float o[CW];
@@ -473,7 +467,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
     __syncthreads();
-    GDN_PHASE(7);
     if (norm_out) {
       // 1 / rms per token: warp w reduces tokens TPW*w .. TPW*w+TPW-1
       constexpr int TPW = 64 / NW;
@@ -521,7 +514,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
     __syncthreads();
-    GDN_PHASE(8);
   }
 
   if (!ok) {
@@ -533,6 +525,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (c + 1 < nchunks)
         mbar_wait(bar_load0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, 100000000ull);
       if (norm_out) mbar_wait(bar_z, (uint32_t)c & 1u, 100000000ull);
+      if (has_lo) mbar_wait(bar_lo, (uint32_t)c & 1u, 100000000ull);
       mbar_wait(bar_o, (uint32_t)c & 1u, 100000000ull);  // tensor-core work of this chunk
     }
   } else if (p.S_out) {
@@ -592,11 +585,14 @@ bool chunk_tc_supported(int d, int chunk, gdn_dtype dt_mid) {
 
 cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st) {
   if (p.N == 0 || p.Hv == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mz;
+  CUtensorMap mq, mk, mv, mz, mql, mkl;
   memset(&mq, 0, sizeof(mq));
   memset(&mk, 0, sizeof(mk));
   memset(&mv, 0, sizeof(mv));
   memset(&mz, 0, sizeof(mz));
+  memset(&mql, 0, sizeof(mql));
+  memset(&mkl, 0, sizeof(mkl));
+  if ((p.q_lo == nullptr) != (p.k_lo == nullptr)) return cudaErrorInvalidValue;
   if (p.T > 0) {
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -607,28 +603,19 @@ cudaError_t launch_chunk_tc(const ChunkParams& p, cudaStream_t st) {
     if (p.out && !make_map(&mz, p.z, (uint64_t)p.T, (uint64_t)p.Hv * D,
                            CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
+    if (p.k_lo && (!make_map(&mql, p.q_lo, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
+                   !make_map(&mkl, p.k_lo, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw)))
+      return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.Hv, p.N);
-  chunk_tc_kernel<<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mz, p);
+  chunk_tc_kernel<<<grid, NT, SMEM_BYTES, st>>>(mq, mk, mv, mz, mql, mkl, p);
   return cudaGetLastError();
 }
 
 }  // namespace gdn
-
-#ifdef GDN_PHASE_TIMING
-extern "C" int gdn_debug_phase_cycles(unsigned long long* out, int clear) {
-  cudaDeviceSynchronize();
-  if (cudaMemcpyFromSymbol(out, gdn::g_phase_cycles, sizeof(unsigned long long) * 16) != cudaSuccess) return -1;
-  if (clear) {
-    unsigned long long z[16] = {0};
-    cudaMemcpyToSymbol(gdn::g_phase_cycles, z, sizeof(z));
-  }
-  return 0;
-}
-#endif
 
 extern "C" gdn_status gdn_device_error(int* code, int clear) {
   if (!code) return GDN_ERR_NULL;
@@ -643,6 +630,32 @@ extern "C" gdn_status gdn_device_error(int* code, int clear) {
   if (v2 < 0) return GDN_ERR_CUDA;
   const int v3 = gdn::conv_error_word(clear);
   if (v3 < 0) return GDN_ERR_CUDA;
-  *code = v != 0 ? v : (v2 != 0 ? v2 : v3);
+  const int v4 = gdn::fused_error_word(clear);
+  if (v4 < 0) return GDN_ERR_CUDA;
+  *code = (v | v2 | v3 | v4) != 0 ? GDN_ERR_TIMEOUT : 0;
   return GDN_OK;
+}
+
+namespace gdn {
+namespace {
+// One warp waits on an mbarrier that nothing arrives at, through the bounded
+// wait of the tensor-core kernels, and records that it gave up.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = ptx::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(b, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = ptx::mbar_wait(b, 0, limit_ns);
+  if (!__any_sync(0xffffffffu, ok) && threadIdx.x == 0) atomicExch(&g_tc_error, 1);
+}
+}  // namespace
+}  // namespace gdn
+
+extern "C" gdn_status gdn_selftest_bounded_wait(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return GDN_ERR_DIMS;
+  gdn::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -64,59 +64,6 @@ namespace gdn {
 
 __device__ int g_split_error = 0;  // nonzero: a bounded wait in a kernel of this file gave up
 
-#ifdef GDN_PHASE_TIMING
-// Development aid (off by default): SM cycles spent by chain-kernel thread 0
-// in each phase of the chunk loop, summed over all CTAs.
-__device__ unsigned long long g_split_phase[32];
-// seg_scan_kernel, thread 0 of every CTA: cycles per phase, summed
-__device__ unsigned long long g_scan_phase[8];
-#define GDN_SCAN_MARK(k)                                                \
-  do {                                                                  \
-    if (tid == 0) {                                                     \
-      const long long t_ = clock64();                                   \
-      atomicAdd(&g_scan_phase[k], (unsigned long long)(t_ - t_prev));   \
-      t_prev = t_;                                                      \
-    }                                                                   \
-  } while (0)
-#define GDN_SPLIT_MARK(k)                                               \
-  do {                                                                  \
-    if (tid == NCW + 64) {                                              \
-      const long long t_ = clock64();                                   \
-      atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
-      t_prev = t_;                                                      \
-    }                                                                   \
-  } while (0)
-#define GDN_SPLIT_PHASE(k)                                              \
-  do {                                                                  \
-    if (tid == 0 || tid == 64) {                                        \
-      const long long t_ = clock64();                                   \
-      atomicAdd(&g_split_phase[(k) + (tid ? 8 : 0)], (unsigned long long)(t_ - t_prev));  \
-      t_prev = t_;                                                      \
-    }                                                                   \
-  } while (0)
-#define GDN_KEYS_MARK(k)                                                \
-  do {                                                                  \
-    if (tid == 0) {                                                     \
-      const long long t_ = clock64();                                   \
-      atomicAdd(&g_split_phase[k], (unsigned long long)(t_ - t_prev));  \
-      t_prev = t_;                                                      \
-    }                                                                   \
-  } while (0)
-#else
-#define GDN_KEYS_MARK(k) \
-  do {                   \
-  } while (0)
-#define GDN_SPLIT_PHASE(k) \
-  do {                     \
-  } while (0)
-#define GDN_SPLIT_MARK(k) \
-  do {                    \
-  } while (0)
-#define GDN_SCAN_MARK(k) \
-  do {                   \
-  } while (0)
-#endif
-
 namespace {
 
 using namespace ptx;
@@ -159,7 +106,8 @@ static_assert(2 * A_SMEM <= 232448, "two key-side CTAs per SM");
 
 __global__ void __launch_bounds__(NTA, 2)
     chunk_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, ChunkParams p) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ql,
+                      const __grid_constant__ CUtensorMap tm_kl, ChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -230,9 +178,6 @@ __global__ void __launch_bounds__(NTA, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-#ifdef GDN_PHASE_TIMING
-  long long t_prev = clock64();
-#endif
   pdl_wait();  // q, k, v and the gates come from the conv kernel
   float gv = 0.f, bv = 0.f;
   if (tid < L) {
@@ -240,14 +185,24 @@ __global__ void __launch_bounds__(NTA, 2)
     bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
   }
 
+  // With the rounding residuals of q and k, D1 also takes [K_lo; Q_lo] K^T
+  // and [K; Q] K_lo^T; their tiles ([K_lo; Q_lo] dk halves, laid out like
+  // [K; Q]) land in A_TBP and A_AF, which nothing uses before D1 completes.
+  const bool has_lo = p.k_lo != nullptr;
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_load, 6 * TILE);
+    mbar_arrive_expect_tx(bar_load, (has_lo ? 10 : 6) * TILE);
     tma_load_2d(sb + A_KQ, &tm_k, hk * D, c0, bar_load);
     tma_load_2d(sb + A_KQ + 16384, &tm_k, hk * D + 64, c0, bar_load);
     tma_load_2d(sb + A_KQ + 8192, &tm_q, hk * D, c0, bar_load);
     tma_load_2d(sb + A_KQ + 16384 + 8192, &tm_q, hk * D + 64, c0, bar_load);
     tma_load_2d(sb + A_V, &tm_v, h * D, c0, bar_load);
     tma_load_2d(sb + A_V + TILE, &tm_v, h * D + 64, c0, bar_load);
+    if (has_lo) {
+      tma_load_2d(sb + A_TBP, &tm_kl, hk * D, c0, bar_load);
+      tma_load_2d(sb + A_AF, &tm_kl, hk * D + 64, c0, bar_load);
+      tma_load_2d(sb + A_TBP + 8192, &tm_ql, hk * D, c0, bar_load);
+      tma_load_2d(sb + A_AF + 8192, &tm_ql, hk * D + 64, c0, bar_load);
+    }
   }
   if (gated && tid < D) wsm[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tid]);
   // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
@@ -267,18 +222,23 @@ __global__ void __launch_bounds__(NTA, 2)
     bet[tid] = bv;
   }
 
-  GDN_KEYS_MARK(21);
   bool ok = mbar_wait(bar_load, 0);
-  GDN_KEYS_MARK(22);
   if (!__syncthreads_or(!ok)) {
-    if (tid == 0) {  // D1 = [K; Q] K^T
+    if (tid == 0) {  // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T)
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, false, false);
       const uint64_t dkq = sdesc_sw128(sb + A_KQ, 16, 1024);
+      const uint64_t dlo[2] = {sdesc_sw128(sb + A_TBP, 16, 1024), sdesc_sw128(sb + A_AF, 16, 1024)};
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tmem + A_TM_D1, sdesc_add(dkq, off), sdesc_add(dkq, off), id, kk > 0);
+        const uint64_t dh = sdesc_add(dkq, off);
+        mma_f16(tmem + A_TM_D1, dh, dh, id, kk > 0);
+        if (has_lo) {
+          const uint64_t lw = sdesc_add(dlo[kk >> 2], (kk & 3) * 32);
+          mma_f16(tmem + A_TM_D1, lw, dh, id, 1);
+          mma_f16(tmem + A_TM_D1, dh, lw, id, 1);
+        }
       }
       mma_commit(bar_m1);
     }
@@ -298,10 +258,8 @@ __global__ void __launch_bounds__(NTA, 2)
       vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
       if (tid == 0) vec[64] = eg[L - 1];
     }
-    GDN_KEYS_MARK(23);
     ok = mbar_wait(bar_m1, 0);
   }
-  GDN_KEYS_MARK(24);
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
     // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
@@ -339,9 +297,7 @@ __global__ void __launch_bounds__(NTA, 2)
       }
     }
     __syncthreads();
-    GDN_KEYS_MARK(25);
     solve_unit_lower<NTA>(Af, Tf, Xs, tid);
-    GDN_KEYS_MARK(26);
     // this thread's 16 entries of T, row i = tid / 4, columns (tid % 4) * 16 ..
     const int i = tid >> 2, qt = tid & 3;
     float tv[16];
@@ -388,7 +344,6 @@ __global__ void __launch_bounds__(NTA, 2)
         mma_f16(tmem + A_TM_D2, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
       mma_commit(bar_m2);
     }
-    GDN_KEYS_MARK(27);
     ok = mbar_wait(bar_m2, 0);
   }
   if (!__syncthreads_or(!ok)) {
@@ -425,10 +380,8 @@ __global__ void __launch_bounds__(NTA, 2)
         mma_f16(tmem + A_TM_D4, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
       mma_commit(bar_m3);
     }
-    GDN_KEYS_MARK(28);
     ok = mbar_wait(bar_m3, 0);
   }
-  GDN_KEYS_MARK(29);
   if (!__syncthreads_or(!ok)) {
     tc_fence_after();
     // The record is assembled in shared memory regions the MMAs no longer
@@ -489,7 +442,6 @@ __global__ void __launch_bounds__(NTA, 2)
     mbar_wait(bar_load, 0, 100000000ull);
     mbar_wait(bar_m3, 0, 100000000ull);
   }
-  GDN_KEYS_MARK(30);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -654,9 +606,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-#ifdef GDN_PHASE_TIMING
-  long long t_prev = clock64();
-#endif
   pdl_wait();  // the records, k and the start states come from the kernels before
 
   // thread LOADER streams K and the records: chunks 0 .. NST-1 up front, then
@@ -667,9 +616,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
     const int row = bos + cc * C;
     const uint32_t bar = bar_full + 8 * s, st = sb + s * G::STAGE;
     const uint8_t* rec = p.rec + ((size_t)(slot0 + cc) * p.Hv + h) * REC;
-#ifdef GDN_PHASE_TIMING
-    reinterpret_cast<long long*>(smem + G::BAR + 8 * (2 * NST + 9))[s] = clock64();
-#endif
     if constexpr (XFER) {
       // only the -W rows (the first 64 of each dk atom) and the U rows (the
       // first 64 of each value block); the MMA rows they leave stale are never read
@@ -717,14 +663,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
       const uint32_t st = sb + s * G::STAGE;
       const float* vec = reinterpret_cast<const float*>(stp + G::S_VEC);
       ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;
-#ifdef GDN_PHASE_TIMING
-      if (tid == 0) {  // cycles from the issue of this stage's copies to their arrival being seen
-        atomicAdd(&g_split_phase[14], (unsigned long long)(clock64() - reinterpret_cast<volatile long long*>(
-                                                                          smem + G::BAR + 8 * (2 * NST + 9))[s]));
-        atomicAdd(&g_split_phase[15], 1ull);
-      }
-#endif
-      GDN_SPLIT_PHASE(0);
       if (c > 0) ok = mbar_wait(bar_s + 8 * (b ^ 1), (uint32_t)((c - 1) >> 1) & 1u) && ok;
       tc_fence_after();
       // the stage of chunk c - 1 is free once its output rows have also read it:
@@ -734,7 +672,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         issue_loads(c - 1 + NST);
         loads_due = false;
       }
-      GDN_SPLIT_PHASE(1);
       {  // state -> fp16 operand, then S *= e^{gamma_L} in TMEM
         const float egL = vec[64];
         float r[CW];
@@ -749,7 +686,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
       fence_proxy_async();
       tc_fence_before();
       if (bar_named_or(BAR_COMPUTE, NCW, !ok)) { bad = true; break; }
-      GDN_SPLIT_PHASE(2);
       if (loads_due) {
         // the state MMAs of chunk c-1 are done; its O rows were read right after them
         const int cc = c - 1 + NST;
@@ -777,12 +713,10 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         __syncwarp();
         ok = go;
       }
-      GDN_SPLIT_PHASE(3);
       if (tl < 64) {
         // Vn = D + U, decayed to the chunk end -> B operand of the state update (over S16)
         ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
         tc_fence_after();
-        GDN_SPLIT_PHASE(4);
         float x[CW];
         tmem_ldw<CW>(lane_base + G::TM_D + b * VS + col, x);
         if (want_u) {
@@ -797,7 +731,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         fence_proxy_async();
         tc_fence_before();
         ok = !bar_named_or(BAR_VN, 256, !ok);
-        GDN_SPLIT_PHASE(5);
         if (warp == 0 && ok) {  // S^T += K^T Vts; with the O-row threads' arrivals the stage is free
           tc_fence_after();
           constexpr uint32_t id = idesc_f16(128, VS, true, true);
@@ -867,7 +800,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         ok = mbar_wait(bar_full + 8 * s, (uint32_t)(c / NST) & 1u) && ok;  // the stage's copies are seen here too
         ok = mbar_wait(bar_a + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
         tc_fence_after();
-        GDN_SPLIT_MARK(16);
 #pragma unroll 1
         for (int j0 = hc; j0 < hc + HV; j0 += 32) {
           float o[32];
@@ -890,7 +822,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
             if (og == 64) mbar_arrive_expect_tx(bar_x + 8 * b, 128 * 4);  // the other CTA's sums of this chunk
           }
         }
-        GDN_SPLIT_MARK(17);
       }
       if (norm_out) {
         cp_async_wait_all();
@@ -901,7 +832,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
             ok = mbar_wait_cluster(bar_x + 8 * b, (uint32_t)(c >> 1) & 1u) && ok;
             ss += xb[(b * 2) * 64 + t] + xb[(b * 2 + 1) * 64 + t];
           }
-          GDN_SPLIT_MARK(18);
           const float ri = rsqrtf(ss * (1.0f / D) + p.eps_norm);
 #pragma unroll 1
           for (int j0 = hc; j0 < hc + HV; j0 += 32) {
@@ -924,7 +854,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
           }
           tc_fence_before();
           mbar_arrive(bar_dfree + 8 * b);  // D[b] read for the last time
-          GDN_SPLIT_MARK(19);
         }
         if (bar_named_or(BAR_OG, NOG, !ok)) { ok = false; break; }  // the output tile is complete
         uint8_t* obase = reinterpret_cast<uint8_t*>(p.out) + ((size_t)c0 * p.Hv * D + h * D + vs * VS) * 2;
@@ -938,7 +867,6 @@ __global__ void __launch_bounds__(XFER ? NCW : NTB, 1)
         }
         // the next chunk's w * silu(z) over the chunks this thread just stored
         if (c + 1 < nchunks) z_copy(c + 1);
-        GDN_SPLIT_MARK(20);
       } else {
         if (orow) {
 #pragma unroll 1
@@ -1023,16 +951,12 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) bulk_load(dst + q * (D * D), M + q * (D * D / 4), D * D, bar);
   };
-#ifdef GDN_PHASE_TIMING
-  long long t_prev = clock64();
-#endif
   if (tid == 0) {
     mbar_init(mbar, 1);
     mbar_init(mbar + 8, 1);
     fence_mbar_init();
   }
   pdl_wait();  // the maps come from the transfer chains
-  GDN_SCAN_MARK(0);
   if (tid < P - 1 && nonempty(tid)) {  // every map and R slice this CTA will read, into L2
     if (tid > 0) bulk_prefetch_l2(map_of(tid), D * D * 4);
     bulk_prefetch_l2(map_of(tid) + hd + (size_t)r0 * D, SR * D * 4);
@@ -1055,7 +979,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       acc[r][1] = make_float2(v.z, v.w);
     }
   }
-  GDN_SCAN_MARK(1);
   for (int sg = 0;; ++sg) {
     if (owner) {
       float* dst = p.seg_start + (((size_t)n * P + sg) * p.Hv + h) * hd;
@@ -1097,7 +1020,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
     for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
     const int buf = j & 1;
     const uint32_t par = (uint32_t)(j >> 1) & 1u;
-    GDN_SCAN_MARK(2);
     if (__syncthreads_or(!mbar_wait(mbar + 8 * buf, par))) {
       // sT is complete but this segment's M never landed: record it, let the copy finish, stop
       if (tid == 0) {
@@ -1106,7 +1028,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       }
       break;
     }
-    GDN_SCAN_MARK(3);
     sg_next = next_map(sg + 1);
     if (tid == 0 && sg_next < P - 1) prefetch(sg_next, buf ^ 1);
     const float* M = Mb + buf * D * D;
@@ -1123,7 +1044,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
         acc[r][1] = __ffma2_rn(s2, m23, acc[r][1]);
       }
     }
-    GDN_SCAN_MARK(4);
     if (!owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
@@ -1132,7 +1052,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
           red[((ks * 16) + r * 4 + c) * SCAN_POS + pos] = (c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x;
     }
     __syncthreads();  // partial tiles written; everyone is done with sT and this buffer
-    GDN_SCAN_MARK(5);
     if (owner) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
@@ -1149,10 +1068,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) seg_scan_kernel(ChunkParams p) {
       }
     }
     ++j;
-    GDN_SCAN_MARK(6);
-#ifdef GDN_PHASE_TIMING
-    if (tid == 0) atomicAdd(&g_scan_phase[7], 1ull);
-#endif
     // the owners' reads of `red` end before its next write: two barriers
     // (the one above sT's completion and the one after the products) lie between
   }
@@ -1327,7 +1242,6 @@ __global__ void __launch_bounds__(FOLD_THREADS) state_fold_kernel(FoldParams p) 
   }
 }
 
-
 }  // namespace
 
 size_t chunk_tc_split_record_bytes(int N, int T, int Hv) {
@@ -1389,16 +1303,22 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
   ChunkParams p = p0;
   if (p.nseg < 1) p.nseg = 1;
   if (!p.rec) return cudaErrorInvalidValue;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mql, mkl;
   memset(&mq, 0, sizeof(mq));
   memset(&mk, 0, sizeof(mk));
   memset(&mv, 0, sizeof(mv));
+  memset(&mql, 0, sizeof(mql));
+  memset(&mkl, 0, sizeof(mkl));
+  if ((p.q_lo == nullptr) != (p.k_lo == nullptr)) return cudaErrorInvalidValue;
   if (p.T > 0) {
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_map(&mq, p.q, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
         !make_map(&mk, p.k, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
         !make_map(&mv, p.v, (uint64_t)p.T, (uint64_t)p.Hv * D, f16, sw))
+      return cudaErrorInvalidValue;
+    if (p.k_lo && (!make_map(&mql, p.q_lo, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw) ||
+                   !make_map(&mkl, p.k_lo, (uint64_t)p.T, (uint64_t)p.Hk * D, f16, sw)))
       return cudaErrorInvalidValue;
   }
   if (p.T > 0 && !p.reuse_records) {
@@ -1416,7 +1336,7 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, chunk_keys_kernel, mq, mk, mv, p);
+    e = cudaLaunchKernelEx(&cfg, chunk_keys_kernel, mq, mk, mv, mql, mkl, p);
     if (e != cudaSuccess) return e;
   }
   const int P = p.nseg;
@@ -1524,27 +1444,6 @@ int chunk_tc_split_auto_segments(int N, int T, int Hv) {
   }
   return best;
 }
-
-#ifdef GDN_PHASE_TIMING
-extern "C" int gdn_debug_phase_cycles_scan(unsigned long long* out, int clear) {
-  cudaDeviceSynchronize();
-  if (cudaMemcpyFromSymbol(out, g_scan_phase, sizeof(unsigned long long) * 8) != cudaSuccess) return -1;
-  if (clear) {
-    unsigned long long z[8] = {0};
-    cudaMemcpyToSymbol(g_scan_phase, z, sizeof(z));
-  }
-  return 0;
-}
-extern "C" int gdn_debug_phase_cycles_split(unsigned long long* out, int clear) {
-  cudaDeviceSynchronize();
-  if (cudaMemcpyFromSymbol(out, g_split_phase, sizeof(unsigned long long) * 32) != cudaSuccess) return -1;
-  if (clear) {
-    unsigned long long z[32] = {0};
-    cudaMemcpyToSymbol(g_split_phase, z, sizeof(z));
-  }
-  return 0;
-}
-#endif
 
 int split_error_word(int clear) {
   int v = 0;

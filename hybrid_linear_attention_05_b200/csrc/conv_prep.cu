@@ -56,6 +56,15 @@ template <> struct Raw8<float> {
   }
 };
 
+// Rounding residual of eight values stored as fp16: fp16(x - fp16(x)).
+__device__ __forceinline__ void store_lo8(__half* p, const float* f) {
+  float r[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = f[i] - __half2float(__float2half_rn(f[i]));
+  store8(p, r);
+}
+__device__ __forceinline__ void store_lo8(float*, const float*) {}  // fp32 intermediates: none
+
 template <typename T, typename TM, int D>
 __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
   constexpr int TPS = D / 8;  // threads per head segment
@@ -163,6 +172,8 @@ __global__ void __launch_bounds__(256) conv_prep_kernel(ConvPrepParams p) {
           TM* dst = static_cast<TM*>(is_q ? p.q : p.k);
           const int col = c0 - (is_q ? 0 : p.Hk * D);
           store8(dst + (size_t)t * p.Hk * D + col, y);
+          void* lo = is_q ? p.q_lo : p.k_lo;
+          if (lo) store_lo8(static_cast<TM*>(lo) + (size_t)t * p.Hk * D + col, y);
         }
       } else if (valid) {
         const int col = c0 - two_hk * D;
@@ -415,14 +426,30 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
       for (int q = 1; q < 4; ++q) a = __ffma2_rn(y[q], y[q], a);
       return a.x + a.y;
     };
+    void* const lo = is_qk ? (is_q ? p.q_lo : p.k_lo) : nullptr;
     auto store = [&](int t, const float2* y, float f) {
       uint4 u;
       __half2* h = reinterpret_cast<__half2*>(&u);
+      float2 x[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) h[q] = __float22half2_rn(__fmul2_rn(y[q], make_float2(f, f)));
-      __half* dst = is_qk ? static_cast<__half*>(is_q ? p.q : p.k) + (size_t)t * p.Hk * D + (c0 - (is_q ? 0 : p.Hk * D))
+      for (int q = 0; q < 4; ++q) {
+        x[q] = __fmul2_rn(y[q], make_float2(f, f));
+        h[q] = __float22half2_rn(x[q]);
+      }
+      const size_t qk_off = (size_t)t * p.Hk * D + (c0 - (is_q ? 0 : p.Hk * D));
+      __half* dst = is_qk ? static_cast<__half*>(is_q ? p.q : p.k) + qk_off
                           : static_cast<__half*>(p.v) + (size_t)t * p.Hv * D + (c0 - 2 * p.Hk * D);
       *reinterpret_cast<uint4*>(dst) = u;
+      if (lo) {  // rounding residuals of q and k: x - fp16(x), itself rounded to fp16
+        uint4 ul;
+        __half2* hl = reinterpret_cast<__half2*>(&ul);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 xh = __half22float2(h[q]);
+          hl[q] = __float22half2_rn(make_float2(x[q].x - xh.x, x[q].y - xh.y));
+        }
+        *reinterpret_cast<uint4*>(static_cast<__half*>(lo) + qk_off) = ul;
+      }
     };
     // two tokens at a time, so that their reductions and MUFU work overlap
 #pragma unroll

@@ -37,6 +37,8 @@ gdn_dtype mid_dtype(gdn_dtype in) { return in == GDN_BF16 ? GDN_F16 : GDN_F32; }
 
 struct Workspace {
   void* q; void* k; void* v; float* g; float* beta;
+  void* q_lo; void* k_lo;  // fp16 intermediates: rounding residuals of q and k (else null)
+  int* sched;              // chain queue of the fused tensor-core path
   uint8_t* rec;  // operand records of the two-kernel tensor-core path (or null)
   float* seg_mr;     // segment maps and start states of its segmented chain (or null)
   float* seg_start;
@@ -57,6 +59,13 @@ Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base, int N = -1) 
   w.v = p ? p + off : nullptr; off += nv;
   w.g = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
   w.beta = p ? reinterpret_cast<float*>(p + off) : nullptr; off += ng;
+  w.q_lo = w.k_lo = nullptr;
+  if (mid_dtype(dt) == GDN_F16) {
+    w.q_lo = p ? p + off : nullptr; off += nq;
+    w.k_lo = p ? p + off : nullptr; off += nq;
+  }
+  w.sched = p ? reinterpret_cast<int*>(p + off) : nullptr;
+  off += align_up(kFusedSchedBytes, 256);
   w.rec = nullptr;
   w.seg_mr = w.seg_start = nullptr;
   if (N >= 0) {
@@ -73,7 +82,7 @@ Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base, int N = -1) 
   return w;
 }
 
-enum class Path { None, Simt, Tc, TcSplit };
+enum class Path { None, Simt, Tc, TcSplit, TcFused };
 
 // `records` tells whether the workspace can hold the two-kernel path's records.
 Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records) {
@@ -82,6 +91,7 @@ Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records) 
   switch (impl) {
     case GDN_IMPL_TC: return tc ? Path::Tc : Path::None;
     case GDN_IMPL_TC_SPLIT: return tc ? Path::TcSplit : Path::None;
+    case GDN_IMPL_TC_FUSED: return tc ? Path::TcFused : Path::None;
     case GDN_IMPL_SIMT: return simt ? Path::Simt : Path::None;
     case GDN_IMPL_AUTO:
       return tc ? (records ? Path::TcSplit : Path::Tc) : (simt ? Path::Simt : Path::None);
@@ -152,8 +162,15 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   cp.A_log = a->A_log; cp.dt_bias = a->dt_bias; cp.cu_seqlens = a->cu_seqlens;
   cp.conv_state_in = a->conv_state_in; cp.conv_state_out = a->conv_state_out;
   cp.q = ws.q; cp.k = ws.k; cp.v = ws.v; cp.g = ws.g; cp.beta = ws.beta;
+  cp.q_lo = ws.q_lo; cp.k_lo = ws.k_lo;
   cp.T = a->T_tot; cp.N = a->N; cp.Hk = dims->Hk; cp.Hv = dims->Hv; cp.Cc = Cc;
   cp.scale = dims->scale; cp.eps_l2 = dims->eps_l2;
+  if (path == Path::TcFused) {  // the chain queue (reads only cu_seqlens), ahead of the conv
+    ChunkParams q{};
+    q.cu_seqlens = a->cu_seqlens; q.N = a->N; q.T = a->T_tot;
+    s = from_cuda(launch_chunk_fused_order(q, ws.sched, st));
+    if (s != GDN_OK) return s;
+  }
   if (!a->reuse_workspace) {
     s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
     if (s != GDN_OK) return s;
@@ -161,6 +178,7 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
 
   ChunkParams ch{};
   ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
+  ch.q_lo = ws.q_lo; ch.k_lo = ws.k_lo;
   ch.cu_seqlens = a->cu_seqlens; ch.S0 = a->initial_state; ch.S_out = a->final_state;
   ch.z = a->z; ch.norm_w = a->norm_w; ch.out = a->out; ch.o_raw = nullptr;
   ch.reuse_records = a->reuse_workspace;
@@ -176,6 +194,7 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   if (a->core_event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->core_event_begin), st) != cudaSuccess)
     return GDN_ERR_CUDA;
   s = from_cuda(path == Path::TcSplit ? launch_chunk_tc_split(ch, st)
+                : path == Path::TcFused ? launch_chunk_fused(ch, ws.sched, st)
                 : path == Path::Tc    ? launch_chunk_tc(ch, st)
                                       : launch_chunk_simt(ch, d, a->dtype, mid_dtype(a->dtype), st));
   if (s != GDN_OK) return s;
@@ -218,6 +237,7 @@ gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* a
   cp.A_log = a->A_log; cp.dt_bias = a->dt_bias; cp.cu_seqlens = a->cu_seqlens;
   cp.conv_state_in = a->conv_state_in; cp.conv_state_out = a->conv_state_out;
   cp.q = ws.q; cp.k = ws.k; cp.v = ws.v; cp.g = ws.g; cp.beta = ws.beta;
+  cp.q_lo = ws.q_lo; cp.k_lo = ws.k_lo;
   cp.T = a->T_tot; cp.N = a->N; cp.Hk = dims->Hk; cp.Hv = dims->Hv; cp.Cc = Cc;
   cp.scale = dims->scale; cp.eps_l2 = dims->eps_l2;
   s = from_cuda(launch_conv_prep(cp, d, a->dtype, st));
@@ -225,6 +245,7 @@ gdn_status gdn_prefill_state_map(const gdn_dims* dims, const gdn_prefill_args* a
 
   ChunkParams ch{};
   ch.q = ws.q; ch.k = ws.k; ch.v = ws.v; ch.g = ws.g; ch.beta = ws.beta;
+  ch.q_lo = ws.q_lo; ch.k_lo = ws.k_lo;
   ch.cu_seqlens = a->cu_seqlens; ch.S0 = nullptr; ch.S_out = nullptr;
   ch.z = a->T_tot > 0 ? a->z : nullptr; ch.norm_w = a->norm_w; ch.out = nullptr; ch.o_raw = nullptr;
   ch.T = a->T_tot; ch.N = a->N; ch.Hk = dims->Hk; ch.Hv = dims->Hv; ch.chunk = a->chunk;
@@ -302,9 +323,11 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
-  // no workspace here, hence no two-kernel path
+  // no record workspace here, hence no two-kernel path
   const Path path = a->impl == GDN_IMPL_TC_SPLIT ? Path::None : pick_path(a->impl, d, a->chunk, a->dtype, false);
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
+  if (path == Path::TcFused && (!a->workspace || a->workspace_bytes < kFusedSchedBytes)) return GDN_ERR_WORKSPACE;
+  if (!aligned16(a->workspace)) return GDN_ERR_ALIGN;
   if (!a->cu_seqlens) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o)) return GDN_ERR_NULL;
   const void* ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
@@ -322,9 +345,17 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   ch.eps_norm = dims->eps_norm;
   ch.nseg = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (path == Path::TcFused) {
+    int* sched = static_cast<int*>(a->workspace);
+    s = from_cuda(launch_chunk_fused_order(ch, sched, st));
+    if (s != GDN_OK) return s;
+    return from_cuda(launch_chunk_fused(ch, sched, st));
+  }
   return from_cuda(path == Path::Tc ? launch_chunk_tc(ch, st)
                                     : launch_chunk_simt(ch, d, GDN_F32, a->dtype, st));
 }
+
+size_t gdn_core_workspace_size(int N) { return N < 0 ? 0 : kFusedSchedBytes; }
 
 const char* gdn_status_string(gdn_status s) {
   switch (s) {
@@ -336,6 +367,7 @@ const char* gdn_status_string(gdn_status s) {
     case GDN_ERR_CUDA: return "a CUDA call failed";
     case GDN_ERR_WORKSPACE: return "workspace missing or too small";
     case GDN_ERR_ALIAS: return "buffers that must not overlap overlap";
+    case GDN_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
   }
   return "unknown status";
 }

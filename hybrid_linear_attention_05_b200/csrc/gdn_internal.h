@@ -25,6 +25,11 @@ struct ConvPrepParams {
   void* q;                    // [T, Hk, d]  fp16 (bf16 inputs) or fp32
   void* k;                    // [T, Hk, d]
   void* v;                    // [T, Hv, d]
+  // fp16 intermediates only: the rounding residuals of q and k,
+  // q_lo = fp16(q - fp16(q)), so that q + q_lo carries about 22 significand
+  // bits into the K K^T and Q K^T products (null: not written)
+  void* q_lo;                 // [T, Hk, d]
+  void* k_lo;                 // [T, Hk, d]
   float* g;                   // [Hv, T]
   float* beta;                // [Hv, T]
   int T, N, Hk, Hv, Cc;
@@ -39,6 +44,10 @@ struct ChunkParams {
   const void* q;              // [T, Hk, d]
   const void* k;              // [T, Hk, d]
   const void* v;              // [T, Hv, d]
+  // residuals of fp16 q and k (see ConvPrepParams), or null: the tensor-core
+  // kernels then form K K^T and Q K^T from the fp16 values alone
+  const void* q_lo;           // [T, Hk, d]
+  const void* k_lo;           // [T, Hk, d]
   const float* g;             // [Hv, T]
   const float* beta;          // [Hv, T]
   const int32_t* cu_seqlens;  // [N+1]
@@ -98,6 +107,17 @@ int split_error_word(int clear);  // host: read (and clear) that path's device e
 // Segments of the state-map mode for N sequences of Hv heads (1 when the
 // segment buffers do not exist for these sizes).
 int chunk_tc_split_map_segments(int N, int Hv);
+
+// chunk_fused.cu: the same core as one persistent warp-specialised kernel.
+// `sched` is kFusedSchedBytes of workspace: the chain counter and the queue
+// order of up to kFusedSortMax sequences, written by
+// launch_chunk_fused_order, which must run first on the stream (it reads
+// only cu_seqlens).
+constexpr int kFusedSortMax = 1024;
+constexpr size_t kFusedSchedBytes = (1 + kFusedSortMax) * sizeof(int);
+cudaError_t launch_chunk_fused_order(const ChunkParams& p, int* sched, cudaStream_t st);
+cudaError_t launch_chunk_fused(const ChunkParams& p, int* sched, cudaStream_t st);
+int fused_error_word(int clear);  // host: read (and clear) that kernel's device error word
 
 // Affine fold, d = 128: for every (sequence n, head h), the rows X (rows x d,
 // fp32) start from x0 (zeros when null) and go through the maps s = 0 ..

@@ -13,31 +13,73 @@
 
 #include <atomic>
 
+#include <cuda.h>
+
 #include "gdn_internal.h"
 
 namespace {
 
-// The scratch itself.  Every device that loads this library holds it (64 MiB)
-// until the process exits.  In host code this name is only a host-side
-// stand-in for the symbol: its device address comes from
-// cudaGetSymbolAddress, once per device (scratch_on_current_device).
+// The scratch itself (64 MiB per device, held until the process exits).
+// With CUDA's lazy module loading (the default) the device memory behind it is
+// committed when this module is first loaded on a device, which is the first
+// gdn_prefill_noalloc call there (its cudaGetSymbolAddress).  In host code
+// this name is only a host-side stand-in for the symbol: its device address
+// comes from cudaGetSymbolAddress (scratch_on_current_device).
 __device__ __align__(256) unsigned char g_gdn_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the scratch on the current device, looked up on the first
-// call for that device and cached.  Returns nullptr if the lookup fails.
+// Process-unique id of the current CUDA context (0 when there is none or it
+// cannot be read).  A context made after cudaDeviceReset gets a new id.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || qb != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+constexpr int kMaxDevices = 64;
+struct CachedAddress {
+  std::atomic<unsigned long long> ctx_id{0};
+  std::atomic<void*> addr{nullptr};
+};
+CachedAddress g_scratch[kMaxDevices];
+
+// Device address of the scratch on the current device.  It is looked up with
+// cudaGetSymbolAddress on the first call for that device and cached together
+// with the id of the context it belongs to; a call in a different context (the
+// device was reset with cudaDeviceReset since) looks it up again.  Returns
+// nullptr if the lookup fails.
 void* scratch_on_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+  const unsigned long long id = current_context_id();
+  void* p = g_scratch[dev].addr.load(std::memory_order_acquire);
+  if (p && id != 0 && g_scratch[dev].ctx_id.load(std::memory_order_acquire) == id) return p;
+  p = nullptr;
   if (cudaGetSymbolAddress(&p, g_gdn_noalloc_scratch) != cudaSuccess || p == nullptr) {
     cudaGetLastError();  // do not leave this error for an unrelated later call to find
     return nullptr;
   }
-  g_scratch_addr[dev].store(p, std::memory_order_release);
+  // the lookup created the context if there was none: take its id now
+  g_scratch[dev].ctx_id.store(id != 0 ? id : current_context_id(), std::memory_order_release);
+  g_scratch[dev].addr.store(p, std::memory_order_release);
   return p;
 }
 

@@ -19,13 +19,24 @@ __device__ __forceinline__ void st_half8(uint8_t* base, uint32_t off, const floa
   *reinterpret_cast<uint4*>(base + off) = u;
 }
 
+// Barrier over the NT threads that run a shared step: the whole CTA
+// (BAR == 0), or named barrier BAR when those threads are one role of a
+// larger CTA.
+template <int NT, int BAR>
+__device__ __forceinline__ void role_sync() {
+  if constexpr (BAR == 0)
+    __syncthreads();
+  else
+    asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
 // Tf := (I + A)^-1 for the strictly lower triangular 64 x 64 A (fp32, row
 // stride AS), by recursive doubling of the block size:
 //   16 x 16 diagonal blocks by forward substitution (one column per thread);
 //   32 x 32: T_{r,r-1} = -T_rr A_{r,r-1} T_{r-1,r-1} for the 16-blocks (1,0), (3,2);
 //   64 x 64: T_{LL}   = -T_bb A_{LL} T_tt for the lower-left 32-block.
 // Every product step gives each thread independent accumulators.
-template <int NT>
+template <int NT, int BAR = 0>
 __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, float* X, int tid) {
   constexpr int NW = NT / 32;
   const int warp = tid >> 5, lane = tid & 31;
@@ -53,7 +64,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
       Tf[(16 * r + i) * AS + 16 * c + m] = 0.f;
     }
   }
-  __syncthreads();
+  role_sync<NT, BAR>();
   // 32 x 32 diagonal blocks: element e = tid + NT k -> 16-block (r, r-1), r = 1 or 3
   constexpr int K1 = 512 / NT;
   {
@@ -72,7 +83,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
 #pragma unroll
     for (int k = 0; k < K1; ++k) X[tid + NT * k] = acc[k];
   }
-  __syncthreads();
+  role_sync<NT, BAR>();
   {
     float acc[K1];
 #pragma unroll
@@ -91,7 +102,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
       Tf[(16 * r + i) * AS + 16 * (r - 1) + m] = -acc[k];
     }
   }
-  __syncthreads();
+  role_sync<NT, BAR>();
   // 64 x 64: rows 32 + warp + NW k of the lower-left block, column `lane`
   constexpr int K2 = 32 / NW;
   {
@@ -112,7 +123,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
 #pragma unroll
     for (int k = 0; k < K2; ++k) X[(warp + NW * k) * 32 + lane] = acc[k];
   }
-  __syncthreads();
+  role_sync<NT, BAR>();
   {
     float acc[K2];
 #pragma unroll
@@ -131,7 +142,7 @@ __device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, flo
 #pragma unroll
     for (int k = 0; k < K2; ++k) Tf[(32 + warp + NW * k) * AS + lane] = -acc[k];
   }
-  __syncthreads();
+  role_sync<NT, BAR>();
 }
 
 

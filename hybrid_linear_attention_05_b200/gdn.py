@@ -23,6 +23,7 @@ GDN_ERR_UNSUPPORTED = -4
 GDN_ERR_CUDA = -5
 GDN_ERR_WORKSPACE = -6
 GDN_ERR_ALIAS = -7
+GDN_ERR_TIMEOUT = -8
 
 GDN_F32 = 0
 GDN_BF16 = 1
@@ -32,11 +33,12 @@ GDN_IMPL_AUTO = 0
 GDN_IMPL_SIMT = 1
 GDN_IMPL_TC = 2
 GDN_IMPL_TC_SPLIT = 3
+GDN_IMPL_TC_FUSED = 4
 
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
             "gdn_prefill_auto_segments", "gdn_prefill_noalloc", "gdn_prefill_state_map",
-            "gdn_state_fold", "gdn_decode", "gdn_chunk_core",
-            "gdn_device_error", "gdn_status_string", "gdn_version"]
+            "gdn_state_fold", "gdn_decode", "gdn_chunk_core", "gdn_core_workspace_size",
+            "gdn_device_error", "gdn_selftest_bounded_wait", "gdn_status_string", "gdn_version"]
 
 # Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
 GDN_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -73,7 +75,8 @@ class gdn_core_args(ctypes.Structure):
     _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp),
                 ("cu_seqlens", _vp), ("N", ctypes.c_int), ("T_tot", ctypes.c_int),
                 ("chunk", ctypes.c_int), ("dtype", ctypes.c_int), ("impl", ctypes.c_int),
-                ("initial_state", _vp), ("final_state", _vp), ("o", _vp)]
+                ("initial_state", _vp), ("final_state", _vp), ("o", _vp), ("workspace", _vp),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -109,8 +112,12 @@ def lib():
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_chunk_core.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_core_args), _vp]
         L.gdn_chunk_core.restype = ctypes.c_int
+        L.gdn_core_workspace_size.argtypes = [ctypes.c_int]
+        L.gdn_core_workspace_size.restype = ctypes.c_size_t
         L.gdn_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
         L.gdn_device_error.restype = ctypes.c_int
+        L.gdn_selftest_bounded_wait.argtypes = [ctypes.c_int, _vp]
+        L.gdn_selftest_bounded_wait.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_version.argtypes = []
@@ -246,12 +253,16 @@ def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, no
                   raise_on_error)
 
 
+def gdn_core_workspace_size(N: int) -> int:
+    return int(lib().gdn_core_workspace_size(int(N)))
+
+
 def gdn_chunk_core(dims: gdn_dims, *, q, k, v, g, beta, cu_seqlens, N, T_tot, chunk, dtype, o,
-                   initial_state=None, final_state=None, impl=GDN_IMPL_AUTO, stream=None,
-                   raise_on_error=True) -> int:
+                   initial_state=None, final_state=None, impl=GDN_IMPL_AUTO, workspace=None,
+                   workspace_bytes=0, stream=None, raise_on_error=True) -> int:
     args = gdn_core_args(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(cu_seqlens), int(N),
                          int(T_tot), int(chunk), int(dtype), int(impl), ptr(initial_state),
-                         ptr(final_state), ptr(o))
+                         ptr(final_state), ptr(o), ptr(workspace), int(workspace_bytes))
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_chunk_core(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_chunk_core", raise_on_error)
@@ -262,6 +273,13 @@ def gdn_device_error(clear: bool = True) -> int:
     code = ctypes.c_int(0)
     _check(lib().gdn_device_error(ctypes.byref(code), int(clear)), "gdn_device_error", True)
     return code.value
+
+
+def gdn_selftest_bounded_wait(limit_us: int, stream=None, raise_on_error=True) -> int:
+    """Launch the failure-path test kernel (gdn.h): a bounded wait that gives up."""
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_selftest_bounded_wait(int(limit_us), s), "gdn_selftest_bounded_wait",
+                  raise_on_error)
 
 
 def gdn_version() -> str:

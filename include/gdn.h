@@ -72,7 +72,10 @@ typedef enum {
   GDN_ERR_UNSUPPORTED = -4, /* valid, but not a shape this build supports       */
   GDN_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed (launch, ...)  */
   GDN_ERR_WORKSPACE = -6,   /* workspace missing or smaller than required       */
-  GDN_ERR_ALIAS = -7        /* buffers that must not overlap do overlap         */
+  GDN_ERR_ALIAS = -7,       /* buffers that must not overlap do overlap         */
+  GDN_ERR_TIMEOUT = -8      /* a bounded wait inside a kernel gave up; reported
+                               after the fact by gdn_device_error, since kernels
+                               run asynchronously to the call that launched them */
 } gdn_status;
 
 /* Element types.  gdn_prefill / gdn_decode take GDN_F32 or GDN_BF16 inputs;
@@ -87,11 +90,17 @@ typedef enum {
   GDN_IMPL_TC = 2,     /* tcgen05 tensor-core chunked core, one kernel per call
                           (bf16 inputs, fp16 operands, d = 128, chunk 64);
                           GDN_ERR_UNSUPPORTED otherwise                       */
-  GDN_IMPL_TC_SPLIT = 3 /* the same tensor-core core as two kernels: the
+  GDN_IMPL_TC_SPLIT = 3, /* the same tensor-core core as two kernels: the
                           state-independent key-side work of every (chunk,
                           head) first, over all SMs, then the per-head state
                           chain.  Needs gdn_prefill_workspace_size_n bytes
                           of workspace (GDN_ERR_WORKSPACE otherwise).         */
+  GDN_IMPL_TC_FUSED = 4 /* the same tensor-core core as one persistent kernel
+                          per SM: warps that do the key-side work of the next
+                          chunk run beside the warps that carry the state, so
+                          nothing passes through HBM between them; (sequence,
+                          value head) chains are taken longest first.  Needs
+                          only gdn_prefill_workspace_size bytes.            */
 } gdn_impl;
 
 /* Layer shape.  Supported: dk == dv in {32, 64, 128}; Hv % Hk == 0;
@@ -251,18 +260,28 @@ gdn_status gdn_state_fold(const gdn_dims* dims, int N, int count, const float* m
  *
  * gdn_prefill_noalloc runs gdn_prefill with its workspace taken from one
  * fixed scratch array inside the library (GDN_NOALLOC_SCRATCH_BYTES of device
- * memory, held on every device that loads the library until the process
- * exits).  It allocates nothing.
+ * memory, held on every device that uses it until the process exits).  It
+ * allocates nothing.
  *   - args->workspace and args->workspace_bytes are ignored; every other
  *     argument means what it means for gdn_prefill, with the same checks,
  *     except reuse_workspace, which must be 0 (GDN_ERR_UNSUPPORTED).
  *   - Returns GDN_ERR_WORKSPACE, launching nothing, when the workspace these
  *     sizes need (gdn_prefill_workspace_size) exceeds
- *     GDN_NOALLOC_SCRATCH_BYTES -- about 5400 tokens at 16 key / 16 value
+ *     GDN_NOALLOC_SCRATCH_BYTES -- about 3200 tokens at 16 key / 16 value
  *     heads of width 128, bf16.
+ *   - With impl GDN_IMPL_AUTO the call takes the path gdn_prefill would take
+ *     with a workspace of GDN_NOALLOC_SCRATCH_BYTES: a batch whose two-kernel
+ *     records (gdn_prefill_workspace_size_n) do not fit in the scratch runs
+ *     on a path that needs none.
+ *   - Under CUDA's lazy module loading (the default) the scratch's device
+ *     memory is committed on the first call on each device.  A runtime that
+ *     divides up device memory in advance should make one call (any size,
+ *     e.g. one sequence of one token) before it does so.
  *   - The first call on a device looks up the scratch's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call outside any
- *     CUDA stream capture.  GDN_ERR_CUDA if the lookup fails.
+ *     (cudaGetSymbolAddress) and caches it with the id of the current CUDA
+ *     context; a call in a new context (after cudaDeviceReset) looks it up
+ *     again.  Make the first call on a device, and the first after a reset,
+ *     outside any CUDA stream capture.  GDN_ERR_CUDA if the lookup fails.
  *   - All calls share the one scratch array, which keeps the previous call's
  *     contents (nothing in it needs to start at zero).  Calls whose work may
  *     overlap on the GPU -- on different streams, or from host threads that
@@ -335,16 +354,32 @@ typedef struct {
   const float* initial_state;
   float* final_state;
   float* o;
+  void* workspace;             /* device scratch of gdn_core_workspace_size bytes
+                                  (GDN_IMPL_TC_FUSED only; may be NULL otherwise) */
+  size_t workspace_bytes;
 } gdn_core_args;
+
+/* Bytes of workspace gdn_chunk_core needs for N sequences (the chain queue of
+ * GDN_IMPL_TC_FUSED). */
+size_t gdn_core_workspace_size(int N);
 
 gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* args, void* stream);
 
-/* Error word of the tensor-core kernels.  Their internal waits (on TMA and
- * tensor-core completion) are bounded; one that gives up records a nonzero
- * code here and the kernel returns instead of hanging.  This call
- * synchronises the current device, stores the code in *code (0 = none) and
- * clears it when clear != 0. */
+/* Error word of the kernels.  Their internal waits (on TMA copies, on
+ * tensor-core completion, on the other CTA of a cluster, between the roles of
+ * a warp-specialised kernel) are bounded; one that gives up records it here,
+ * lets the copies and tensor-core work it started land (bounded again), frees
+ * its TMEM and returns instead of hanging.  This call synchronises the current
+ * device, stores GDN_ERR_TIMEOUT in *code if any wait gave up since the word
+ * was last cleared (0 otherwise), and clears the word when clear != 0. */
 gdn_status gdn_device_error(int* code, int clear);
+
+/* Test of that failure path, with no counterpart on the pages: launches on
+ * `stream` one warp that waits, through the same bounded wait the kernels
+ * use, on an mbarrier nothing ever arrives at, gives up after limit_us
+ * microseconds (1 .. 1000000; GDN_ERR_DIMS otherwise) and records the
+ * timeout in the error word.  Nothing else is in flight in that kernel. */
+gdn_status gdn_selftest_bounded_wait(int limit_us, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* gdn_status_string(gdn_status status);

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_status_strings(L):
     assert gdn.gdn_version().startswith("gdn-b200")
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         assert gdn.status_string(code) not in ("", "unknown status")
     assert gdn.status_string(-99) == "unknown status"
 
@@ -47,8 +47,11 @@ def test_workspace_size():
     dims = gdn.make_dims(16, 32, 128)
     T = 1000
     n = gdn.gdn_prefill_workspace_size(dims, T, gdn.GDN_BF16)
-    raw = T * (2 * 16 * 128 * 2 + 32 * 128 * 2 + 2 * 32 * 4)
-    assert raw <= n <= raw + 5 * 256
+    # fp16 q, k, v, the fp32 gates, the fp16 rounding residuals of q and k, and
+    # the chain queue of the fused path (a counter and the order of up to 1024
+    # sequences)
+    raw = T * (2 * 16 * 128 * 2 + 32 * 128 * 2 + 2 * 32 * 4 + 2 * 16 * 128 * 2) + 4 * 1025
+    assert raw <= n <= raw + 8 * 256
     assert gdn.gdn_prefill_workspace_size(dims, T, gdn.GDN_F32) > n
     assert gdn.gdn_prefill_workspace_size(gdn.make_dims(3, 4, 128), T, gdn.GDN_BF16) == 0
     assert gdn.gdn_prefill_workspace_size(dims, -1, gdn.GDN_BF16) == 0
@@ -227,3 +230,10 @@ def test_state_map_gate_inputs_both_or_neither(L):
     dims = gdn.make_dims(2, 4, 128)
     assert gdn.gdn_prefill_state_map(dims, **map_kwargs(z=FAKE)) == gdn.GDN_ERR_NULL
     assert gdn.gdn_prefill_state_map(dims, **map_kwargs(norm_w=FAKE)) == gdn.GDN_ERR_NULL
+
+
+def test_selftest_rejects_limits_before_launching(L):
+    """The failure-path test kernel checks its limit on the host (no GPU
+    needed): outside 1 .. 1e6 microseconds nothing is launched."""
+    for bad in (0, -5, 1000001):
+        assert gdn.gdn_selftest_bounded_wait(bad, stream=0, raise_on_error=False) == gdn.GDN_ERR_DIMS

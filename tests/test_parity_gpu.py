@@ -6,6 +6,8 @@ tensor-core operands, fp32 accumulation; the CUDA-core kernel is held to the
 same bar), 1e-4 for the fp32 decode step (state exactly; bf16 outputs after
 allowing their own rounding).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -36,7 +38,7 @@ D9B = WORKLOADS["decode_B256_Hk16_Hv32_d128"]
 P397 = WORKLOADS["prefill_varlen8_T65536_Hk16_Hv64_d128"]
 
 IMPLS = {"simt": (gdn.GDN_IMPL_SIMT, 32), "tc": (gdn.GDN_IMPL_TC, 64),
-         "split": (gdn.GDN_IMPL_TC_SPLIT, 64)}
+         "split": (gdn.GDN_IMPL_TC_SPLIT, 64), "fused": (gdn.GDN_IMPL_TC_FUSED, 64)}
 # A_log range of a slow decay (alpha ~ 0.995-0.9995 per token): the workloads'
 # own U(0, ln 16) decays the state by e^-45 or more per 64-token chunk, so only
 # slow-decay cases show whether the state is carried right across chunks
@@ -108,7 +110,7 @@ def test_simt_small_heads(chunk, d):
     check_full(inp, bufs)
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split", "fused"])
 def test_qwen08b_shapes_ragged(impl):
     """16/16 heads of width 128 over several chunks with a ragged tail."""
     code, chunk = IMPLS[impl]
@@ -117,7 +119,7 @@ def test_qwen08b_shapes_ragged(impl):
     check_full(inp, bufs)
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split", "fused"])
 def test_9b_shapes_gqa_varlen(impl):
     """16 key / 32 value heads, nonzero initial states, conv history,
     sequences of lengths 1, 2, 3, 64 and one spanning several chunks."""
@@ -176,7 +178,8 @@ def test_split_segments_agree_with_serial_chain():
         assert relerr(S, outs[0][1]) <= PREFILL_TOL
 
 
-@pytest.mark.parametrize("impl,segments", [("tc", 0), ("split", 1), ("split", 4), ("split", 8)])
+@pytest.mark.parametrize("impl,segments", [("tc", 0), ("split", 1), ("split", 4), ("split", 8),
+                                           ("fused", 0)])
 def test_slow_decay_state_carry(impl, segments):
     """Slow decay (exp(A_log) ~ 1e-3, alpha near 1) so that the state written
     in early chunks still shapes the outputs and the final state many chunks
@@ -211,7 +214,7 @@ def test_split_segments_in_place_state():
     assert relerr(np64(bufs.out), ref.out) <= PREFILL_TOL
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc", "split"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "split", "fused"])
 def test_397b_shapes_varlen(impl):
     code, chunk = IMPLS[impl]
     inp = make_prefill(P397, seqlens=(65, 130, 7, 64))
@@ -240,6 +243,15 @@ def test_in_place_state_update():
 
 # ------------------------------------------------------- full-size workloads
 
+_INPUTS = {}
+
+
+def workload_inputs(name):
+    """The full workload, drawn once per test session (cfg 4 takes ~20 s)."""
+    if name not in _INPUTS:
+        _INPUTS[name] = make_prefill(WORKLOADS[name])
+    return _INPUTS[name]
+
 
 def sampled_check(inp, bufs, pairs):
     worst = 0.0
@@ -253,22 +265,97 @@ def sampled_check(inp, bufs, pairs):
     return worst
 
 
-@pytest.mark.parametrize("name,pairs", [
-    ("prefill_T4096_Hk16_Hv16_d128", [(0, 0), (0, 7), (0, 15)]),
-    ("prefill_4x8192_Hk16_Hv32_d128", [(0, 0), (1, 13), (3, 31)]),
-    ("prefill_varlen8_T65536_Hk16_Hv64_d128", [(0, 0), (3, 21), (7, 63)]),
-])
-@pytest.mark.parametrize("impl", ["auto", "tc"])
-def test_full_size_sampled(name, pairs, impl):
-    """Full benchmark sizes in the benchmark's launch configuration (AUTO:
-    the two-kernel tensor-core path), and the single-kernel path; the oracle
-    recomputes a few (sequence, value head) pairs on their own."""
-    w = WORKLOADS[name]
-    inp = make_prefill(w)
-    code = gdn.GDN_IMPL_AUTO if impl == "auto" else gdn.GDN_IMPL_TC
-    bufs = run_prefill(inp, code, w.chunk, guard=False)
-    sampled_check(inp, bufs, pairs)
+# Value heads checked at full size: the first and the last head of four GQA
+# groups (key heads 0, 7, 8 and 15), in every sequence.
+SAMPLED_HEADS = {
+    "prefill_4x8192_Hk16_Hv32_d128": [0, 1, 14, 15, 16, 17, 30, 31],
+    "prefill_varlen8_T65536_Hk16_Hv64_d128": [0, 3, 28, 31, 32, 35, 60, 63],
+}
+
+
+def heads_check(inp, bufs, heads):
+    """Every sequence, the given value heads: one multithreaded oracle run on
+    the sub-layer made of those heads and the key heads they read (the mixer
+    is separable over value heads, so its rows equal the full problem's)."""
+    w = inp.w
+    G, d = w.Hv // w.Hk, w.d
+    kheads = sorted({h // G for h in heads})
+    assert all(heads[2 * i] // G == heads[2 * i + 1] // G == kheads[i] for i in range(len(kheads)))
+    q_cols = np.concatenate([np.arange(kh * d, (kh + 1) * d) for kh in kheads])
+    v_cols = np.concatenate([2 * w.Hk * d + np.arange(h * d, (h + 1) * d) for h in heads])
+    cols = np.concatenate([q_cols, w.Hk * d + q_cols, v_cols])
+    zc = np.concatenate([np.arange(h * d, (h + 1) * d) for h in heads])
+    ref = oracle.prefill(
+        len(kheads), len(heads), d, d, inp.cu_seqlens, inp.mixed_qkv[:, cols], inp.conv_w[cols],
+        inp.a[:, heads], inp.b[:, heads], inp.A_log[heads], inp.dt_bias[heads], inp.z[:, zc],
+        inp.norm_w, None if inp.initial_state is None else inp.initial_state[:, heads],
+        None if inp.conv_state_in is None else inp.conv_state_in[:, cols], scale=w.scale)
+    e_out = relerr(np64(bufs.out[:, heads]), ref.out)
+    e_S = relerr(np64(bufs.final_state[:, heads]), ref.final_state)
+    np.testing.assert_array_equal(np64(bufs.conv_state_out[:, cols]), ref.conv_state_out)
+    assert e_out <= PREFILL_TOL and e_S <= PREFILL_TOL, (e_out, e_S)
+    return e_out, e_S
+
+
+@pytest.mark.parametrize("impl", ["auto", "tc", "fused"])
+def test_full_size_08b_every_head(impl):
+    """The 0.8B-shaped workload (4096 tokens, 16/16 heads) at full size in the
+    benchmark's launch configuration (AUTO) and on the single-kernel path:
+    every output, the final state and the conv tail against the oracle."""
+    inp = workload_inputs("prefill_T4096_Hk16_Hv16_d128")
+    code = gdn.GDN_IMPL_AUTO if impl == "auto" else IMPLS[impl][0]
+    bufs = run_prefill(inp, code, 64, guard=False)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("name", list(SAMPLED_HEADS))
+@pytest.mark.parametrize("impl", ["auto", "tc", "split", "fused"])
+def test_full_size_sampled(name, impl):
+    """The 9B- and 397B-shaped workloads at full size in the benchmark's
+    launch configuration (AUTO), and on the single-kernel path: every
+    sequence, eight value heads (first and last of four GQA groups)."""
+    inp = workload_inputs(name)
+    code = gdn.GDN_IMPL_AUTO if impl == "auto" else IMPLS[impl][0]
+    bufs = run_prefill(inp, code, 64, guard=False)
+    heads_check(inp, bufs, SAMPLED_HEADS[name])
     assert torch.isfinite(bufs.out.float()).all()
+
+
+# The statement of the method writes o_t = S_t q_t with no factor on q: these
+# cases run the whole mixer at q scale 1, where the gated RMSNorm passes the
+# relative error of every token's o straight to its output (at dk^-1/2 the
+# norm's eps damps it for the smallest outputs).
+@pytest.mark.parametrize("impl", ["simt", "tc", "split", "fused"])
+@pytest.mark.parametrize("name,seqlens", [
+    ("prefill_T4096_Hk16_Hv16_d128", (1024,)),
+    ("prefill_4x8192_Hk16_Hv32_d128", (700, 333, 1, 64)),
+    ("prefill_varlen8_T65536_Hk16_Hv64_d128", (400, 90, 257)),
+])
+def test_unit_q_scale(impl, name, seqlens):
+    w = resized(WORKLOADS[name], q_scale=1.0)
+    inp = make_prefill(w, seqlens=seqlens, with_conv_state=True)
+    code, chunk = IMPLS[impl]
+    bufs = run_prefill(inp, code, chunk)
+    check_full(inp, bufs)
+
+
+def test_unit_q_scale_08b_full_size():
+    """The full 0.8B-shaped workload at q scale 1 in the benchmark's launch
+    configuration: every output against the oracle."""
+    base = workload_inputs("prefill_T4096_Hk16_Hv16_d128")
+    inp = dataclasses.replace(base, w=resized(base.w, q_scale=1.0))  # same draws, scale 1
+    bufs = run_prefill(inp, gdn.GDN_IMPL_AUTO, 64, guard=False)
+    check_full(inp, bufs)
+
+
+@pytest.mark.parametrize("name", list(SAMPLED_HEADS))
+def test_unit_q_scale_full_size_sampled(name):
+    """The 9B- and 397B-shaped workloads at q scale 1, full size, AUTO:
+    every sequence, eight value heads."""
+    base = workload_inputs(name)
+    inp = dataclasses.replace(base, w=resized(base.w, q_scale=1.0))  # same draws, scale 1
+    bufs = run_prefill(inp, gdn.GDN_IMPL_AUTO, 64, guard=False)
+    heads_check(inp, bufs, SAMPLED_HEADS[name])
 
 
 # ------------------------------------------------------------------- decode
@@ -433,12 +520,13 @@ def run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, impl, S0=None, dtype=torch.
     t = lambda x, dt=dtype: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev, dt)
     o = torch.empty((T, Hv, d), dtype=torch.float32, device=dev)
     S = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.gdn_core_workspace_size(N), dtype=torch.uint8, device=dev)
     status = gdn.gdn_chunk_core(
         gdn.make_dims(Hk, Hv, d, scale=1.0), q=t(q), k=t(k), v=t(v),
         g=t(np.ascontiguousarray(g.T), torch.float32), beta=t(np.ascontiguousarray(beta.T), torch.float32),
         cu_seqlens=torch.tensor(cu, dtype=torch.int32, device=dev), N=N, T_tot=T, chunk=chunk,
         dtype=gdn.dtype_code(t(q)), o=o, initial_state=None if S0 is None else t(S0, torch.float32),
-        final_state=S, impl=impl, raise_on_error=False)
+        final_state=S, impl=impl, workspace=ws, workspace_bytes=ws.numel(), raise_on_error=False)
     if status == gdn.GDN_ERR_UNSUPPORTED:
         pytest.skip("implementation not available for this shape")
     assert status == gdn.GDN_OK
@@ -448,7 +536,7 @@ def run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, impl, S0=None, dtype=torch.
 
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
     ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.float32),
-    ("tc", 128, 64, torch.float16)])
+    ("tc", 128, 64, torch.float16), ("fused", 128, 64, torch.float16)])
 def test_core_orthonormal_overwrite(impl, d, chunk, dtype):
     """alpha = 1, beta = 1, orthonormal keys: S k_i = v_i after writing, and
     a rewritten key returns its new value (exact in real arithmetic)."""
@@ -478,7 +566,8 @@ def test_core_orthonormal_overwrite(impl, d, chunk, dtype):
 
 
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
-    ("simt", 64, 32, torch.float32), ("tc", 128, 64, torch.float16)])
+    ("simt", 64, 32, torch.float32), ("tc", 128, 64, torch.float16),
+    ("fused", 128, 64, torch.float16)])
 def test_core_beta_zero_only_decays(impl, d, chunk, dtype):
     code = IMPLS[impl][0]
     rng = np.random.default_rng(61)
@@ -499,7 +588,8 @@ def test_core_beta_zero_only_decays(impl, d, chunk, dtype):
 
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
     ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.bfloat16),
-    ("simt", 64, 64, torch.float16), ("tc", 128, 64, torch.float16)])
+    ("simt", 64, 64, torch.float16), ("tc", 128, 64, torch.float16),
+    ("fused", 128, 64, torch.float16)])
 def test_core_matches_oracle(impl, d, chunk, dtype):
     code = IMPLS[impl][0]
     rng = np.random.default_rng(62)
