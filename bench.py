@@ -1,22 +1,34 @@
 """Benchmark of the Gated DeltaNet mixer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--decode-workload NAME]
+                    [--workload NAME] [--also NAME ...] [--decode-workload NAME]
 
-Prints ONE JSON line (rank 0).  `value` is prefill tokens/s of one mixer layer
-over all ranks (each rank runs its own copy of the workload: the mixer is
-independent per sequence, so ranks share nothing and scaling is weak).  The
-decode half of the metric (one recurrent step for a batch of sequences on an
-fp32 state in HBM) is reported under "decode".
+Prints ONE JSON line (rank 0).  The metric is the mixer layer's prefill
+tokens/s and decode tokens/s on B200, with the fraction of roofline.
+
+  value     prefill tokens/s of one mixer layer over all ranks on the headline
+            workload (default: 8 packed sequences of 65536 tokens in all, 16
+            key / 64 value heads of width 128 -- the largest single-GPU
+            configuration).  Each rank runs its own copy (the mixer shares
+            nothing across sequences), so scaling is weak.
+  prefill   the same measurement (value, roofline, e2e, CPU baseline) for the
+            other prefill workloads (--also).
+  decode    one recurrent step for a batch of sequences on an fp32 state in
+            HBM (and the bf16-state and 4-token variants).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; before every timed step a 256 MiB buffer is written
 to flush L2 (outside the events).  Max over ranks.  `roofline` reports the
-chunked-core kernel alone (CUDA events recorded by the library around that
-launch).  `e2e` repeats the prefill through the public API with every step's
-inputs copied from pinned host memory and its outputs copied back inside the
-timed region (two buffer sets, copies of one step overlapping the compute of
-the next).  `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
+chunked core alone (events the library records around its launches, in a
+second pass of the same steps).  `e2e` repeats the prefill through the public
+call with every step's inputs copied from pinned host memory and its outputs
+copied back inside the timed region (two buffer sets, copies of one step
+overlapping the compute of the next).  `cpu_baseline` times the fp64 CPU
+oracle on a bounded sample.
+
+With --gpus N > 1 and no torchrun environment, the script starts N ranks
+itself (torch.distributed.run on 127.0.0.1) and fails if the node has fewer
+GPUs.
 """
 from __future__ import annotations
 
@@ -24,6 +36,7 @@ import argparse
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -37,7 +50,9 @@ sys.path.insert(0, ROOT)
 
 from hybrid_linear_attention_05_b200.workloads import WORKLOADS, make_decode, make_prefill  # noqa: E402
 
-DEFAULT_PREFILL = "prefill_T4096_Hk16_Hv16_d128"
+METRIC = "GDN prefill tokens/s & decode tokens/s per layer at 1 B200; % of roofline"
+DEFAULT_PREFILL = "prefill_varlen8_T65536_Hk16_Hv64_d128"
+DEFAULT_ALSO = ["prefill_4x8192_Hk16_Hv32_d128", "prefill_T4096_Hk16_Hv16_d128"]
 DEFAULT_DECODE = "decode_B256_Hk16_Hv32_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -70,6 +85,18 @@ def job_throughput(units_per_rank: int, world: int, max_seconds: float) -> float
     return units_per_rank * world / max_seconds
 
 
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(argv, n: int, port: int):
+    """The command that runs this script as n ranks on this node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=%d" % n,
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
 # ------------------------------------------------------ profiled traffic
 
 PROFILES = os.path.join(ROOT, "profiles", "ncu_traffic.tsv")
@@ -100,7 +127,7 @@ def profiled_traffic(source: str, workload: str):
 
 def prefill_counts(inp, chunk):
     """Algorithmic bytes and FLOPs of one prefill (whole call) and of the
-    chunked-core kernel alone."""
+    chunked core alone."""
     w = inp.w
     T, N, Hk, Hv, d = inp.T, inp.N, w.Hk, w.Hv, w.d
     e = 2 if w.dtype == "bf16" else 4
@@ -196,14 +223,14 @@ class ClockSampler:
 # ---------------------------------------------------------- CPU baseline
 
 
-def cpu_oracle_prefill_sample(inp, budget_s=12.0, max_threads=None):
-    """Time the fp64 oracle on the first `n` tokens of the first sequence
-    (all heads), growing n until the run takes about budget_s/4, then one
-    timed run at the size that fills the budget.  Returns (tokens/s, cores,
-    description)."""
+def cpu_oracle_prefill_sample(inp, budget_s=12.0):
+    """Time the fp64 oracle on the first n tokens of the first sequence (all
+    value heads, one host thread per head up to the core count), growing n
+    until the run takes about budget_s/8, then one timed run at the size that
+    fills the budget.  Returns (tokens/s, threads, description, seconds)."""
     import oracle
     w = inp.w
-    threads = min(os.cpu_count() or 1, w.Hv * 1, max_threads or 1 << 30)
+    threads = min(os.cpu_count() or 1, w.Hv)
     first = int(inp.cu_seqlens[1])
 
     def run(n):
@@ -223,7 +250,7 @@ def cpu_oracle_prefill_sample(inp, budget_s=12.0, max_threads=None):
     if n_final != n:
         dt = run(n_final)
         n = n_final
-    return n / dt, threads, "first %d tokens of one sequence, all %d value heads" % (n, w.Hv)
+    return n / dt, threads, "first %d tokens of one sequence, all %d value heads" % (n, w.Hv), dt
 
 
 def cpu_oracle_decode_sample(inp, budget_s=6.0):
@@ -249,25 +276,39 @@ def cpu_oracle_decode_sample(inp, budget_s=6.0):
 
 # ------------------------------------------------------------- GPU arm
 
+IMPL_NAMES = {1: "simt", 2: "tc", 3: "tc_split", 4: "tc_fused"}
 
-def run_ours(args, rank, world, local_rank):
+
+def core_description(gdn, impl, nseg):
+    """(kernel names, source file, launches per call) of the chunked core that
+    `impl` runs, and the launches of the whole call."""
+    if impl == gdn.GDN_IMPL_TC_FUSED:
+        return "chunk_fused_kernel", "chunk_fused.cu", 1, 3  # + queue order, conv
+    if impl == gdn.GDN_IMPL_TC_SPLIT:
+        if nseg > 1:
+            return ("chunk_keys_kernel + chunk_chain_kernel<xfer> + seg_scan_kernel + chunk_chain_kernel"
+                    " (%d segments)" % nseg, "chunk_tc_split.cu", 4, 5)
+        return "chunk_keys_kernel + chunk_chain_kernel", "chunk_tc_split.cu", 2, 3
+    if impl == gdn.GDN_IMPL_TC:
+        return "chunk_tc_kernel", "chunk_tc.cu", 1, 2
+    return "chunk_simt_kernel", "chunk_simt.cu", 1, 2
+
+
+def bench_prefill(name, args, world, dev, peaks, peak_kind, flush, stream, want_cp=False):
+    """One prefill workload: the timed steps, the core's roofline, e2e and
+    (single GPU, one sequence) the context-parallel pieces."""
     import torch
     import torch.distributed as dist
     from hybrid_linear_attention_05_b200 import api, gdn
-    from hybrid_linear_attention_05_b200 import build as libbuild
 
-    libbuild.build()
-    gdn.lib()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    peaks, peak_kind = load_peaks()
-
-    wp = WORKLOADS[args.workload]
+    wp = WORKLOADS[name]
     inp = make_prefill(wp)
     dp = api.to_device(inp, device=dev, chunk=args.chunk)
     bufs = api.PrefillBuffers(dp)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    impl = gdn.gdn_prefill_resolve_impl(bufs.dims, inp.N, inp.T, dp.chunk, bufs.dtype_code,
+                                        gdn.GDN_IMPL_AUTO, bufs.ws_bytes)
+    nseg = gdn.gdn_prefill_auto_segments(bufs.dims, inp.N, inp.T) if impl == gdn.GDN_IMPL_TC_SPLIT else 1
+    core_name, core_src, core_launches, call_launches = core_description(gdn, impl, nseg)
 
     def step(core_ev=None):
         api.prefill(dp, bufs=bufs, core_events=core_ev)
@@ -280,21 +321,19 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    # the headline steps run as a user would call them: an event recorded
-    # between the conv and the core would keep the key-side kernel from
-    # starting early (programmatic dependent launch), about 10 us per step
-    with ClockSampler(local_rank) as clk:
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
+    # the headline steps run as a user would call them (no event between the
+    # library's launches, which would keep a kernel from starting early)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    # the core's own time: the same steps again, with the library recording
+    # the core's own time: the same steps again with the library recording
     # events around its core launches (for the roofline only)
     cevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
@@ -308,24 +347,11 @@ def run_ours(args, rank, world, local_rank):
     core_ms = [a.elapsed_time(b) for a, b in cevs]
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
-    tokens = inp.T * world
     value = job_throughput(inp.T, world, ms_per_step * 1e-3)
 
     cnt = prefill_counts(inp, dp.chunk)
-    core_avg_s = statistics.mean(core_ms) * 1e-3
+    core_avg_s = max_over_ranks(statistics.mean(core_ms), dev) * 1e-3
     hbm = peaks["hbm_gbs"]
-    # AUTO with room for the records runs the two-kernel tensor-core core
-    # (chunk_keys_kernel, then the chains: with segmented chains the segment
-    # maps and the scan of their start states come first); the library's core
-    # events bracket all of its launches
-    split = dp.chunk == 64
-    nseg = gdn.gdn_prefill_auto_segments(gdn.make_dims(wp.Hk, wp.Hv, wp.d), inp.N, inp.T) if split else 1
-    core_launches = (2 + (2 if nseg > 1 else 0)) if split else 1
-    core_src = "chunk_tc_split.cu" if split else "chunk_simt.cu"
-    core_name = "chunk_simt_kernel"
-    if split:
-        core_name = ("chunk_keys_kernel + chunk_chain_kernel<xfer> + seg_scan_kernel + chunk_chain_kernel"
-                     " (%d segments)" % nseg if nseg > 1 else "chunk_keys_kernel + chunk_chain_kernel")
     roofline = {
         "kernel": core_name,
         "bound": "hbm",
@@ -333,8 +359,7 @@ def run_ours(args, rank, world, local_rank):
         "peak": hbm,
         "unit": "GB/s",
         "frac": cnt["core_bytes"] / core_avg_s / 1e9 / hbm,
-        "traffic": args.core_traffic if args.core_traffic is not None else
-                   profiled_traffic(core_src, args.workload),
+        "traffic": profiled_traffic(core_src, name),
         "peak_source": peak_kind,
         "algorithmic_bytes_per_launch": cnt["core_bytes"],
         "algorithmic_flops_per_launch": cnt["core_flops"],
@@ -342,6 +367,8 @@ def run_ours(args, rank, world, local_rank):
         "tensor_tflops": cnt["core_flops"] / core_avg_s / 1e12,
         "tensor_frac_of_burst": cnt["core_flops"] / core_avg_s / 1e12 / peaks["bf16_tflops"],
         "whole_call_hbm_frac": cnt["call_bytes"] / (ms_per_step * 1e-3) / 1e9 / hbm,
+        "roofline_tokens_per_s": inp.T / max(cnt["call_bytes"] / (hbm * 1e9),
+                                             cnt["call_flops"] / (peaks["bf16_tflops"] * 1e12)),
     }
 
     # ---------------- e2e: pinned host inputs -> device -> prefill -> host
@@ -355,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
             for k in ("mixed_qkv", "a", "b", "z")}
     h_cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).pin_memory()
     h_S0 = None if inp.initial_state is None else torch.from_numpy(inp.initial_state).pin_memory()
-    slots = [(dp, bufs), (api.to_device(inp, device=dev), None)]
+    slots = [(dp, bufs), (api.to_device(inp, device=dev, chunk=args.chunk), None)]
     slots[1] = (slots[1][0], api.PrefillBuffers(slots[1][0]))
     h_out = [torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory() for _ in range(2)]
     h_S = [torch.empty(bufs.final_state.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
@@ -373,8 +400,8 @@ def run_ours(args, rank, world, local_rank):
         d, b = slots[k]
         with torch.cuda.stream(s_in):
             s_in.wait_event(computed[k])  # the step two back is done with these inputs
-            for name, t in host.items():
-                getattr(d, name).copy_(t, non_blocking=True)
+            for nm, t in host.items():
+                getattr(d, nm).copy_(t, non_blocking=True)
             d.cu_seqlens.copy_(h_cu, non_blocking=True)
             if h_S0 is not None:
                 d.initial_state.copy_(h_S0, non_blocking=True)
@@ -412,13 +439,13 @@ def run_ours(args, rank, world, local_rank):
            "pipelined": "two buffer sets; copy-in, compute and copy-out streams"}
     del host, h_out, h_S, slots
 
-    # ---------------- context-parallel pieces: the kernels one rank runs for its
-    # part of a long sequence (the map of the part, the fold of the earlier
-    # parts' maps, the part's prefill), timed on this GPU with the L2 flushed
-    # before each call.  Only on a single-GPU run: the exchange between ranks
-    # (one all-gather of the maps) is not part of these numbers.
+    # ---------------- context-parallel pieces (one sequence, one GPU): the
+    # kernels one rank runs for its part of a long sequence -- the map of the
+    # part, the fold of the earlier parts' maps, the part's prefill -- each with
+    # the L2 flushed before it.  The exchange between ranks (one all-gather of
+    # the maps) is not part of these numbers.
     context_parallel = None
-    if world == 1 and inp.N == 1 and wp.d == 128 and wp.dtype == "bf16":
+    if want_cp and world == 1 and inp.N == 1 and wp.d == 128 and wp.dtype == "bf16":
         W_cp = 8
         maps = api.state_map(dp, bufs)
         gathered = maps.expand(W_cp - 1, *maps.shape).contiguous()
@@ -441,7 +468,6 @@ def run_ours(args, rank, world, local_rank):
 
         map_us = timed(lambda: api.state_map(dp, bufs))
         fold_us = timed(lambda: api.state_fold(gathered, None, wp.Hk, wp.Hv, wp.d, out=S_buf))
-        # the part's prefill on the workspace its map left (conv and key-side kernels skipped)
         part_us = timed(lambda: api.prefill(dp, bufs=bufs, reuse_workspace=True))
         rank_us = map_us + fold_us + part_us
         context_parallel = {
@@ -455,7 +481,28 @@ def run_ours(args, rank, world, local_rank):
         }
         del maps, gathered, S_buf
 
-    # ---------------- decode half of the metric (fp32 state; then a bf16 state)
+    res = {
+        "workload": name, "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step,
+        "config": {"workload": name, "sequences": inp.N, "tokens": inp.T,
+                   "sequence_lengths": [int(x) for x in np.diff(inp.cu_seqlens)],
+                   "key_heads": wp.Hk, "value_heads": wp.Hv, "head_dim": wp.d, "chunk": dp.chunk,
+                   "impl": IMPL_NAMES.get(impl, str(impl)),
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": roofline, "e2e": e2e, "launches_per_step": call_launches,
+    }
+    if context_parallel:
+        res["context_parallel"] = context_parallel
+    del dp, bufs
+    torch.cuda.empty_cache()
+    return res, inp
+
+
+def bench_decode(args, world, dev, peaks, peak_kind, stream):
+    import torch
+    import torch.distributed as dist
+    from hybrid_linear_attention_05_b200 import api
+
+    hbm = peaks["hbm_gbs"]
     wd = WORKLOADS[args.decode_workload]
     dinp = make_decode(wd)
 
@@ -493,11 +540,10 @@ def run_ours(args, rank, world, local_rank):
         "metric": "GDN decode tokens/s per layer", "unit": "tokens/s",
         "value": job_throughput(dinp.mixed_qkv.shape[0], world, d_step_s), "ms_per_step": d_step_s * 1e3,
         "workload": args.decode_workload,
-        "roofline": {"kernel": "gdn_decode", "bound": "hbm",
+        "roofline": {"kernel": "decode_kernel", "bound": "hbm",
                      "achieved": dcnt["bytes"] / d_step_s / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": dcnt["bytes"] / d_step_s / 1e9 / hbm,
-                     "traffic": args.decode_traffic if args.decode_traffic is not None else
-                                profiled_traffic("decode.cu", args.decode_workload),
+                     "traffic": profiled_traffic("decode.cu", args.decode_workload),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": dcnt["bytes"]},
         "l2": "state (%d MiB) larger than L2" % state_mib,
     }
@@ -507,7 +553,7 @@ def run_ours(args, rank, world, local_rank):
     decode["bf16_state"] = {
         "value": job_throughput(dinp.mixed_qkv.shape[0], world, b_step_s), "unit": "tokens/s",
         "ms_per_step": b_step_s * 1e3,
-        "roofline": {"kernel": "gdn_decode (bf16 state)", "bound": "hbm",
+        "roofline": {"kernel": "decode_kernel (bf16 state)", "bound": "hbm",
                      "achieved": bcnt["bytes"] / b_step_s / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": bcnt["bytes"] / b_step_s / 1e9 / hbm, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": bcnt["bytes"]},
@@ -522,30 +568,51 @@ def run_ours(args, rank, world, local_rank):
         "tokens_per_sequence": T_mt,
         "value": job_throughput(dinp.mixed_qkv.shape[0] * T_mt, world, m_step_s), "unit": "tokens/s",
         "ms_per_step": m_step_s * 1e3,
-        "roofline": {"kernel": "gdn_decode (T = 4)", "bound": "hbm",
+        "roofline": {"kernel": "decode_multi_kernel (T = 4)", "bound": "hbm",
                      "achieved": mcnt["bytes"] / m_step_s / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": mcnt["bytes"] / m_step_s / 1e9 / hbm, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": mcnt["bytes"]},
     }
+    return decode, dinp
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from hybrid_linear_attention_05_b200 import gdn
+    from hybrid_linear_attention_05_b200 import build as libbuild
+
+    libbuild.build()
+    gdn.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    with ClockSampler(local_rank) as clk:
+        head, inp = bench_prefill(args.workload, args, world, dev, peaks, peak_kind, flush, stream)
+        others = []
+        for name in args.also:
+            r, o_inp = bench_prefill(name, args, world, dev, peaks, peak_kind, flush, stream, want_cp=True)
+            others.append((r, o_inp))
+        decode, dinp = bench_decode(args, world, dev, peaks, peak_kind, stream)
 
     result = {
-        "metric": "GDN prefill tokens/s per layer (decode tokens/s under 'decode')",
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wp.dtype, "data": "synthetic",
-        "config": {"workload": args.workload, "sequences": inp.N, "tokens": inp.T,
-                   "key_heads": wp.Hk, "value_heads": wp.Hv, "head_dim": wp.d,
-                   "chunk": dp.chunk, "parallelism": "replica per GPU (weak)",
-                   "l2": "flushed before every timed step (256 MiB write)"},
-        "roofline": roofline,
+        "metric": METRIC,
+        "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": WORKLOADS[args.workload].dtype,
+        "data": "synthetic (seeded draws of the workload's shapes and distributions)",
+        "config": {**head["config"], "parallelism": "replica per GPU (weak)"},
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "prefill": {r["workload"]: {k: v for k, v in r.items() if k != "workload"} for r, _ in others},
         "decode": decode,
-        "context_parallel": context_parallel,
-        "e2e": e2e,
-        # conv_prep + the core's launches per prefill step
-        "gpu_launches": (1 + core_launches) * args.steps,
+        # the library's kernels launched in the headline's timed steps
+        "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clk.summary(),
     }
-    return result, inp, dinp
+    return result, inp, others, dinp
 
 
 def main():
@@ -555,37 +622,73 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_PREFILL)
+    ap.add_argument("--also", nargs="*", default=DEFAULT_ALSO,
+                    help="further prefill workloads measured in the same run")
     ap.add_argument("--decode-workload", default=DEFAULT_DECODE)
     ap.add_argument("--chunk", type=int, default=None, help="override the workload's chunk length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--core-traffic", type=float, default=None,
-                    help="dram bytes per chunked-core launch from an ncu capture of this build")
-    ap.add_argument("--decode-traffic", type=float, default=None)
+    ap.add_argument("--launcher-selftest", action="store_true",
+                    help="start the ranks, join them on gloo and report them (no GPU work)")
     args = ap.parse_args()
+
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks ourselves
+        if not args.launcher_selftest and args.impl == "ours":
+            import torch
+            have = torch.cuda.device_count()
+            if have < args.gpus:
+                print(json.dumps({"metric": METRIC, "error": "--gpus %d but this node has %d GPUs"
+                                  % (args.gpus, have)}))
+                sys.exit(1)
+        cmd = launch_command(sys.argv[1:], args.gpus, _free_port())
+        sys.exit(subprocess.call(cmd))
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "error": "WORLD_SIZE %d differs from --gpus %d"
+                              % (world, args.gpus)}))
+        sys.exit(1)
+
+    if args.launcher_selftest:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        got = [None] * world
+        dist.all_gather_object(got, (rank, local_rank, os.getpid()))
+        if rank == 0:
+            print(json.dumps({"world": world, "ranks": [g[0] for g in got],
+                              "local_ranks": [g[1] for g in got], "pids": [g[2] for g in got]}))
+        dist.destroy_process_group()
+        return
 
     if args.impl == "reference":
-        # The reference arm is the fp64 CPU oracle (no reference implementation
-        # exists to install); rank 0 runs it, other ranks exit without work.
+        # The reference arm is the fp64 CPU oracle (there is no reference
+        # implementation to install: the reference is a text of web pages).
+        # Rank 0 runs it on the host cores; other ranks exit without work.
         if rank != 0:
             return
         wp = WORKLOADS[args.workload]
         inp = make_prefill(wp)
-        vals = []
+        vals, secs = [], []
+        cores, sample = 1, ""
         for i in range(args.warmup + args.steps):
-            v, cores, sample = cpu_oracle_prefill_sample(inp, budget_s=3.0)
+            v, cores, sample, dt = cpu_oracle_prefill_sample(inp, budget_s=3.0)
             if i >= args.warmup:
                 vals.append(v)
+                secs.append(dt)
         value = statistics.mean(vals)
         print(json.dumps({
-            "impl": "reference", "metric": "GDN prefill tokens/s per layer", "value": value,
-            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": inp.T / value * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "tokens": inp.T},
+            "impl": "reference", "metric": METRIC, "value": value,
+            "unit": "tokens/s", "n_gpus": 0, "gpus_requested": args.gpus, "runs_on": "host CPU cores",
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.mean(secs) * 1e3, "step": "one bounded sample: " + sample,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded draws of the workload's shapes and distributions)",
+            "config": {"workload": args.workload, "sequences": inp.N, "tokens": inp.T},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -599,12 +702,16 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    result, inp, dinp = run_ours(args, rank, world, local_rank)
+    result, inp, others, dinp = run_ours(args, rank, world, local_rank)
     if rank == 0:
         if not args.no_cpu_baseline:
-            v, cores, sample = cpu_oracle_prefill_sample(inp)
+            v, cores, sample, _ = cpu_oracle_prefill_sample(inp, budget_s=10.0)
             result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
                                       "kind": "oracle", "sample": sample}
+            for r, o_inp in others:
+                v, cores, sample, _ = cpu_oracle_prefill_sample(o_inp, budget_s=5.0)
+                result["prefill"][r["workload"]]["cpu_baseline"] = {
+                    "value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
             dv, dcores, dsample = cpu_oracle_decode_sample(dinp)
             result["decode"]["cpu_baseline"] = {"value": dv, "unit": "tokens/s", "cores": dcores,
                                                 "kind": "oracle", "sample": dsample}

@@ -96,15 +96,16 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // ---- TMEM columns
 constexpr uint32_t TM_S = 0;      // S^T [dk lanes][v columns], fp32
-constexpr uint32_t TM_D = 128;    // two [Vn; O] accumulators, one per stage
-constexpr uint32_t TM_KEY = 384;  // D1, D2, D3 of the key side
+constexpr uint32_t TM_D = 128;    // the chain's [Vn; O] accumulator
+constexpr uint32_t TM_D1 = 256;   // D1 of each stage (64 columns each), issued ahead by the producer
+constexpr uint32_t TM_KEY = 384;  // D2, D3 of the key side
 constexpr uint32_t TM_COLS = 512;
 
 // mbarriers (8 bytes each, from M_BAR).  issued[i] counts the phases of
 // barrier i that a copy or a tensor-core commit was started for, so that
 // the CTA can let them all land before it frees TMEM and leaves.
-enum { B_FULL = 0, B_VFULL = 2, B_READY = 4, B_FREE = 6, B_K1 = 8, B_K2 = 9, B_K3 = 10, B_D = 11,
-       B_S = 13, NBARS = 14 };
+enum { B_FULL = 0, B_VFULL = 2, B_READY = 4, B_FREE = 6, B_K1 = 8, B_K2 = 10, B_K3 = 11, B_D = 12,
+       B_S = 13, B_DFREE = 14, NBARS = 15 };
 
 // Bounded wait that also gives up when another role has given up.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -159,10 +160,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(bar(B_FULL + s), 32);       // the producer warp's lanes (lane 0 with the TMA bytes)
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_READY + s), 1);
-      mbar_init(bar(B_FREE + s), 2);        // the chain's MMAs, and its O-row threads
-      mbar_init(bar(B_D + s), 1);
+      mbar_init(bar(B_FREE + s), 1);        // the chain's MMAs of the stage's chunk have completed
+      mbar_init(bar(B_K1 + s), 1);
     }
-    mbar_init(bar(B_K1), 1);
+    mbar_init(bar(B_D), 1);
+    mbar_init(bar(B_DFREE), 2);             // the chain's new-value and O-row threads read D
     mbar_init(bar(B_K2), 1);
     mbar_init(bar(B_K3), 1);
     mbar_init(bar(B_S), 1);
@@ -246,6 +248,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
           mbar_arrive(bar(B_FULL + s));
         }
+        if (more) {
+          // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T) into this stage's
+          // D1 columns as soon as the tiles land (the key side took the previous
+          // D1 of the stage before the chain released it), then the V tile over
+          // the residual tiles D1 has read
+          bool w = true;
+          if (lane == 0) {
+            const uint32_t ph = (uint32_t)(ci >> 1) & 1u;
+            const uint32_t st = sb + s * STAGE;
+            w = wait_bar(bar(B_FULL + s), ph, abort_flag);
+            if (w) {
+              tc_fence_after();
+              constexpr uint32_t id = idesc_f16(128, 64, false, false);
+              const uint64_t dkq = sdesc_sw128(st + ST_KQ, 16, 1024);
+              const uint64_t dlo = sdesc_sw128(st + ST_LOV, 16, 1024);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint64_t dh = sdesc_add(dkq, off);
+                mma_f16(tmem + TM_D1 + s * 64, dh, dh, id, kk > 0);
+                if (has_lo) {
+                  const uint64_t dl = sdesc_add(dlo, off);
+                  mma_f16(tmem + TM_D1 + s * 64, dl, dh, id, 1);
+                  mma_f16(tmem + TM_D1 + s * 64, dh, dl, id, 1);
+                }
+              }
+              mma_commit(bar(B_K1 + s));
+              issued[B_K1 + s]++;
+              w = wait_bar(bar(B_K1 + s), ph, abort_flag);
+            }
+            if (w) {
+              mbar_arrive_expect_tx(bar(B_VFULL + s), 2 * TILE);
+              tma_load_2d(st + ST_LOV, &tm_v, h * D, c0, bar(B_VFULL + s));
+              tma_load_2d(st + ST_LOV + TILE, &tm_v, h * D + 64, c0, bar(B_VFULL + s));
+              issued[B_VFULL + s]++;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+        }
       }
       if (!more) break;
     }
@@ -258,7 +299,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float* Af = reinterpret_cast<float*>(smem + OFF_AF);
     float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
-    float* Ef = Tf;
     float* Xs = reinterpret_cast<float*>(smem + OFF_X);
     bool ok = true;
     for (int ci = 0;; ++ci) {
@@ -272,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (done && kt == 0) mbar_arrive(bar(B_READY + s));  // tell the chain
         break;
       }
-      const int h = m->h, c0 = m->c0, L = m->L;
+      const int L = m->L;
       const uint32_t st = sb + s * STAGE;
       // gates: gamma = cumulative g, e^gamma, beta
       float gv = 0.f, bv = 0.f;
@@ -293,77 +333,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         eg[kt] = __expf(gv);
         bet[kt] = bv;
       }
-      if (kt == 0 && ok) {  // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T)
-        tc_fence_after();
-        constexpr uint32_t id = idesc_f16(128, 64, false, false);
-        const uint64_t dkq = sdesc_sw128(st + ST_KQ, 16, 1024);
-        const uint64_t dlo = sdesc_sw128(st + ST_LOV, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t dh = sdesc_add(dkq, off);
-          mma_f16(tmem + TM_KEY, dh, dh, id, kk > 0);
-          if (has_lo) {
-            const uint64_t dl = sdesc_add(dlo, off);
-            mma_f16(tmem + TM_KEY, dl, dh, id, 1);
-            mma_f16(tmem + TM_KEY, dh, dl, id, 1);
-          }
-        }
-        mma_commit(bar(B_K1));
-        issued[B_K1]++;
-      }
       role_sync<NK, BAR_K>();  // gamma is in shared memory
-      // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and the stage's vectors
-      {
-        const int j = kt & 63, i0 = (kt >> 6) * 16;
-        const float gj = gam[j];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = i0 + u;
-          if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
-        }
-      }
       if (kt < 64) m->decL[kt] = kt < L ? __expf(gam[L - 1] - gam[kt]) : 0.f;
       if (kt == 0) m->egL = eg[L - 1];
-      ok = wait_bar(bar(B_K1), pk, abort_flag) && ok;
-      if (kt == 0 && ok) {
-        // D1 has read the residual tiles: the V tile goes over them
-        mbar_arrive_expect_tx(bar(B_VFULL + s), 2 * TILE);
-        tma_load_2d(st + ST_LOV, &tm_v, h * D, c0, bar(B_VFULL + s));
-        tma_load_2d(st + ST_LOV + TILE, &tm_v, h * D + 64, c0, bar(B_VFULL + s));
-        issued[B_VFULL + s]++;
-      }
-      role_sync<NK, BAR_K>();  // the decay table is complete
+      ok = wait_bar(bar(B_K1 + s), ph, abort_flag) && ok;  // D1, issued by the producer
       tc_fence_after();
       // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
       // This thread: row tl, columns wg*32 .. wg*32+31.
+      // the decay factors e^{gamma_i - gamma_j} (j <= i) are formed here, from
+      // the row's gamma_i and the columns' gamma_j (clamped so that the masked
+      // entries j > i never overflow)
       {
         float x[32];
-        tmem_ld32(lane_base + TM_KEY + wg * 32, x);
+        tmem_ld32(lane_base + TM_D1 + s * 64 + wg * 32, x);
+        const int i = tl & 63;
+        const float gi = gam[i];
         if (tl < 64) {
-          const int i = tl;
           const float bi = i < L ? bet[i] : 0.f;
 #pragma unroll
           for (int e4 = 0; e4 < 32; e4 += 4) {
+            const float4 g4 = *reinterpret_cast<const float4*>(gam + wg * 32 + e4);
+            const float gj[4] = {g4.x, g4.y, g4.z, g4.w};
             float4 v;
             float* vf = reinterpret_cast<float*>(&v);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int j = wg * 32 + e4 + u;
-              vf[u] = j < i ? bi * Ef[i * ES + j] * x[e4 + u] : 0.f;
+              vf[u] = j < i ? bi * __expf(fminf(gi - gj[u], 0.f)) * x[e4 + u] : 0.f;
             }
             *reinterpret_cast<float4*>(Af + i * AS + wg * 32 + e4) = v;
           }
         } else {
-          const int i = tl - 64;
           const float keep = i < L ? 1.f : 0.f;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            const float4 ga = *reinterpret_cast<const float4*>(gam + wg * 32 + q * 8);
+            const float4 gb = *reinterpret_cast<const float4*>(gam + wg * 32 + q * 8 + 4);
+            const float gj[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int j = wg * 32 + q * 8 + e;
-              f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
+              f[e] = j <= i ? keep * __expf(fminf(gi - gj[e], 0.f)) * x[q * 8 + e] : 0.f;
             }
             st_half8(smem + OFF_TBP, swz(tl, wg * 4 + q), f);
           }
@@ -392,18 +403,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           st_half8(smem + OFF_TBP, swz(i, qt * 2 + q), fb);  // Tb: A rows 0..63 and B block 0 of D2
           st_half8(smem + OFF_AW, swz(i, qt * 2 + q), fe);   // -Tbe: AW rows 0..63 and B block 1 of D2
-        }
-        // AW's second K atom: zero on rows 0..63, E = diag(e^gamma) on rows 64..127
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = kt + NK * k, r = e >> 3, ch = e & 7;
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int ii = r - 64, jj = ch * 8 + u;
-            f[u] = (r >= 64 && jj == ii && ii < L) ? eg[ii] : 0.f;
-          }
-          st_half8(smem + OFF_AW + 16384, swz(r, ch), f);
         }
       }
       fence_proxy_async();
@@ -437,37 +436,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_before();
       role_sync<NK, BAR_K>();
       if (kt == 0) {
-        // (the stage's accumulator is free: the chain released the stage's last
-        // chunk before the producer refilled it)
         ok = wait_bar(bar(B_VFULL + s), ph, abort_flag) && ok;
+        // the chain has read its accumulator for the previous chunk
+        if (ci > 0) ok = wait_bar(bar(B_DFREE), (uint32_t)(ci - 1) & 1u, abort_flag) && ok;
         if (ok) {
           tc_fence_after();
-          // D3 = [-Tbe 0; -Ph E] [K; Q] = [-W; Qt]
+          // D3 = [-Tbe; -Ph] K = [-W; -Ph K]; the diagonal term e^gamma Q of Qt
+          // is added on the CUDA cores as D3 is read
           constexpr uint32_t id = idesc_f16(128, 128, false, true);
           const uint64_t da = sdesc_sw128(sb + OFF_AW, 16, 1024);
           const uint64_t db = sdesc_sw128(st + ST_KQ, 16384, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_f16(tmem + TM_KEY, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(db, kk * 2048),
-                    id, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + TM_KEY, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
           // D4 = [Tb; Pt] V = [U; Pt V], the start of the chain's accumulator
           const uint64_t dt = sdesc_sw128(sb + OFF_TBP, 16, 1024);
           const uint64_t dv = sdesc_sw128(st + ST_LOV, TILE, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + TM_D + s * 128, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
+            mma_f16(tmem + TM_D, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
           mma_commit(bar(B_K3));
           issued[B_K3]++;
         }
       }
       ok = wait_bar(bar(B_K3), pk, abort_flag) && ok;
       tc_fence_after();
-      // [-W; Qt] -> fp16 K-major A operand of the chain, over V: row tl, dk atom wg
+      // [-W; Qt] -> fp16 K-major A operand of the chain, over V: row tl, dk atom
+      // wg; the Qt rows (tl >= 64, token i = tl - 64) add e^{gamma_i} Q[i]
       {
+        const int i = tl - 64;
+        const float egi = (tl >= 64 && i < L) ? eg[i] : 0.f;
+        const uint8_t* qrow = smem + s * STAGE + ST_KQ + wg * 16384;
         float x[32];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           tmem_ld32(lane_base + TM_KEY + wg * 64 + hh * 32, x);
+          if (tl >= 64) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = *reinterpret_cast<const uint4*>(qrow + swz(tl, hh * 4 + q));
+              const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h2[e]);
+                x[q * 8 + 2 * e] = fmaf(egi, f.x, x[q * 8 + 2 * e]);
+                x[q * 8 + 2 * e + 1] = fmaf(egi, f.y, x[q * 8 + 2 * e + 1]);
+              }
+            }
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) st_half8(smem + s * STAGE + ST_LOV + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
         }
@@ -547,12 +563,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t db = sdesc_sw128(sb + OFF_S16, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_f16(tmem + TM_D + s * 128, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
+          mma_f16(tmem + TM_D, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
                   sdesc_add(db, kk * 2048), id, 1);
-        mma_commit(bar(B_D + s));
-        issued[B_D + s]++;
+        mma_commit(bar(B_D));
+        issued[B_D]++;
       }
-      ok = wait_bar(bar(B_D + s), ph, abort_flag) && ok;
+      ok = wait_bar(bar(B_D), pk, abort_flag) && ok;
       tc_fence_after();
       if (vn_role) {
         // Vn decayed to the chunk end -> B operand of the state update (over the image)
@@ -560,7 +576,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float x[32];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(lane_base + TM_D + s * 128 + half * 64 + hh * 32, x);
+          tmem_ld32(lane_base + TM_D + half * 64 + hh * 32, x);
 #pragma unroll
           for (int j = 0; j < 32; ++j) x[j] *= dec;
 #pragma unroll
@@ -569,7 +585,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_proxy_async();
         tc_fence_before();
         ok = !bar_named_or(BAR_VN, 128, !ok);
-        if (ct == 0 && ok) {  // S^T += K^T Vn_d; with the O rows' arrival the stage is then free
+        if (ct == 0 && ok) mbar_arrive(bar(B_DFREE));  // the new-value rows of D are read
+        if (ct == 0 && ok) {  // S^T += K^T Vn_d; then the stage is free
           tc_fence_after();
           constexpr uint32_t id = idesc_f16(128, 128, true, true);
           const uint64_t da = sdesc_sw128(st + ST_KQ, 16384, 1024);
@@ -585,8 +602,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // O rows: token t = tl - 64, this thread's 64 value columns
         const int t = tl - 64;
         float o[64];
-        tmem_ld32(lane_base + TM_D + s * 128 + half * 64, o);
-        tmem_ld32(lane_base + TM_D + s * 128 + half * 64 + 32, o + 32);
+        tmem_ld32(lane_base + TM_D + half * 64, o);
+        tmem_ld32(lane_base + TM_D + half * 64 + 32, o + 32);
         float ss = 0.f;
 #pragma unroll
         for (int j = 0; j < 64; ++j) ss = fmaf(o[j], o[j], ss);
@@ -594,7 +611,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sp[half * 64 + t] = ss;
         tc_fence_before();
         ok = !bar_named_or(BAR_O, 128, !ok);  // both halves' sums are in; D's O rows are read
-        if (ct == 64 && ok) mbar_arrive(bar(B_FREE + s));
+        if (ct == 64 && ok) mbar_arrive(bar(B_DFREE));  // the O rows of D are read
         if (t < L && ok) {
           if (norm_out) {
             const float ri = rsqrtf((sp[t] + sp[64 + t]) * (1.0f / D) + p.eps_norm);
@@ -651,7 +668,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // before TMEM is freed (at once unless a wait above gave up)
     if (lane == 0) {
       for (int i = 0; i < NBARS; ++i)
-        if (issued[i] > 0 && i != B_FREE && i != B_FREE + 1 && i != B_READY && i != B_READY + 1)
+        if (issued[i] > 0 && i != B_FREE && i != B_FREE + 1 && i != B_READY && i != B_READY + 1 &&
+            i != B_DFREE)
           mbar_wait(bar(i), (uint32_t)(issued[i] - 1) & 1u, 100000000ull);
     }
     __syncwarp();

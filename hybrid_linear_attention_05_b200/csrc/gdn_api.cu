@@ -85,9 +85,10 @@ Workspace carve(const gdn_dims* d, int T, gdn_dtype dt, void* base, int N = -1) 
 enum class Path { None, Simt, Tc, TcSplit, TcFused };
 
 // `records` tells whether the workspace can hold the two-kernel path's records.
-Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records) {
+Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records, int N = 0, int Hv = 0) {
   const bool tc = chunk_tc_supported(d, chunk, dt_mid);
   const bool simt = chunk_simt_supported(d, chunk);
+  (void)N; (void)Hv;
   switch (impl) {
     case GDN_IMPL_TC: return tc ? Path::Tc : Path::None;
     case GDN_IMPL_TC_SPLIT: return tc ? Path::TcSplit : Path::None;
@@ -115,6 +116,24 @@ size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_
   return carve(dims, T_tot, dtype, nullptr, N).bytes;
 }
 
+int gdn_prefill_resolve_impl(const gdn_dims* dims, int N, int T_tot, int chunk, gdn_dtype dtype,
+                             gdn_impl impl, size_t workspace_bytes) {
+  const gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (N < 1 || T_tot < 0 || !dtype_ok(dtype)) return GDN_ERR_DIMS;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  const size_t full = carve(dims, T_tot, dtype, nullptr, N).bytes;
+  const Path path = pick_path(impl, dims->dk, chunk, mid_dtype(dtype), workspace_bytes >= full, N, dims->Hv);
+  switch (path) {
+    case Path::Simt: return GDN_IMPL_SIMT;
+    case Path::Tc: return GDN_IMPL_TC;
+    case Path::TcSplit: return workspace_bytes >= full ? GDN_IMPL_TC_SPLIT : GDN_ERR_WORKSPACE;
+    case Path::TcFused: return GDN_IMPL_TC_FUSED;
+    case Path::None: break;
+  }
+  return GDN_ERR_UNSUPPORTED;
+}
+
 int gdn_prefill_auto_segments(const gdn_dims* dims, int N, int T_tot) {
   if (check_dims(dims) != GDN_OK || N < 1 || T_tot < 0) return 0;
   return chunk_tc_split_auto_segments(N, T_tot, dims->Hv);
@@ -134,7 +153,7 @@ gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* a, void* st
   const int Cc = 2 * dims->Hk * d + dims->Hv * d;
   const size_t full = carve(dims, a->T_tot, a->dtype, nullptr, a->N).bytes;
   const bool records = a->workspace && a->workspace_bytes >= full;
-  const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype), records);
+  const Path path = pick_path(a->impl, d, a->chunk, mid_dtype(a->dtype), records, a->N, dims->Hv);
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
   if (path == Path::TcSplit && !records) return GDN_ERR_WORKSPACE;
   if (a->reuse_workspace != 0 && (a->reuse_workspace != 1 || path != Path::TcSplit)) return GDN_ERR_UNSUPPORTED;

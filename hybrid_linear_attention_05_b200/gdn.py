@@ -36,7 +36,7 @@ GDN_IMPL_TC_SPLIT = 3
 GDN_IMPL_TC_FUSED = 4
 
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
-            "gdn_prefill_auto_segments", "gdn_prefill_noalloc", "gdn_prefill_state_map",
+            "gdn_prefill_auto_segments", "gdn_prefill_resolve_impl", "gdn_prefill_noalloc", "gdn_prefill_state_map",
             "gdn_state_fold", "gdn_decode", "gdn_chunk_core", "gdn_core_workspace_size",
             "gdn_device_error", "gdn_selftest_bounded_wait", "gdn_status_string", "gdn_version"]
 
@@ -98,6 +98,9 @@ def lib():
         L.gdn_prefill_workspace_size_n.restype = ctypes.c_size_t
         L.gdn_prefill_auto_segments.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
         L.gdn_prefill_auto_segments.restype = ctypes.c_int
+        L.gdn_prefill_resolve_impl.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_size_t]
+        L.gdn_prefill_resolve_impl.restype = ctypes.c_int
         L.gdn_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args), _vp]
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_prefill_noalloc.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_prefill_args),
@@ -184,6 +187,13 @@ def gdn_prefill_workspace_size_n(dims: gdn_dims, N: int, T_tot: int, dtype: int)
 def gdn_prefill_auto_segments(dims: gdn_dims, N: int, T_tot: int) -> int:
     """Segments per sequence the two-kernel path picks by itself (gdn.h)."""
     return int(lib().gdn_prefill_auto_segments(ctypes.byref(dims), int(N), int(T_tot)))
+
+
+def gdn_prefill_resolve_impl(dims: gdn_dims, N: int, T_tot: int, chunk: int, dtype: int,
+                             impl: int = GDN_IMPL_AUTO, workspace_bytes: int = 0) -> int:
+    """The implementation gdn_prefill runs for these sizes and workspace (gdn.h)."""
+    return int(lib().gdn_prefill_resolve_impl(ctypes.byref(dims), int(N), int(T_tot), int(chunk),
+                                              int(dtype), int(impl), int(workspace_bytes)))
 
 
 def gdn_prefill(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, norm_w,

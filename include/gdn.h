@@ -195,6 +195,13 @@ size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_
  * conv_state_out when given.  The workspace is overwritten. */
 gdn_status gdn_prefill(const gdn_dims* dims, const gdn_prefill_args* args, void* stream);
 
+/* The implementation gdn_prefill runs for these sizes when called with
+ * `impl` (GDN_IMPL_AUTO resolved to a concrete one) and a workspace of
+ * workspace_bytes bytes on the current device; negative gdn_status when that
+ * call would be rejected for its sizes or impl. */
+int gdn_prefill_resolve_impl(const gdn_dims* dims, int N, int T_tot, int chunk, gdn_dtype dtype,
+                             gdn_impl impl, size_t workspace_bytes);
+
 /* Number of segments the two-kernel tensor-core path cuts each sequence's
  * state chain into when gdn_prefill_args.segments is 0, for N sequences of
  * T_tot tokens in total on the current device (1: one serial chain per

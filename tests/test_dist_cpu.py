@@ -58,3 +58,29 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.job_throughput(10, 1, 2.0) == 5.0
+
+
+def test_bench_gpus_2_starts_two_ranks():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself (the same
+    launch path the GPU run takes; here the ranks only join a gloo group and
+    report who they are)."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--launcher-selftest"], capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1]
+    got = json.loads(line)
+    assert got["world"] == 2 and sorted(got["ranks"]) == [0, 1] and sorted(got["local_ranks"]) == [0, 1]
+    assert len(set(got["pids"])) == 2
+
+
+def test_bench_refuses_world_size_mismatch():
+    """Under a launcher whose WORLD_SIZE differs from --gpus the bench fails
+    instead of timing the wrong number of GPUs."""
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0
+    assert "differs from --gpus" in r.stdout
