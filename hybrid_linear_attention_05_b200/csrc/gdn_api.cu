@@ -95,7 +95,9 @@ Path pick_path(gdn_impl impl, int d, int chunk, gdn_dtype dt_mid, bool records, 
     case GDN_IMPL_TC_FUSED: return tc ? Path::TcFused : Path::None;
     case GDN_IMPL_SIMT: return simt ? Path::Simt : Path::None;
     case GDN_IMPL_AUTO:
-      return tc ? (records ? Path::TcSplit : Path::Tc) : (simt ? Path::Simt : Path::None);
+      // two kernels when the workspace holds their records; otherwise the fused
+      // kernel, which needs no more than the base workspace
+      return tc ? (records ? Path::TcSplit : Path::TcFused) : (simt ? Path::Simt : Path::None);
   }
   return Path::None;
 }
@@ -342,8 +344,12 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
-  // no record workspace here, hence no two-kernel path
-  const Path path = a->impl == GDN_IMPL_TC_SPLIT ? Path::None : pick_path(a->impl, d, a->chunk, a->dtype, false);
+  // no record workspace here, hence no two-kernel path; AUTO takes the fused
+  // kernel only when given its chain-queue workspace
+  Path path = a->impl == GDN_IMPL_TC_SPLIT ? Path::None : pick_path(a->impl, d, a->chunk, a->dtype, false);
+  if (a->impl == GDN_IMPL_AUTO && path == Path::TcFused &&
+      (!a->workspace || a->workspace_bytes < kFusedSchedBytes))
+    path = Path::Tc;
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
   if (path == Path::TcFused && (!a->workspace || a->workspace_bytes < kFusedSchedBytes)) return GDN_ERR_WORKSPACE;
   if (!aligned16(a->workspace)) return GDN_ERR_ALIGN;

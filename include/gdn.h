@@ -85,7 +85,11 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype;
 
 /* Implementation selector for the chunked core of gdn_prefill. */
 typedef enum {
-  GDN_IMPL_AUTO = 0,   /* tensor cores when supported, else CUDA cores        */
+  GDN_IMPL_AUTO = 0,   /* tensor cores when supported (GDN_IMPL_TC_SPLIT when the
+                          workspace holds its records, else GDN_IMPL_TC_FUSED;
+                          for gdn_chunk_core GDN_IMPL_TC_FUSED only when given
+                          its workspace, else GDN_IMPL_TC), CUDA cores
+                          otherwise                                          */
   GDN_IMPL_SIMT = 1,   /* fp32 CUDA-core chunked kernel                       */
   GDN_IMPL_TC = 2,     /* tcgen05 tensor-core chunked core, one kernel per call
                           (bf16 inputs, fp16 operands, d = 128, chunk 64);
@@ -187,7 +191,7 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int T_tot, gdn_dtype dty
  * segment maps and start states of a segmented state chain (see
  * gdn_prefill_args.segments).  With at least this much, GDN_IMPL_AUTO takes
  * the two-kernel path where the tensor cores apply; with only
- * gdn_prefill_workspace_size bytes it takes the single-kernel one.  0 when
+ * gdn_prefill_workspace_size bytes it takes the fused one.  0 when
  * the sizes are invalid. */
 size_t gdn_prefill_workspace_size_n(const gdn_dims* dims, int N, int T_tot, gdn_dtype dtype);
 
