@@ -3,4 +3,4 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` import this package.  The CUDA product path never does.
 """
-from .oracle import build, prefill, decode, core, state_map, PrefillResult, default_threads, silu, gated_rmsnorm  # noqa: F401
+from .oracle import build, prefill, decode, core, state_map, PrefillResult, default_threads, silu, gated_rmsnorm, layer, LayerResult, bf16  # noqa: F401

@@ -218,3 +218,53 @@ def gated_rmsnorm(o, z, w, eps=1e-6):
     lib.gdn_oracle_gated_rmsnorm(int(o.size // max(dv, 1)), dv, float(eps), _ptr(o), _ptr(z), _ptr(w),
                                  _ptr(out))
     return out
+
+
+def bf16(x):
+    """x rounded to the nearest bf16 (ties to even), through its fp32 value;
+    returned as float64."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).copy()
+    u += np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    u &= np.uint32(0xFFFF0000)
+    return u.view(np.float32).astype(np.float64)
+
+
+@dataclass
+class LayerResult:
+    y: np.ndarray          # [T, d_model] layer output (out_proj of the mixer output)
+    mixed_qkv: np.ndarray  # [T, Cc] in_proj_qkv output, as the mixer consumed it
+    z: np.ndarray          # [T, Hv*dv]
+    a: np.ndarray          # [T, Hv]
+    b: np.ndarray          # [T, Hv]
+    mixer: PrefillResult
+
+
+def layer(Hk, Hv, dk, dv, cu_seqlens, hidden, W_qkv, W_z, W_a, W_b, W_out, conv_w, A_log, dt_bias,
+          norm_w, initial_state=None, conv_state_in=None, scale=None, activations_bf16=True,
+          nthreads=None) -> LayerResult:
+    """The linear-attention layer around the mixer ("Qwen/Qwen3.5-9B", module
+    tree of a Gated DeltaNet block: in_proj_qkv, in_proj_z, in_proj_b,
+    in_proj_a, the mixer, out_proj): the four input projections of the hidden
+    states (x W^T with W in [out, in] layout), the mixer, and the output
+    projection of its gated-norm output.
+
+    With activations_bf16 the tensors that pass between the projections and
+    the mixer -- the projections' outputs and the mixer output -- are rounded
+    to bf16, the layer's activation type; every product is fp64."""
+    hid = _d(hidden)
+    T, d_model = hid.shape
+    Cc = 2 * Hk * dk + Hv * dv
+    W_qkv, W_z, W_a, W_b, W_out = (_d(w) for w in (W_qkv, W_z, W_a, W_b, W_out))
+    assert W_qkv.shape == (Cc, d_model) and W_z.shape == (Hv * dv, d_model)
+    assert W_a.shape == (Hv, d_model) and W_b.shape == (Hv, d_model)
+    assert W_out.shape == (d_model, Hv * dv)
+    act = bf16 if activations_bf16 else (lambda v: v)
+    mixed = act(hid @ W_qkv.T)
+    z = act(hid @ W_z.T)
+    a = act(hid @ W_a.T)
+    b = act(hid @ W_b.T)
+    r = prefill(Hk, Hv, dk, dv, cu_seqlens, mixed, conv_w, a, b, A_log, dt_bias, z, norm_w,
+                initial_state, conv_state_in, scale=scale, nthreads=nthreads)
+    out = act(r.out.reshape(T, Hv * dv))
+    return LayerResult(y=out @ W_out.T, mixed_qkv=mixed, z=z, a=a, b=b, mixer=r)

@@ -517,3 +517,97 @@ def test_parts_fold_to_the_whole_sequence(oracle_mod):
         t0 += L
     assert rel(np.concatenate(outs), whole.out) < 1e-12
     assert rel(S, whole.final_state[0]) < 1e-12
+
+
+# ------------------------------------------------------- layer projections
+
+
+def _loop_matmul_t(x, w):
+    """x w^T by explicit loops (x [m, k], w [n, k])."""
+    m, k = x.shape
+    n = w.shape[0]
+    y = np.zeros((m, n))
+    for i in range(m):
+        for j in range(n):
+            acc = 0.0
+            for t in range(k):
+                acc += x[i, t] * w[j, t]
+            y[i, j] = acc
+    return y
+
+
+def _layer_inputs(rng, lens, Hk, Hv, d, d_model):
+    inp = mixer_inputs(rng, lens, Hk, Hv, d)
+    Cc = 2 * Hk * d + Hv * d
+    T = int(np.sum(lens))
+    hidden = rng.standard_normal((T, d_model))
+    Ws = dict(W_qkv=rng.standard_normal((Cc, d_model)) * 0.3, W_z=rng.standard_normal((Hv * d, d_model)) * 0.3,
+              W_a=rng.standard_normal((Hv, d_model)) * 0.3, W_b=rng.standard_normal((Hv, d_model)) * 0.3,
+              W_out=rng.standard_normal((d_model, Hv * d)) * 0.3)
+    for k in ("mixed_qkv", "a", "b", "z"):
+        inp.pop(k)
+    return hidden, Ws, inp
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_layer_projections_brute_force(oracle_mod, act):
+    """The layer's four input projections and out_proj against explicit loops
+    (x W^T, weights in [out, in] layout), around the oracle's own mixer; with
+    activations_bf16 the projections' outputs and the mixer output are the
+    bf16 roundings of those products."""
+    rng = np.random.default_rng(31)
+    Hk, Hv, d, d_model = 1, 2, 4, 6
+    hidden, Ws, inp = _layer_inputs(rng, [3, 2], Hk, Hv, d, d_model)
+    r = oracle_mod.layer(Hk, Hv, d, d, hidden=hidden, **Ws, **inp, activations_bf16=act)
+    rnd = oracle_mod.bf16 if act else (lambda v: v)
+    np.testing.assert_allclose(r.mixed_qkv, rnd(_loop_matmul_t(hidden, Ws["W_qkv"])), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(r.z, rnd(_loop_matmul_t(hidden, Ws["W_z"])), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(r.a, rnd(_loop_matmul_t(hidden, Ws["W_a"])), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(r.b, rnd(_loop_matmul_t(hidden, Ws["W_b"])), rtol=1e-13, atol=1e-14)
+    out = rnd(r.mixer.out.reshape(5, Hv * d))
+    np.testing.assert_allclose(r.y, _loop_matmul_t(out, Ws["W_out"]), rtol=1e-12, atol=1e-14)
+
+
+def test_layer_linear_in_out_proj(oracle_mod):
+    """y is linear in W_out (zero weight -> zero output, twice the weight ->
+    twice the output), and the mixer inside sees exactly the projections."""
+    rng = np.random.default_rng(32)
+    Hk, Hv, d, d_model = 1, 2, 4, 8
+    hidden, Ws, inp = _layer_inputs(rng, [4], Hk, Hv, d, d_model)
+    r = oracle_mod.layer(Hk, Hv, d, d, hidden=hidden, **Ws, **inp, activations_bf16=False)
+    r0 = oracle_mod.layer(Hk, Hv, d, d, hidden=hidden, **{**Ws, "W_out": 0 * Ws["W_out"]}, **inp,
+                          activations_bf16=False)
+    r2 = oracle_mod.layer(Hk, Hv, d, d, hidden=hidden, **{**Ws, "W_out": 2 * Ws["W_out"]}, **inp,
+                          activations_bf16=False)
+    assert np.all(r0.y == 0.0)
+    np.testing.assert_allclose(r2.y, 2 * r.y, rtol=1e-14, atol=0)
+    m = oracle_mod.prefill(Hk, Hv, d, d, inp["cu_seqlens"], r.mixed_qkv, inp["conv_w"], r.a, r.b,
+                           inp["A_log"], inp["dt_bias"], r.z, inp["norm_w"], inp["initial_state"],
+                           inp["conv_state_in"])
+    np.testing.assert_array_equal(m.out, r.mixer.out)
+
+
+def test_bf16_rounding_points(oracle_mod):
+    """The oracle's bf16 rounding at hand-checked values: exact bf16 numbers
+    stay, halfway cases go to the even significand, 1 + 2^-9 rounds to 1."""
+    x = np.array([1.0, 1.0 + 2 ** -7, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5, 3.0e38])
+    got = oracle_mod.bf16(x)
+    expect = np.array([1.0, 1.0 + 2 ** -7, 1.0, 1.0 + 2 ** -6, 1.0, -2.5, 2.9993510e38])
+    np.testing.assert_allclose(got[:6], expect[:6], rtol=0, atol=0)
+    assert abs(got[6] - 3.0e38) / 3.0e38 < 2 ** -8
+
+
+def test_9b_layer_weight_shapes_accepted(oracle_mod):
+    """The layer function takes the 9B module tree's weight shapes (in_proj_qkv
+    8192x4096, in_proj_z 4096x4096, in_proj_a/b 32x4096, out_proj 4096x4096):
+    shape checks only, on a one-token call with small random values."""
+    rng = np.random.default_rng(33)
+    Hk, Hv, d, d_model = 16, 32, 128, 4096
+    Cc = 2 * Hk * d + Hv * d
+    assert (Cc, Hv * d) == (8192, 4096)
+    hidden = rng.standard_normal((1, d_model)) * 0.01
+    Ws = dict(W_qkv=np.zeros((Cc, d_model)), W_z=np.zeros((Hv * d, d_model)), W_a=np.zeros((Hv, d_model)),
+              W_b=np.zeros((Hv, d_model)), W_out=np.zeros((d_model, Hv * d)))
+    r = oracle_mod.layer(Hk, Hv, d, d, [0, 1], hidden, **Ws, conv_w=np.zeros((Cc, 4)), A_log=np.zeros(Hv),
+                         dt_bias=np.zeros(Hv), norm_w=np.ones(d))
+    assert r.y.shape == (1, d_model) and np.all(r.y == 0.0)
