@@ -182,3 +182,58 @@ def decode(dd: DeviceDecode, out: Optional[torch.Tensor] = None, T: int = 1) -> 
                    conv_state=dd.conv_state, out=out, B=dd.B,
                    dtype=gdn.dtype_code(dd.mixed_qkv), state_dtype=gdn.dtype_code(dd.state), T=T)
     return out
+
+
+def linear(x: torch.Tensor, w: torch.Tensor, splits=None):
+    """y = x w^T on the tensor cores (bf16); with `splits` (column counts) the
+    columns of y come back as separate tensors."""
+    M, K = x.shape
+    N = w.shape[0]
+    splits = list(splits or [N])
+    outs = [torch.empty((M, c), dtype=torch.bfloat16, device=x.device) for c in splits]
+    gdn.gdn_linear(x=x, w=w, M=M, N=N, K=K, outs=[(o, c, c) for o, c in zip(outs, splits)])
+    return outs if len(outs) > 1 else outs[0]
+
+
+@dataclass
+class DeviceLayer:
+    mixer: DevicePrefill
+    d_model: int
+    hidden: torch.Tensor
+    w_in: torch.Tensor
+    w_out: torch.Tensor
+
+
+def layer_to_device(li, device="cuda") -> DeviceLayer:
+    dp = to_device(li.mixer, device=device)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=torch.bfloat16)  # noqa: E731
+    return DeviceLayer(dp, li.d_model, t(li.hidden), t(li.w_in), t(li.w_out))
+
+
+class LayerBuffers:
+    def __init__(self, dl: DeviceLayer, records: bool = True):
+        dp = dl.mixer
+        dev = dl.hidden.device
+        self.dims = gdn.make_dims(dp.Hk, dp.Hv, dp.d, scale=dp.scale)
+        self.y = torch.empty((dp.T, dl.d_model), dtype=torch.bfloat16, device=dev)
+        self.final_state = torch.empty((dp.N, dp.Hv, dp.d, dp.d), dtype=torch.float32, device=dev)
+        self.conv_state_out = torch.empty((dp.N, dp.Cc, 3), dtype=torch.bfloat16, device=dev)
+        if records:
+            self.ws_bytes = gdn.gdn_layer_workspace_size(self.dims, dl.d_model, dp.N, dp.T)
+        else:
+            self.ws_bytes = (gdn.gdn_layer_activation_bytes(self.dims, dl.d_model, dp.T)
+                             + gdn.gdn_prefill_workspace_size(self.dims, dp.T, gdn.GDN_BF16))
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+
+def layer_prefill(dl: DeviceLayer, bufs: Optional[LayerBuffers] = None, impl: int = gdn.GDN_IMPL_AUTO):
+    """The whole layer: in_proj, the mixer, out_proj (gdn_layer_prefill)."""
+    dp = dl.mixer
+    bufs = bufs or LayerBuffers(dl)
+    gdn.gdn_layer_prefill(bufs.dims, hidden=dl.hidden, w_in=dl.w_in, w_out=dl.w_out, y=bufs.y,
+                          d_model=dl.d_model, conv_w=dp.conv_w, A_log=dp.A_log, dt_bias=dp.dt_bias,
+                          norm_w=dp.norm_w, cu_seqlens=dp.cu_seqlens, N=dp.N, T_tot=dp.T, chunk=dp.chunk,
+                          workspace=bufs.workspace, workspace_bytes=bufs.ws_bytes,
+                          initial_state=dp.initial_state, final_state=bufs.final_state,
+                          conv_state_in=dp.conv_state_in, conv_state_out=bufs.conv_state_out, impl=impl)
+    return bufs

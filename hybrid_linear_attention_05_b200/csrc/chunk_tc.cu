@@ -632,7 +632,9 @@ extern "C" gdn_status gdn_device_error(int* code, int clear) {
   if (v3 < 0) return GDN_ERR_CUDA;
   const int v4 = gdn::fused_error_word(clear);
   if (v4 < 0) return GDN_ERR_CUDA;
-  *code = (v | v2 | v3 | v4) != 0 ? GDN_ERR_TIMEOUT : 0;
+  const int v5 = gdn::linear_error_word(clear);
+  if (v5 < 0) return GDN_ERR_CUDA;
+  *code = (v | v2 | v3 | v4 | v5) != 0 ? GDN_ERR_TIMEOUT : 0;
   return GDN_OK;
 }
 

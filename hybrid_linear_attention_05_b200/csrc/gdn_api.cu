@@ -382,6 +382,117 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
 
 size_t gdn_core_workspace_size(int N) { return N < 0 ? 0 : kFusedSchedBytes; }
 
+gdn_status gdn_linear(const gdn_linear_args* a, void* stream) {
+  if (!a) return GDN_ERR_NULL;
+  if (a->M < 0 || a->N < 1 || a->K < 1 || a->n_outputs < 1 || a->n_outputs > 4) return GDN_ERR_DIMS;
+  if (a->K % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  if (a->ldx < a->K || a->ldw < a->K || a->ldx % 8 != 0 || a->ldw % 8 != 0) return GDN_ERR_DIMS;
+  long cols = 0;
+  for (int i = 0; i < a->n_outputs; ++i) {
+    if (a->out_cols[i] < 8 || a->out_cols[i] % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (a->out_ld[i] < a->out_cols[i] || a->out_ld[i] % 8 != 0) return GDN_ERR_DIMS;
+    cols += a->out_cols[i];
+  }
+  if (cols != a->N) return GDN_ERR_DIMS;
+  if (a->M == 0) return GDN_OK;
+  if (!a->x || !a->w) return GDN_ERR_NULL;
+  if (!aligned16(a->x) || !aligned16(a->w)) return GDN_ERR_ALIGN;
+  for (int i = 0; i < a->n_outputs; ++i) {
+    if (!a->out[i]) return GDN_ERR_NULL;
+    if (!aligned16(a->out[i])) return GDN_ERR_ALIGN;
+  }
+  LinearParams p{};
+  p.M = a->M; p.N = a->N; p.K = a->K; p.n_out = a->n_outputs;
+  for (int i = 0; i < a->n_outputs; ++i) {
+    p.out[i] = a->out[i];
+    p.out_cols[i] = a->out_cols[i];
+    p.out_ld[i] = a->out_ld[i];
+  }
+  return from_cuda(launch_linear_tc(p, a->x, a->ldx, a->w, a->ldw, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+// Activations of the layer in its workspace: mixed_qkv, z, b, a, and the mixer output.
+struct LayerWs {
+  void* mixed; void* z; void* b; void* a; void* out;
+  size_t bytes;
+};
+LayerWs carve_layer(const gdn_dims* d, int T, void* base) {
+  LayerWs w{};
+  const int Cc = 2 * d->Hk * d->dk + d->Hv * d->dv;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t n) { void* r = p ? p + off : nullptr; off += align_up(n, 256); return r; };
+  w.mixed = take((size_t)T * Cc * 2);
+  w.z = take((size_t)T * d->Hv * d->dv * 2);
+  w.b = take((size_t)T * d->Hv * 2);
+  w.a = take((size_t)T * d->Hv * 2);
+  w.out = take((size_t)T * d->Hv * d->dv * 2);
+  w.bytes = off;
+  return w;
+}
+bool layer_dims_ok(const gdn_dims* d, int d_model) {
+  return d_model > 0 && d_model % 64 == 0 && (d->Hv * d->dv) % 64 == 0;
+}
+}  // namespace
+
+size_t gdn_layer_activation_bytes(const gdn_dims* dims, int d_model, int T_tot) {
+  if (check_dims(dims) != GDN_OK || T_tot < 0 || !layer_dims_ok(dims, d_model)) return 0;
+  return carve_layer(dims, T_tot, nullptr).bytes;
+}
+
+size_t gdn_layer_workspace_size(const gdn_dims* dims, int d_model, int N, int T_tot) {
+  if (check_dims(dims) != GDN_OK || T_tot < 0 || N < 0 || !layer_dims_ok(dims, d_model)) return 0;
+  return carve_layer(dims, T_tot, nullptr).bytes + carve(dims, T_tot, GDN_BF16, nullptr, N).bytes;
+}
+
+gdn_status gdn_layer_prefill(const gdn_dims* dims, const gdn_layer_args* a, void* stream) {
+  gdn_status s = check_dims(dims);
+  if (s != GDN_OK) return s;
+  if (!a) return GDN_ERR_NULL;
+  if (a->N < 0 || a->T_tot < 0) return GDN_ERR_DIMS;
+  if (!layer_dims_ok(dims, a->d_model)) return GDN_ERR_UNSUPPORTED;
+  if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
+  const int Cc = 2 * dims->Hk * dims->dk + dims->Hv * dims->dv;
+  const int HVd = dims->Hv * dims->dv;
+  const LayerWs need = carve_layer(dims, a->T_tot, nullptr);
+  if (a->T_tot > 0 && (!a->hidden || !a->w_in || !a->w_out || !a->y)) return GDN_ERR_NULL;
+  if (!a->workspace || a->workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
+  const void* ptrs[] = {a->hidden, a->w_in, a->w_out, a->y, a->workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_ERR_ALIGN;
+  const LayerWs w = carve_layer(dims, a->T_tot, a->workspace);
+  // in_proj: [mixed_qkv | z | b | a] = hidden w_in^T
+  gdn_linear_args li{};
+  li.x = a->hidden; li.w = a->w_in; li.M = a->T_tot; li.N = Cc + HVd + 2 * dims->Hv; li.K = a->d_model;
+  li.ldx = a->d_model; li.ldw = a->d_model; li.n_outputs = 4;
+  li.out[0] = w.mixed; li.out_cols[0] = Cc; li.out_ld[0] = Cc;
+  li.out[1] = w.z; li.out_cols[1] = HVd; li.out_ld[1] = HVd;
+  li.out[2] = w.b; li.out_cols[2] = dims->Hv; li.out_ld[2] = dims->Hv;
+  li.out[3] = w.a; li.out_cols[3] = dims->Hv; li.out_ld[3] = dims->Hv;
+  if (a->T_tot > 0) {
+    s = gdn_linear(&li, stream);
+    if (s != GDN_OK) return s;
+  }
+  // the mixer on the rest of the workspace
+  gdn_prefill_args pa{};
+  pa.mixed_qkv = w.mixed; pa.conv_w = a->conv_w; pa.a = w.a; pa.b = w.b; pa.A_log = a->A_log;
+  pa.dt_bias = a->dt_bias; pa.z = w.z; pa.norm_w = a->norm_w; pa.cu_seqlens = a->cu_seqlens;
+  pa.N = a->N; pa.T_tot = a->T_tot; pa.chunk = a->chunk; pa.dtype = GDN_BF16; pa.impl = a->impl;
+  pa.initial_state = a->initial_state; pa.final_state = a->final_state;
+  pa.conv_state_in = a->conv_state_in; pa.conv_state_out = a->conv_state_out; pa.out = w.out;
+  pa.workspace = static_cast<char*>(a->workspace) + need.bytes;
+  pa.workspace_bytes = a->workspace_bytes - need.bytes;
+  s = gdn_prefill(dims, &pa, stream);
+  if (s != GDN_OK || a->T_tot == 0) return s;
+  // out_proj: y = out w_out^T
+  gdn_linear_args lo{};
+  lo.x = w.out; lo.w = a->w_out; lo.M = a->T_tot; lo.N = a->d_model; lo.K = HVd;
+  lo.ldx = HVd; lo.ldw = HVd; lo.n_outputs = 1;
+  lo.out[0] = a->y; lo.out_cols[0] = a->d_model; lo.out_ld[0] = a->d_model;
+  return gdn_linear(&lo, stream);
+}
+
 const char* gdn_status_string(gdn_status s) {
   switch (s) {
     case GDN_OK: return "ok";

@@ -139,6 +139,21 @@ struct FoldParams {
 };
 cudaError_t launch_state_fold(const FoldParams& p, cudaStream_t st);
 
+// linear_tc.cu: Y = X W^T in bf16 on the tensor cores (X [M, K], W [N, K],
+// K a multiple of 64), the N columns of Y split into n_out consecutive ranges,
+// range i stored to out[i] ([M, out_cols[i]], row stride out_ld[i]).
+struct LinearParams {
+  int M, N, K;
+  int n_out;
+  void* out[4];
+  int out_cols[4];
+  int out_ld[4];
+  int tiles_m, tiles_n;  // set by the launcher
+};
+cudaError_t launch_linear_tc(const LinearParams& p, const void* x, int ldx, const void* w, int ldw,
+                             cudaStream_t st);
+int linear_error_word(int clear);
+
 // decode.cu
 struct DecodeParams {
   const void* x;              // [B, Cc]

@@ -38,6 +38,7 @@ GDN_IMPL_TC_FUSED = 4
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
             "gdn_prefill_auto_segments", "gdn_prefill_resolve_impl", "gdn_prefill_noalloc", "gdn_prefill_state_map",
             "gdn_state_fold", "gdn_decode", "gdn_chunk_core", "gdn_core_workspace_size",
+            "gdn_linear", "gdn_layer_activation_bytes", "gdn_layer_workspace_size", "gdn_layer_prefill",
             "gdn_device_error", "gdn_selftest_bounded_wait", "gdn_status_string", "gdn_version"]
 
 # Size of the library's own scratch used by gdn_prefill_noalloc (gdn.h).
@@ -79,6 +80,20 @@ class gdn_core_args(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
+class gdn_linear_args(ctypes.Structure):
+    _fields_ = [("x", _vp), ("w", _vp), ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+                ("ldx", ctypes.c_int), ("ldw", ctypes.c_int), ("n_outputs", ctypes.c_int),
+                ("out", _vp * 4), ("out_cols", ctypes.c_int * 4), ("out_ld", ctypes.c_int * 4)]
+
+
+class gdn_layer_args(ctypes.Structure):
+    _fields_ = [("hidden", _vp), ("w_in", _vp), ("w_out", _vp), ("y", _vp), ("d_model", ctypes.c_int),
+                ("conv_w", _vp), ("A_log", _vp), ("dt_bias", _vp), ("norm_w", _vp), ("cu_seqlens", _vp),
+                ("N", ctypes.c_int), ("T_tot", ctypes.c_int), ("chunk", ctypes.c_int), ("impl", ctypes.c_int),
+                ("initial_state", _vp), ("final_state", _vp), ("conv_state_in", _vp),
+                ("conv_state_out", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 _lib = None
 
 
@@ -117,6 +132,15 @@ def lib():
         L.gdn_chunk_core.restype = ctypes.c_int
         L.gdn_core_workspace_size.argtypes = [ctypes.c_int]
         L.gdn_core_workspace_size.restype = ctypes.c_size_t
+        L.gdn_linear.argtypes = [ctypes.POINTER(gdn_linear_args), _vp]
+        L.gdn_linear.restype = ctypes.c_int
+        L.gdn_layer_activation_bytes.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
+        L.gdn_layer_activation_bytes.restype = ctypes.c_size_t
+        L.gdn_layer_workspace_size.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int]
+        L.gdn_layer_workspace_size.restype = ctypes.c_size_t
+        L.gdn_layer_prefill.argtypes = [ctypes.POINTER(gdn_dims), ctypes.POINTER(gdn_layer_args), _vp]
+        L.gdn_layer_prefill.restype = ctypes.c_int
         L.gdn_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
         L.gdn_device_error.restype = ctypes.c_int
         L.gdn_selftest_bounded_wait.argtypes = [ctypes.c_int, _vp]
@@ -276,6 +300,44 @@ def gdn_chunk_core(dims: gdn_dims, *, q, k, v, g, beta, cu_seqlens, N, T_tot, ch
     s = current_stream_handle() if stream is None else stream
     return _check(lib().gdn_chunk_core(ctypes.byref(dims), ctypes.byref(args), s),
                   "gdn_chunk_core", raise_on_error)
+
+
+def gdn_linear(*, x, w, M, N, K, outs, ldx=None, ldw=None, stream=None, raise_on_error=True) -> int:
+    """Y = x w^T (bf16); `outs` lists (tensor or pointer, columns, row stride) for
+    the consecutive column ranges of Y (gdn.h)."""
+    args = gdn_linear_args()
+    args.x, args.w = ptr(x), ptr(w)
+    args.M, args.N, args.K = int(M), int(N), int(K)
+    args.ldx = int(K if ldx is None else ldx)
+    args.ldw = int(K if ldw is None else ldw)
+    args.n_outputs = len(outs)
+    for i, (o, cols, ld) in enumerate(outs[:4]):  # more than four: the library rejects n_outputs
+        args.out[i] = ptr(o)
+        args.out_cols[i] = int(cols)
+        args.out_ld[i] = int(ld)
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_linear(ctypes.byref(args), s), "gdn_linear", raise_on_error)
+
+
+def gdn_layer_activation_bytes(dims: gdn_dims, d_model: int, T_tot: int) -> int:
+    return int(lib().gdn_layer_activation_bytes(ctypes.byref(dims), int(d_model), int(T_tot)))
+
+
+def gdn_layer_workspace_size(dims: gdn_dims, d_model: int, N: int, T_tot: int) -> int:
+    return int(lib().gdn_layer_workspace_size(ctypes.byref(dims), int(d_model), int(N), int(T_tot)))
+
+
+def gdn_layer_prefill(dims: gdn_dims, *, hidden, w_in, w_out, y, d_model, conv_w, A_log, dt_bias, norm_w,
+                      cu_seqlens, N, T_tot, chunk, workspace, workspace_bytes, initial_state=None,
+                      final_state=None, conv_state_in=None, conv_state_out=None, impl=GDN_IMPL_AUTO,
+                      stream=None, raise_on_error=True) -> int:
+    args = gdn_layer_args(ptr(hidden), ptr(w_in), ptr(w_out), ptr(y), int(d_model), ptr(conv_w), ptr(A_log),
+                          ptr(dt_bias), ptr(norm_w), ptr(cu_seqlens), int(N), int(T_tot), int(chunk), int(impl),
+                          ptr(initial_state), ptr(final_state), ptr(conv_state_in), ptr(conv_state_out),
+                          ptr(workspace), int(workspace_bytes))
+    s = current_stream_handle() if stream is None else stream
+    return _check(lib().gdn_layer_prefill(ctypes.byref(dims), ctypes.byref(args), s), "gdn_layer_prefill",
+                  raise_on_error)
 
 
 def gdn_device_error(clear: bool = True) -> int:

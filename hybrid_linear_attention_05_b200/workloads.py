@@ -197,3 +197,29 @@ def make_decode(w: Workload, batch: Optional[int] = None) -> DecodeInputs:
 def resized(w: Workload, **kw) -> Workload:
     """A copy of a workload with some fields replaced (same distributions)."""
     return replace(w, **kw)
+
+
+@dataclass
+class LayerInputs:
+    """The layer around the mixer: hidden states and the projection weights
+    (in the [out, in] layout), drawn after the mixer's own inputs."""
+    mixer: PrefillInputs
+    d_model: int
+    hidden: np.ndarray         # [T, d_model]
+    w_in: np.ndarray           # [Cc + Hv*dv + 2*Hv, d_model]: in_proj_qkv; in_proj_z; in_proj_b; in_proj_a
+    w_out: np.ndarray          # [d_model, Hv*dv]
+
+
+def make_layer(w: Workload, d_model: int, seqlens: Optional[tuple] = None,
+               with_conv_state: bool = False) -> LayerInputs:
+    """Hidden states ~ N(0, 1) and weights ~ N(0, 1/fan_in) -- so that the
+    projections come out near unit scale, as the mixer workloads draw them --
+    rounded to bf16 for bf16 workloads; the mixer's parameters, states and
+    lengths are those of make_prefill (its projection outputs are replaced)."""
+    mix = make_prefill(w, seqlens=seqlens, with_conv_state=with_conv_state)
+    rng = np.random.Generator(np.random.PCG64(w.seed + 1000))
+    n_in = w.Cc + w.Hv * w.d + 2 * w.Hv
+    hidden = _cast(_normal(rng, (mix.T, d_model)), w.dtype)
+    w_in = _cast(_normal(rng, (n_in, d_model), d_model ** -0.5), w.dtype)
+    w_out = _cast(_normal(rng, (d_model, w.Hv * w.d), (w.Hv * w.d) ** -0.5), w.dtype)
+    return LayerInputs(mix, d_model, hidden, w_in, w_out)

@@ -341,6 +341,72 @@ typedef struct {
 
 gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* args, void* stream);
 
+/* ------------------------------------------------ projections and the layer
+ * The dense projections around the mixer ("Qwen/Qwen3.5-9B", module tree of a
+ * Gated DeltaNet block: in_proj_qkv 4096->8192, in_proj_z 4096->4096,
+ * in_proj_b and in_proj_a 4096->32, out_proj 4096->4096), on the tcgen05
+ * tensor cores in bf16 with fp32 accumulation.
+ *
+ * gdn_linear: Y = X W^T for X [M, K] and W [N, K] (the [out, in] layout of the
+ * layer's weights), bf16 in and out.  The N columns of Y are cut into
+ * n_outputs consecutive ranges; range i (out_cols[i] columns) is stored to
+ * out[i] as an [M, out_cols[i]] array with row stride out_ld[i], so one call
+ * over the stacked input-projection weights writes mixed_qkv, z, b and a
+ * directly.
+ *   Supported: K a positive multiple of 64; every out_cols[i] a positive
+ *   multiple of 8 with the ranges summing to N; ldx, ldw >= K and out_ld[i] >=
+ *   out_cols[i], all multiples of 8 elements; every pointer 16-byte aligned.
+ *   GDN_ERR_UNSUPPORTED / GDN_ERR_DIMS / GDN_ERR_ALIGN / GDN_ERR_NULL otherwise.
+ */
+typedef struct {
+  const void* x;               /* device [M, K] bf16, rows ldx elements apart   */
+  const void* w;               /* device [N, K] bf16, rows ldw elements apart   */
+  int M, N, K;
+  int ldx, ldw;
+  int n_outputs;               /* 1 .. 4                                        */
+  void* out[4];                /* device bf16 [M, out_cols[i]], rows out_ld[i]  */
+  int out_cols[4];
+  int out_ld[4];
+} gdn_linear_args;
+
+gdn_status gdn_linear(const gdn_linear_args* args, void* stream);
+
+/* gdn_layer_prefill: the layer on packed sequences, y = out_proj(mixer(
+ * in_proj(hidden))).  The input projection is one gdn_linear over w_in, the
+ * rows of in_proj_qkv, in_proj_z, in_proj_b and in_proj_a stacked in that
+ * order ([Cc + Hv*dv + 2*Hv, d_model]); its outputs and the mixer output are
+ * bf16 arrays in the workspace; the mixer is gdn_prefill with `impl` on the
+ * rest of the workspace (AUTO: the two-kernel path when that rest holds its
+ * records).  bf16 only; d_model and Hv*dv multiples of 64.
+ * gdn_layer_workspace_size gives the bytes for both (0 for invalid sizes);
+ * with gdn_layer_activation_bytes + gdn_prefill_workspace_size bytes the
+ * mixer runs without records.  The other arguments mean what they mean for
+ * gdn_prefill. */
+typedef struct {
+  const void* hidden;          /* device [T_tot, d_model] bf16                   */
+  const void* w_in;            /* device [Cc + Hv*dv + 2*Hv, d_model] bf16       */
+  const void* w_out;           /* device [d_model, Hv*dv] bf16                   */
+  void* y;                     /* device [T_tot, d_model] bf16                   */
+  int d_model;
+  const void* conv_w;          /* device [Cc, 4] bf16                            */
+  const float* A_log;          /* device [Hv]                                    */
+  const float* dt_bias;        /* device [Hv]                                    */
+  const void* norm_w;          /* device [dv] bf16                               */
+  const int32_t* cu_seqlens;   /* device [N+1]                                   */
+  int N, T_tot, chunk;
+  gdn_impl impl;
+  const float* initial_state;  /* as in gdn_prefill_args                         */
+  float* final_state;
+  const void* conv_state_in;
+  void* conv_state_out;
+  void* workspace;
+  size_t workspace_bytes;
+} gdn_layer_args;
+
+size_t gdn_layer_activation_bytes(const gdn_dims* dims, int d_model, int T_tot);
+size_t gdn_layer_workspace_size(const gdn_dims* dims, int d_model, int N, int T_tot);
+gdn_status gdn_layer_prefill(const gdn_dims* dims, const gdn_layer_args* args, void* stream);
+
 /* --------------------------------------------------------------- core only
  * Step 4 alone, chunked form, on given q, k (already normalised/scaled), v,
  * log-decay g and beta.  It exists so that the exact invariants of the delta

@@ -237,3 +237,51 @@ def test_selftest_rejects_limits_before_launching(L):
     needed): outside 1 .. 1e6 microseconds nothing is launched."""
     for bad in (0, -5, 1000001):
         assert gdn.gdn_selftest_bounded_wait(bad, stream=0, raise_on_error=False) == gdn.GDN_ERR_DIMS
+
+
+def lin(**over):
+    kw = dict(x=FAKE, w=FAKE, M=300, N=208, K=128, outs=[(FAKE, 64, 64), (FAKE, 128, 128), (FAKE, 8, 8),
+                                                         (FAKE, 8, 8)], stream=0, raise_on_error=False)
+    kw.update(over)
+    return gdn.gdn_linear(**kw)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(K=96), gdn.GDN_ERR_UNSUPPORTED),                      # K a multiple of 64
+    (dict(K=0), gdn.GDN_ERR_DIMS),
+    (dict(N=216), gdn.GDN_ERR_DIMS),                            # ranges do not add up to N
+    (dict(outs=[(FAKE, 204, 204), (FAKE, 4, 8)]), gdn.GDN_ERR_UNSUPPORTED),  # ranges of 8 columns
+    (dict(outs=[(FAKE, 200, 200), (FAKE, 8, 4)]), gdn.GDN_ERR_DIMS),         # row stride below the range
+    (dict(outs=[(FAKE, 208, 212)]), gdn.GDN_ERR_DIMS),          # row stride of whole 16-byte units
+    (dict(outs=[(FAKE, 8, 8)] * 5, N=40), gdn.GDN_ERR_DIMS),    # at most four ranges
+    (dict(ldx=100), gdn.GDN_ERR_DIMS),                          # row stride below K
+    (dict(x=None), gdn.GDN_ERR_NULL),
+    (dict(outs=[(FAKE + 2, 208, 208)]), gdn.GDN_ERR_ALIGN),
+])
+def test_linear_rejects_bad_args(L, over, status):
+    assert lin(**over) == status
+
+
+def test_linear_empty_is_noop(L):
+    assert lin(M=0, x=None, w=None) == gdn.GDN_OK
+
+
+def test_layer_sizes_and_checks(L):
+    """Activation bytes: mixed_qkv, z, b, a and the mixer output in bf16, each
+    rounded up to 256 bytes; the full workspace adds the mixer's own."""
+    dims = gdn.make_dims(16, 32, 128)
+    T = 1000
+    Cc, HVd = 2 * 16 * 128 + 32 * 128, 32 * 128
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    act = up(T * Cc * 2) + 2 * up(T * HVd * 2) + 2 * up(T * 32 * 2)
+    assert gdn.gdn_layer_activation_bytes(dims, 4096, T) == act
+    assert gdn.gdn_layer_workspace_size(dims, 4096, 3, T) == \
+        act + gdn.gdn_prefill_workspace_size_n(dims, 3, T, gdn.GDN_BF16)
+    assert gdn.gdn_layer_activation_bytes(dims, 4000, T) == 0     # d_model a multiple of 64
+    kw = dict(hidden=FAKE, w_in=FAKE, w_out=FAKE, y=FAKE, d_model=4096, conv_w=FAKE, A_log=FAKE,
+              dt_bias=FAKE, norm_w=FAKE, cu_seqlens=FAKE, N=1, T_tot=T, chunk=64, workspace=FAKE,
+              stream=0, raise_on_error=False)
+    assert gdn.gdn_layer_prefill(dims, workspace_bytes=act - 256, **kw) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_layer_prefill(dims, workspace_bytes=act, **dict(kw, d_model=100)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_layer_prefill(dims, workspace_bytes=act, **dict(kw, hidden=None)) == gdn.GDN_ERR_NULL
+    assert gdn.gdn_layer_prefill(dims, workspace_bytes=0, **dict(kw, N=0, T_tot=0)) == gdn.GDN_OK
