@@ -15,6 +15,9 @@ tokens/s and decode tokens/s on B200, with the fraction of roofline.
             other prefill workloads (--also).
   decode    one recurrent step for a batch of sequences on an fp32 state in
             HBM (and the bf16-state and 4-token variants).
+  layer     the whole layer (in_proj GEMM, mixer, out_proj GEMM) with the
+            9B model's hidden size 4096 on the 4 x 8192 workload, and each
+            projection's tensor-core throughput against the bf16 peak.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; before every timed step a 256 MiB buffer is written
@@ -497,6 +500,106 @@ def bench_prefill(name, args, world, dev, peaks, peak_kind, flush, stream, want_
     return res, inp
 
 
+LAYER_D_MODEL = 4096  # the 9B model's hidden size (its mixer shapes are the 4 x 8192 workload's)
+
+
+def layer_counts(inp, d_model):
+    """FLOPs and bytes of the two projections of one layer call."""
+    w = inp.w
+    T, Cc, HVd = inp.T, w.Cc, w.Hv * w.d
+    n_in = Cc + HVd + 2 * w.Hv
+    return dict(in_flops=2 * T * n_in * d_model, out_flops=2 * T * d_model * HVd,
+                in_bytes=2 * (T * d_model + n_in * d_model + T * n_in),
+                out_bytes=2 * (T * HVd + d_model * HVd + T * d_model))
+
+
+def cpu_oracle_layer_sample(li, budget_s=5.0):
+    """The fp64 oracle's whole layer on the first n tokens of the first
+    sequence, n grown until the run takes about budget_s."""
+    import oracle
+    w, m = li.mixer.w, li.mixer
+    threads = min(os.cpu_count() or 1, w.Hv)
+    first = int(m.cu_seqlens[1])
+    Cc, HVd = w.Cc, w.Hv * w.d
+
+    def run(n):
+        x0 = time.perf_counter()
+        oracle.layer(w.Hk, w.Hv, w.d, w.d, [0, n], li.hidden[:n], li.w_in[:Cc], li.w_in[Cc:Cc + HVd],
+                     li.w_in[Cc + HVd + w.Hv:], li.w_in[Cc + HVd:Cc + HVd + w.Hv], li.w_out, m.conv_w,
+                     m.A_log, m.dt_bias, m.norm_w, None if m.initial_state is None else m.initial_state[:1],
+                     None, scale=w.scale, nthreads=threads)
+        return time.perf_counter() - x0
+
+    n = min(32, first)
+    dt = run(n)
+    while dt < budget_s / 4 and n < first:
+        n = min(first, n * 2)
+        dt = run(n)
+    return n / dt, threads, "first %d tokens of one sequence, d_model %d" % (n, li.d_model)
+
+
+def bench_layer(name, args, world, dev, peaks, peak_kind, flush, stream):
+    """The whole layer (in_proj, mixer, out_proj through gdn_layer_prefill) on
+    a mixer workload with the 9B model's hidden size, and each projection's
+    tensor-core throughput timed alone."""
+    import torch
+    from hybrid_linear_attention_05_b200 import api, gdn
+    from hybrid_linear_attention_05_b200.workloads import make_layer
+
+    wp = WORKLOADS[name]
+    li = make_layer(wp, LAYER_D_MODEL)
+    dl = api.layer_to_device(li, device=dev)
+    lb = api.LayerBuffers(dl)
+    T = li.mixer.T
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return max_over_ranks(statistics.mean(ms), dev)
+
+    layer_ms = timed(lambda: api.layer_prefill(dl, bufs=lb))
+    cnt = layer_counts(li.mixer, LAYER_D_MODEL)
+    HVd = wp.Hv * wp.d
+    n_in = dl.w_in.shape[0]
+    y_in = torch.empty((T, n_in), dtype=torch.bfloat16, device=dev)
+    o_in = torch.empty((T, HVd), dtype=torch.bfloat16, device=dev).normal_()
+    in_ms = timed(lambda: gdn.gdn_linear(x=dl.hidden, w=dl.w_in, M=T, N=n_in, K=LAYER_D_MODEL,
+                                         outs=[(y_in, n_in, n_in)]))
+    out_ms = timed(lambda: gdn.gdn_linear(x=o_in, w=dl.w_out, M=T, N=LAYER_D_MODEL, K=HVd,
+                                          outs=[(lb.y, LAYER_D_MODEL, LAYER_D_MODEL)]))
+    peak = peaks["bf16_tflops"]
+    proj = {}
+    for key, ms, fl, by in (("in_proj", in_ms, cnt["in_flops"], cnt["in_bytes"]),
+                            ("out_proj", out_ms, cnt["out_flops"], cnt["out_bytes"])):
+        tf = fl / (ms * 1e-3) / 1e12
+        proj[key] = {"kernel": "linear_tc_kernel", "bound": "tensor", "achieved": tf, "peak": peak,
+                     "unit": "TFLOP/s", "frac": tf / peak, "peak_source": peak_kind + " (burst: timed alone)",
+                     "kernel_us": ms * 1e3, "algorithmic_flops_per_launch": fl,
+                     "algorithmic_bytes_per_launch": by}
+    proj["in_proj"]["shape"] = "M %d, N %d (qkv %d | z %d | b %d | a %d), K %d" % (
+        T, n_in, wp.Cc, HVd, wp.Hv, wp.Hv, LAYER_D_MODEL)
+    proj["out_proj"]["shape"] = "M %d, N %d, K %d" % (T, LAYER_D_MODEL, HVd)
+    res = {"workload": name + " + projections d_model %d" % LAYER_D_MODEL,
+           "value": job_throughput(T, world, layer_ms * 1e-3), "unit": "tokens/s", "ms_per_step": layer_ms,
+           "config": {"workload": name, "d_model": LAYER_D_MODEL, "tokens": T, "sequences": li.mixer.N,
+                      "impl": "gdn_layer_prefill (in_proj GEMM, mixer, out_proj GEMM)",
+                      "l2": "flushed before every timed step (256 MiB write)"},
+           "projections": proj, "launches_per_step": 5}
+    del dl, lb, y_in, o_in
+    torch.cuda.empty_cache()
+    return res, li
+
+
 def bench_decode(args, world, dev, peaks, peak_kind, stream):
     import torch
     import torch.distributed as dist
@@ -596,6 +699,8 @@ def run_ours(args, rank, world, local_rank):
             r, o_inp = bench_prefill(name, args, world, dev, peaks, peak_kind, flush, stream, want_cp=True)
             others.append((r, o_inp))
         decode, dinp = bench_decode(args, world, dev, peaks, peak_kind, stream)
+        layer, linp = (None, None) if args.no_layer else bench_layer(
+            args.layer_workload, args, world, dev, peaks, peak_kind, flush, stream)
 
     result = {
         "metric": METRIC,
@@ -608,11 +713,12 @@ def run_ours(args, rank, world, local_rank):
         "e2e": head["e2e"],
         "prefill": {r["workload"]: {k: v for k, v in r.items() if k != "workload"} for r, _ in others},
         "decode": decode,
+        "layer": layer,
         # the library's kernels launched in the headline's timed steps
         "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clk.summary(),
     }
-    return result, inp, others, dinp
+    return result, inp, others, dinp, linp
 
 
 def main():
@@ -626,6 +732,9 @@ def main():
                     help="further prefill workloads measured in the same run")
     ap.add_argument("--decode-workload", default=DEFAULT_DECODE)
     ap.add_argument("--chunk", type=int, default=None, help="override the workload's chunk length")
+    ap.add_argument("--layer-workload", default="prefill_4x8192_Hk16_Hv32_d128",
+                    help="mixer workload of the whole-layer line (hidden size %d)" % LAYER_D_MODEL)
+    ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--launcher-selftest", action="store_true",
                     help="start the ranks, join them on gloo and report them (no GPU work)")
@@ -702,7 +811,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    result, inp, others, dinp = run_ours(args, rank, world, local_rank)
+    result, inp, others, dinp, linp = run_ours(args, rank, world, local_rank)
     if rank == 0:
         if not args.no_cpu_baseline:
             v, cores, sample, _ = cpu_oracle_prefill_sample(inp, budget_s=10.0)
@@ -715,6 +824,10 @@ def main():
             dv, dcores, dsample = cpu_oracle_decode_sample(dinp)
             result["decode"]["cpu_baseline"] = {"value": dv, "unit": "tokens/s", "cores": dcores,
                                                 "kind": "oracle", "sample": dsample}
+            if linp is not None:
+                lv, lcores, lsample = cpu_oracle_layer_sample(linp)
+                result["layer"]["cpu_baseline"] = {"value": lv, "unit": "tokens/s", "cores": lcores,
+                                                   "kind": "oracle", "sample": lsample}
         print(json.dumps(result))
     if world > 1:
         import torch.distributed as dist

@@ -10,7 +10,7 @@
 //     O  = Qt S0^T + Pt V,   Qt = diag(e^gamma) Q - P W,   Pt = P Tb,
 // so one M = 128 accumulator [-W; Qt] S0^T plus [U; Pt V] holds both.
 //
-//  1. chunk_keys_kernel, one CTA per (chunk, value head), on every SM:
+//  1. chunk_keys_kernel, one unit per (chunk, value head), persistent CTAs:
 //       D1 = [K; Q] K^T              ->  A = beta e^{gamma_i-gamma_j} K K^T,  P
 //       T  = (I + A)^-1              (CUDA cores, fp32)
 //       D2 = [Tb; P] [Tb | Tbe]      ->  Pt = P Tb,  Ph = P Tbe
@@ -57,6 +57,7 @@
 #include <math.h>
 
 #include "gdn_internal.h"
+#include "host_util.h"
 #include "tc_chunk_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -104,10 +105,44 @@ constexpr uint32_t A_TM_D1 = 0, A_TM_D3 = 0, A_TM_D2 = 128, A_TM_D4 = 128, A_TM_
 static_assert(A_AW + 32768 <= A_MISC, "AW image inside the dead fp32 scratch");
 static_assert(2 * A_SMEM <= 232448, "two key-side CTAs per SM");
 
+// Where a unit (chunk slot g, value head h) of the key-side kernel lies: its
+// sequence's chunk c0 .. c0 + L - 1.  Units run heads fastest and chunk slots
+// from the last down, so that the records the chains read first are the most
+// recently written (in L2).  Returns false for a slot without a chunk.
+struct KeyUnit {
+  int g, h, c0, L;
+};
+__device__ __forceinline__ bool key_unit(const ChunkParams& p, int slots, int u, KeyUnit& k) {
+  k.h = u % p.Hv;
+  k.g = slots - 1 - u / p.Hv;
+  int lo = 0, hi = p.N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (slot_start(p.cu_seqlens, mid, p.T) <= k.g) lo = mid; else hi = mid - 1;
+  }
+  const int bos = clampi(__ldg(p.cu_seqlens + lo), 0, p.T);
+  const int eos = clampi(__ldg(p.cu_seqlens + lo + 1), bos, p.T);
+  const int c = k.g - slot_start(p.cu_seqlens, lo, p.T);
+  if (c < 0 || c >= (eos - bos + C - 1) / C) return false;
+  k.c0 = bos + c * C;
+  k.L = min(C, eos - k.c0);
+  return true;
+}
+// The first unit with a chunk at or after u in this CTA's stride (u >= units: none).
+__device__ __forceinline__ int next_key_unit(const ChunkParams& p, int slots, int u, KeyUnit& k) {
+  const int units = slots * p.Hv;
+  for (; u < units; u += (int)gridDim.x)
+    if (key_unit(p, slots, u, k)) return u;
+  return units;
+}
+
+// Persistent: each CTA walks the units u = blockIdx.x + k gridDim.x.  While a
+// unit's MMAs run, the next unit's place and gates are looked up, so that
+// only its operand copies stand between two units.
 __global__ void __launch_bounds__(NTA, 2)
     chunk_keys_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ql,
-                      const __grid_constant__ CUtensorMap tm_kl, ChunkParams p) {
+                      const __grid_constant__ CUtensorMap tm_kl, ChunkParams p, int slots) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -126,41 +161,13 @@ __global__ void __launch_bounds__(NTA, 2)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = tid >> 7, tl = tid & 127;
-  // heads vary fastest and chunk slots run from the last down, so that the
-  // records the chains read first are the most recently written (in L2)
-  const int g = (int)(gridDim.y - 1 - blockIdx.y), h = blockIdx.x;
   pdl_launch();
-  // the sequence whose chunk owns this slot
-  int lo = 0, hi = p.N - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (slot_start(p.cu_seqlens, mid, p.T) <= g) lo = mid; else hi = mid - 1;
-  }
-  const int n = lo;
-  const int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
-  const int eos = clampi(__ldg(p.cu_seqlens + n + 1), bos, p.T);
-  const int c = g - slot_start(p.cu_seqlens, n, p.T);
-  if (c < 0 || c >= (eos - bos + C - 1) / C) return;  // slot without a chunk
-  const int c0 = bos + c * C;
-  const int L = min(C, eos - c0);
-  const int hk = h / (p.Hv / p.Hk);
-  uint8_t* rec = p.rec + ((size_t)g * p.Hv + h) * REC;
-
-  // z of the chunk (an input of the call) is requested first: its latency
-  // overlaps the set-up and the wait for the conv kernel
-  // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
-  // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
+  const int units = slots * p.Hv;
   const bool gated = p.z != nullptr;  // w * silu(z) into the record (the gated norm's factor)
-  uint4 zv[4];
-  if (gated) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
-      zv[k] = r < L ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.z) +
-                                                           (size_t)(c0 + r) * p.Hv * D + h * D + ch * 8))
-                    : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+  // With the rounding residuals of q and k, D1 also takes [K_lo; Q_lo] K^T
+  // and [K; Q] K_lo^T; their tiles ([K_lo; Q_lo] dk halves, laid out like
+  // [K; Q]) land in A_TBP and A_AF, which nothing uses before D1 completes.
+  const bool has_lo = p.k_lo != nullptr;
 
   if (tid == 0) {
     mbar_init(bar_load, 1);
@@ -173,274 +180,324 @@ __global__ void __launch_bounds__(NTA, 2)
     tmem_alloc(smem_u32(tmem_slot), A_TM_COLS);
     tmem_relinquish();
   }
+  if (gated && tid < D) wsm[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tid]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   pdl_wait();  // q, k, v and the gates come from the conv kernel
-  float gv = 0.f, bv = 0.f;
-  if (tid < L) {
-    gv = __ldg(p.g + (size_t)h * p.T + c0 + tid);
-    bv = __ldg(p.beta + (size_t)h * p.T + c0 + tid);
-  }
 
-  // With the rounding residuals of q and k, D1 also takes [K_lo; Q_lo] K^T
-  // and [K; Q] K_lo^T; their tiles ([K_lo; Q_lo] dk halves, laid out like
-  // [K; Q]) land in A_TBP and A_AF, which nothing uses before D1 completes.
-  const bool has_lo = p.k_lo != nullptr;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_load, (has_lo ? 10 : 6) * TILE);
-    tma_load_2d(sb + A_KQ, &tm_k, hk * D, c0, bar_load);
-    tma_load_2d(sb + A_KQ + 16384, &tm_k, hk * D + 64, c0, bar_load);
-    tma_load_2d(sb + A_KQ + 8192, &tm_q, hk * D, c0, bar_load);
-    tma_load_2d(sb + A_KQ + 16384 + 8192, &tm_q, hk * D + 64, c0, bar_load);
-    tma_load_2d(sb + A_V, &tm_v, h * D, c0, bar_load);
-    tma_load_2d(sb + A_V + TILE, &tm_v, h * D + 64, c0, bar_load);
-    if (has_lo) {
-      tma_load_2d(sb + A_TBP, &tm_kl, hk * D, c0, bar_load);
-      tma_load_2d(sb + A_AF, &tm_kl, hk * D + 64, c0, bar_load);
-      tma_load_2d(sb + A_TBP + 8192, &tm_ql, hk * D, c0, bar_load);
-      tma_load_2d(sb + A_AF + 8192, &tm_ql, hk * D + 64, c0, bar_load);
-    }
+  KeyUnit cur{}, nxt{};
+  int u = next_key_unit(p, slots, (int)blockIdx.x, cur);
+  // gates of the unit about to start (thread i < 64: token i of its chunk)
+  float gv_n = 0.f, bv_n = 0.f;
+  if (u < units && tid < cur.L) {
+    gv_n = __ldg(p.g + (size_t)cur.h * p.T + cur.c0 + tid);
+    bv_n = __ldg(p.beta + (size_t)cur.h * p.T + cur.c0 + tid);
   }
-  if (gated && tid < D) wsm[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[tid]);
-  // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
-  if (tid < 64) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float t = __shfl_up_sync(0xffffffffu, gv, o);
-      if (lane >= o) gv += t;
-    }
-    if (tid == 31) scan[0] = gv;
-  }
-  __syncthreads();
-  if (tid < 64) {
-    if (tid >= 32) gv += scan[0];
-    gam[tid] = gv;
-    eg[tid] = __expf(gv);
-    bet[tid] = bv;
-  }
+  // barrier phases completed so far (one per unit each), and what thread 0
+  // has started in the current unit (to let it land on a failure)
+  uint32_t par = 0;
+  bool started_load = false, started_m1 = false, started_m2 = false, started_m3 = false;
+  bool failed = false;
+  while (u < units) {
+    const int h = cur.h, g = cur.g, c0 = cur.c0, L = cur.L;
+    const int hk = h / (p.Hv / p.Hk);
+    uint8_t* rec = p.rec + ((size_t)g * p.Hv + h) * REC;
+    started_load = started_m1 = started_m2 = started_m3 = false;
 
-  bool ok = mbar_wait(bar_load, 0);
-  if (!__syncthreads_or(!ok)) {
-    if (tid == 0) {  // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T)
-      tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 64, false, false);
-      const uint64_t dkq = sdesc_sw128(sb + A_KQ, 16, 1024);
-      const uint64_t dlo[2] = {sdesc_sw128(sb + A_TBP, 16, 1024), sdesc_sw128(sb + A_AF, 16, 1024)};
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        const uint64_t dh = sdesc_add(dkq, off);
-        mma_f16(tmem + A_TM_D1, dh, dh, id, kk > 0);
-        if (has_lo) {
-          const uint64_t lw = sdesc_add(dlo[kk >> 2], (kk & 3) * 32);
-          mma_f16(tmem + A_TM_D1, lw, dh, id, 1);
-          mma_f16(tmem + A_TM_D1, dh, lw, id, 1);
-        }
-      }
-      mma_commit(bar_m1);
-    }
-    // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and
-    // the record's vectors; this thread: column j = tid % 64, rows 16 (tid / 64) .. +15
-    {
-      const int j = tid & 63, i0 = (tid >> 6) * 16;
-      const float gj = gam[j];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + u;
-        if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
-      }
-    }
-    if (tid < 64) {
-      float* vec = reinterpret_cast<float*>(rec + R_VEC);
-      vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
-      if (tid == 0) vec[64] = eg[L - 1];
-    }
-    ok = mbar_wait(bar_m1, 0);
-  }
-  if (!__syncthreads_or(!ok)) {
-    tc_fence_after();
-    // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
-    // This thread: row tl, columns wg*32 .. wg*32+31.
-    {
-      float x[32];
-      tmem_ld32(lane_base + A_TM_D1 + wg * 32, x);
-      if (tl < 64) {
-        const int i = tl;
-        const float bi = i < L ? bet[i] : 0.f;
-#pragma unroll
-        for (int e4 = 0; e4 < 32; e4 += 4) {
-          float4 v;
-          float* vf = reinterpret_cast<float*>(&v);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = wg * 32 + e4 + u;
-            vf[u] = j < i ? bi * Ef[i * ES + j] * x[e4 + u] : 0.f;
-          }
-          *reinterpret_cast<float4*>(Af + i * AS + wg * 32 + e4) = v;
-        }
-      } else {
-        const int i = tl - 64;
-        const float keep = i < L ? 1.f : 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = wg * 32 + q * 8 + e;
-            f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
-          }
-          st_half8(smem + A_TBP, swz(tl, wg * 4 + q), f);
-        }
-      }
-    }
-    __syncthreads();
-    solve_unit_lower<NTA>(Af, Tf, Xs, tid);
-    // this thread's 16 entries of T, row i = tid / 4, columns (tid % 4) * 16 ..
-    const int i = tid >> 2, qt = tid & 3;
-    float tv[16];
-#pragma unroll
-    for (int e4 = 0; e4 < 16; e4 += 4) {
-      const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + qt * 16 + e4);
-      tv[e4] = t4.x; tv[e4 + 1] = t4.y; tv[e4 + 2] = t4.z; tv[e4 + 3] = t4.w;
-    }
-    __syncthreads();  // the fp32 scratch is dead from here: the AW image goes over it
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      float fb[8], fe[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = qt * 16 + q * 8 + e;
-        fb[e] = tv[q * 8 + e] * bet[j];
-        fe[e] = fb[e] * eg[j];
-      }
-      st_half8(smem + A_TBP, swz(i, qt * 2 + q), fb);  // Tb: A rows 0..63 and B block 0 of D2
-      st_half8(smem + A_AW, swz(i, qt * 2 + q), fe);   // Tbe: AW rows 0..63 and B block 1 of D2
-    }
-    // AW's second K atom: zero on rows 0..63, -E on rows 64..127
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int e = tid + NTA * k, r = e >> 3, ch = e & 7;
-      float f[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int ii = r - 64, j = ch * 8 + u;
-        f[u] = (r >= 64 && j == ii && ii < L) ? -eg[ii] : 0.f;
-      }
-      st_half8(smem + A_AW + 16384, swz(r, ch), f);
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {  // D2 = [Tb; P] [Tb | Tbe]
-      tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 128, false, true);
-      const uint64_t da = sdesc_sw128(sb + A_TBP, 16, 1024);
-      const uint64_t db = sdesc_sw128(sb + A_TBP, A_AW - A_TBP, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + A_TM_D2, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
-      mma_commit(bar_m2);
-    }
-    ok = mbar_wait(bar_m2, 0);
-  }
-  if (!__syncthreads_or(!ok)) {
-    tc_fence_after();
-    // rows 64..127 of D2: Pt (columns 0..63) over P in [Tb; P], Ph (64..127) -> AW rows 64..127
-    if (tl >= 64) {
-      float x[32];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(lane_base + A_TM_D2 + wg * 64 + hh * 32, x);
-        uint8_t* dst = smem + (wg == 0 ? A_TBP : A_AW);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) st_half8(dst, swz(tl, hh * 4 + q), x + q * 8);
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      // D3 = [Tbe 0; Ph -E] [K; Q] = [W; -Qt]
-      constexpr uint32_t id = idesc_f16(128, 128, false, true);
-      const uint64_t da = sdesc_sw128(sb + A_AW, 16, 1024);
-      const uint64_t db = sdesc_sw128(sb + A_KQ, 16384, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_f16(tmem + A_TM_D3, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(db, kk * 2048),
-                id, kk > 0);
-      // D4 = [Tb; Pt] V = [U; Pt V]
-      const uint64_t dt = sdesc_sw128(sb + A_TBP, 16, 1024);
-      const uint64_t dv = sdesc_sw128(sb + A_V, TILE, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + A_TM_D4, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
-      mma_commit(bar_m3);
-    }
-    ok = mbar_wait(bar_m3, 0);
-  }
-  if (!__syncthreads_or(!ok)) {
-    tc_fence_after();
-    // The record is assembled in shared memory regions the MMAs no longer
-    // read: [-W; Qt] over AW, [U; Pt V] over [K; Q], w * silu(z) over [Tb; Pt].
-    // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.  Each
-    // warpgroup's part leaves by bulk copy as soon as that warpgroup has
-    // written it (a named barrier per warpgroup), overlapping the rest.
-    const bool wg_lead = tl == 0;
-    float x[32];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      tmem_ld32(lane_base + A_TM_D3 + wg * 64 + hh * 32, x);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = -x[j];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(smem + A_AW + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
-    }
-    fence_proxy_async();
-    bar_named(1 + wg, 128);
-    if (wg_lead) bulk_store(rec + R_WQ + wg * 16384, sb + A_AW + wg * 16384, 16384);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      tmem_ld32(lane_base + A_TM_D4 + wg * 64 + hh * 32, x);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_half8(smem + A_KQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
-    }
-    fence_proxy_async();
-    bar_named(1 + wg, 128);
-    if (wg_lead) {
-      bulk_store(rec + R_UO + wg * 16384, sb + A_KQ + wg * 16384, 16384);
-      bulk_commit();
-    }
-    // w * silu(z) in the chain's tile layout (value block ch / 8, row r, swizzled chunk)
+    // z of the chunk for the gated norm: thread tid takes the 16-byte chunks
+    // e = tid + 256 k of the 64 x 128 tile, row e / 16, value chunk e % 16
+    uint4 zv[4];
     if (gated) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
-        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
-        uint4 res;
-        __half2* r2 = reinterpret_cast<__half2*>(&res);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 zf = __bfloat1622float2(z2[q]);
-          r2[q] = __floats2half2_rn(wsm[ch * 8 + 2 * q] * silu_tanh(zf.x), wsm[ch * 8 + 2 * q + 1] * silu_tanh(zf.y));
-        }
-        *reinterpret_cast<uint4*>(smem + A_TBP + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
-      }
-      fence_proxy_async();
-      __syncthreads();
-      if (tid == 0) {
-        bulk_store(rec + R_ZW, sb + A_TBP, 16384);
-        bulk_commit();
+        zv[k] = r < L ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.z) +
+                                                             (size_t)(c0 + r) * p.Hv * D + h * D + ch * 8))
+                      : make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    if (wg_lead) bulk_wait_read();  // shared memory stays valid until the copies have read it
-  } else if (tid == 0) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(bar_load, (has_lo ? 10 : 6) * TILE);
+      tma_load_2d(sb + A_KQ, &tm_k, hk * D, c0, bar_load);
+      tma_load_2d(sb + A_KQ + 16384, &tm_k, hk * D + 64, c0, bar_load);
+      tma_load_2d(sb + A_KQ + 8192, &tm_q, hk * D, c0, bar_load);
+      tma_load_2d(sb + A_KQ + 16384 + 8192, &tm_q, hk * D + 64, c0, bar_load);
+      tma_load_2d(sb + A_V, &tm_v, h * D, c0, bar_load);
+      tma_load_2d(sb + A_V + TILE, &tm_v, h * D + 64, c0, bar_load);
+      if (has_lo) {
+        tma_load_2d(sb + A_TBP, &tm_kl, hk * D, c0, bar_load);
+        tma_load_2d(sb + A_AF, &tm_kl, hk * D + 64, c0, bar_load);
+        tma_load_2d(sb + A_TBP + 8192, &tm_ql, hk * D, c0, bar_load);
+        tma_load_2d(sb + A_AF + 8192, &tm_ql, hk * D + 64, c0, bar_load);
+      }
+      started_load = true;
+    }
+    // gates of the chunk: gamma = cumulative g, e^gamma, beta (0 past the chunk)
+    float gv = gv_n, bv = bv_n;
+    if (tid < 64) {
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, gv, o);
+        if (lane >= o) gv += t;
+      }
+      if (tid == 31) scan[0] = gv;
+    }
+    __syncthreads();
+    if (tid < 64) {
+      if (tid >= 32) gv += scan[0];
+      gam[tid] = gv;
+      eg[tid] = __expf(gv);
+      bet[tid] = bv;
+    }
+    // the next unit's place and gates, while this one's copies and MMAs run
+    const int u_next = next_key_unit(p, slots, u + (int)gridDim.x, nxt);
+    gv_n = 0.f;
+    bv_n = 0.f;
+    if (u_next < units && tid < nxt.L) {
+      gv_n = __ldg(p.g + (size_t)nxt.h * p.T + nxt.c0 + tid);
+      bv_n = __ldg(p.beta + (size_t)nxt.h * p.T + nxt.c0 + tid);
+    }
+
+    bool ok = mbar_wait(bar_load, par);
+    if (!__syncthreads_or(!ok)) {
+      if (tid == 0) {  // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T)
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16(128, 64, false, false);
+        const uint64_t dkq = sdesc_sw128(sb + A_KQ, 16, 1024);
+        const uint64_t dlo[2] = {sdesc_sw128(sb + A_TBP, 16, 1024), sdesc_sw128(sb + A_AF, 16, 1024)};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t dh = sdesc_add(dkq, off);
+          mma_f16(tmem + A_TM_D1, dh, dh, id, kk > 0);
+          if (has_lo) {
+            const uint64_t lw = sdesc_add(dlo[kk >> 2], (kk & 3) * 32);
+            mma_f16(tmem + A_TM_D1, lw, dh, id, 1);
+            mma_f16(tmem + A_TM_D1, dh, lw, id, 1);
+          }
+        }
+        mma_commit(bar_m1);
+        started_m1 = true;
+      }
+      // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and
+      // the record's vectors; this thread: column j = tid % 64, rows 16 (tid / 64) .. +15
+      {
+        const int j = tid & 63, i0 = (tid >> 6) * 16;
+        const float gj = gam[j];
+#pragma unroll
+        for (int u2 = 0; u2 < 16; ++u2) {
+          const int i = i0 + u2;
+          if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
+        }
+      }
+      if (tid < 64) {
+        float* vec = reinterpret_cast<float*>(rec + R_VEC);
+        vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
+        if (tid == 0) vec[64] = eg[L - 1];
+      }
+      ok = mbar_wait(bar_m1, par);
+    }
+    if (!__syncthreads_or(!ok)) {
+      tc_fence_after();
+      // A (rows 0..63) -> fp32; P (rows 64..127) -> fp16 rows 64..127 of [Tb; P].
+      // This thread: row tl, columns wg*32 .. wg*32+31.
+      {
+        float x[32];
+        tmem_ld32(lane_base + A_TM_D1 + wg * 32, x);
+        if (tl < 64) {
+          const int i = tl;
+          const float bi = i < L ? bet[i] : 0.f;
+#pragma unroll
+          for (int e4 = 0; e4 < 32; e4 += 4) {
+            float4 v;
+            float* vf = reinterpret_cast<float*>(&v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j = wg * 32 + e4 + q;
+              vf[q] = j < i ? bi * Ef[i * ES + j] * x[e4 + q] : 0.f;
+            }
+            *reinterpret_cast<float4*>(Af + i * AS + wg * 32 + e4) = v;
+          }
+        } else {
+          const int i = tl - 64;
+          const float keep = i < L ? 1.f : 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int j = wg * 32 + q * 8 + e;
+              f[e] = j <= i ? keep * Ef[i * ES + j] * x[q * 8 + e] : 0.f;
+            }
+            st_half8(smem + A_TBP, swz(tl, wg * 4 + q), f);
+          }
+        }
+      }
+      __syncthreads();
+      solve_unit_lower<NTA>(Af, Tf, Xs, tid);
+      // this thread's 16 entries of T, row i = tid / 4, columns (tid % 4) * 16 ..
+      const int i = tid >> 2, qt = tid & 3;
+      float tv[16];
+#pragma unroll
+      for (int e4 = 0; e4 < 16; e4 += 4) {
+        const float4 t4 = *reinterpret_cast<const float4*>(Tf + i * AS + qt * 16 + e4);
+        tv[e4] = t4.x; tv[e4 + 1] = t4.y; tv[e4 + 2] = t4.z; tv[e4 + 3] = t4.w;
+      }
+      __syncthreads();  // the fp32 scratch is dead from here: the AW image goes over it
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float fb[8], fe[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = qt * 16 + q * 8 + e;
+          fb[e] = tv[q * 8 + e] * bet[j];
+          fe[e] = fb[e] * eg[j];
+        }
+        st_half8(smem + A_TBP, swz(i, qt * 2 + q), fb);  // Tb: A rows 0..63 and B block 0 of D2
+        st_half8(smem + A_AW, swz(i, qt * 2 + q), fe);   // Tbe: AW rows 0..63 and B block 1 of D2
+      }
+      // AW's second K atom: zero on rows 0..63, -E on rows 64..127
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = tid + NTA * k, r = e >> 3, ch = e & 7;
+        float f[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int ii = r - 64, j = ch * 8 + q;
+          f[q] = (r >= 64 && j == ii && ii < L) ? -eg[ii] : 0.f;
+        }
+        st_half8(smem + A_AW + 16384, swz(r, ch), f);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {  // D2 = [Tb; P] [Tb | Tbe]
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16(128, 128, false, true);
+        const uint64_t da = sdesc_sw128(sb + A_TBP, 16, 1024);
+        const uint64_t db = sdesc_sw128(sb + A_TBP, A_AW - A_TBP, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + A_TM_D2, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
+        mma_commit(bar_m2);
+        started_m2 = true;
+      }
+      ok = mbar_wait(bar_m2, par);
+    }
+    if (!__syncthreads_or(!ok)) {
+      tc_fence_after();
+      // rows 64..127 of D2: Pt (columns 0..63) over P in [Tb; P], Ph (64..127) -> AW rows 64..127
+      if (tl >= 64) {
+        float x[32];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          tmem_ld32(lane_base + A_TM_D2 + wg * 64 + hh * 32, x);
+          uint8_t* dst = smem + (wg == 0 ? A_TBP : A_AW);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st_half8(dst, swz(tl, hh * 4 + q), x + q * 8);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        // D3 = [Tbe 0; Ph -E] [K; Q] = [W; -Qt]
+        constexpr uint32_t id = idesc_f16(128, 128, false, true);
+        const uint64_t da = sdesc_sw128(sb + A_AW, 16, 1024);
+        const uint64_t db = sdesc_sw128(sb + A_KQ, 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16(tmem + A_TM_D3, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(db, kk * 2048),
+                  id, kk > 0);
+        // D4 = [Tb; Pt] V = [U; Pt V]
+        const uint64_t dt = sdesc_sw128(sb + A_TBP, 16, 1024);
+        const uint64_t dv = sdesc_sw128(sb + A_V, TILE, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + A_TM_D4, sdesc_add(dt, kk * 32), sdesc_add(dv, kk * 2048), id, kk > 0);
+        mma_commit(bar_m3);
+        started_m3 = true;
+      }
+      ok = mbar_wait(bar_m3, par);
+    }
+    if (!__syncthreads_or(!ok)) {
+      tc_fence_after();
+      // The record is assembled in shared memory regions the MMAs no longer
+      // read: [-W; Qt] over AW, [U; Pt V] over [K; Q], w * silu(z) over [Tb; Pt].
+      // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.  Each
+      // warpgroup's part leaves by bulk copy as soon as that warpgroup has
+      // written it (a named barrier per warpgroup), overlapping the rest.
+      const bool wg_lead = tl == 0;
+      float x[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(lane_base + A_TM_D3 + wg * 64 + hh * 32, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = -x[j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_half8(smem + A_AW + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+      }
+      fence_proxy_async();
+      bar_named(1 + wg, 128);
+      if (wg_lead) bulk_store(rec + R_WQ + wg * 16384, sb + A_AW + wg * 16384, 16384);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(lane_base + A_TM_D4 + wg * 64 + hh * 32, x);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_half8(smem + A_KQ + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
+      }
+      fence_proxy_async();
+      bar_named(1 + wg, 128);
+      if (wg_lead) {
+        bulk_store(rec + R_UO + wg * 16384, sb + A_KQ + wg * 16384, 16384);
+        bulk_commit();
+      }
+      // w * silu(z) in the chain's tile layout (value block ch / 8, row r, swizzled chunk)
+      if (gated) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+          const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
+          uint4 res;
+          __half2* r2 = reinterpret_cast<__half2*>(&res);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 zf = __bfloat1622float2(z2[q]);
+            r2[q] = __floats2half2_rn(wsm[ch * 8 + 2 * q] * silu_tanh(zf.x), wsm[ch * 8 + 2 * q + 1] * silu_tanh(zf.y));
+          }
+          *reinterpret_cast<uint4*>(smem + A_TBP + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+          bulk_store(rec + R_ZW, sb + A_TBP, 16384);
+          bulk_commit();
+        }
+      }
+      if (wg_lead) bulk_wait_read();  // shared memory stays valid until the copies have read it
+    }
+    // End of the unit: its copies have read shared memory and its TMEM has
+    // been read; the next unit's copies and MMAs may overwrite both.
+    fence_proxy_async();
+    tc_fence_before();
+    failed = __syncthreads_or(!ok);
+    tc_fence_after();
+    if (failed) break;
+    par ^= 1u;
+    u = u_next;
+    cur = nxt;
+  }
+  if (failed && tid == 0) {
+    // let every copy and MMA this thread started in the unit land (bounded)
     atomicExch(&g_split_error, 1);
-    mbar_wait(bar_load, 0, 100000000ull);
-    mbar_wait(bar_m3, 0, 100000000ull);
+    if (started_load) mbar_wait(bar_load, par, 100000000ull);
+    if (started_m1) mbar_wait(bar_m1, par, 100000000ull);
+    if (started_m2) mbar_wait(bar_m2, par, 100000000ull);
+    if (started_m3) mbar_wait(bar_m3, par, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();
@@ -1327,7 +1384,11 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)p.Hv, (unsigned)record_slots(p.N, p.T), 1);
+    // persistent: two CTAs per SM (shared memory, registers and TMEM allow two)
+    const int slots = (int)record_slots(p.N, p.T);
+    const long long units = (long long)slots * p.Hv;
+    const int ctas = (int)(units < 2LL * host::sm_count() ? units : 2LL * host::sm_count());
+    cfg.gridDim = dim3((unsigned)ctas, 1, 1);
     cfg.blockDim = dim3(NTA, 1, 1);
     cfg.dynamicSmemBytes = A_SMEM;
     cfg.stream = st;
@@ -1336,7 +1397,7 @@ cudaError_t launch_chunk_tc_split(const ChunkParams& p0, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, chunk_keys_kernel, mq, mk, mv, mql, mkl, p);
+    e = cudaLaunchKernelEx(&cfg, chunk_keys_kernel, mq, mk, mv, mql, mkl, p, slots);
     if (e != cudaSuccess) return e;
   }
   const int P = p.nseg;

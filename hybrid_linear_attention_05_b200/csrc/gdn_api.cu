@@ -129,7 +129,7 @@ int gdn_prefill_resolve_impl(const gdn_dims* dims, int N, int T_tot, int chunk, 
   switch (path) {
     case Path::Simt: return GDN_IMPL_SIMT;
     case Path::Tc: return GDN_IMPL_TC;
-    case Path::TcSplit: return workspace_bytes >= full ? GDN_IMPL_TC_SPLIT : GDN_ERR_WORKSPACE;
+    case Path::TcSplit: return workspace_bytes >= full ? (int)GDN_IMPL_TC_SPLIT : (int)GDN_ERR_WORKSPACE;
     case Path::TcFused: return GDN_IMPL_TC_FUSED;
     case Path::None: break;
   }
