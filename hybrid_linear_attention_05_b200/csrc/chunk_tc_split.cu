@@ -14,7 +14,8 @@
 //       D1 = [K; Q] K^T              ->  A = beta e^{gamma_i-gamma_j} K K^T,  P
 //       T  = (I + A)^-1              (CUDA cores, fp32)
 //       D2 = [Tb; P] [Tb | Tbe]      ->  Pt = P Tb,  Ph = P Tbe
-//       D3 = [Tbe 0; Ph -E] [K; Q]   =   [W; -Qt]    (E = diag(e^gamma))
+//       D3 = [Tbe; Ph] K             =   [W; P W],   Qt = E Q - P W in fp32
+//                                                  (E = diag(e^gamma))
 //       D4 = [Tb; Pt] V              =   [U; Pt V]
 //     and writes one record per (chunk, head): fp16 images of [-W; Qt] (the
 //     A operand of the chain, 128-byte swizzle) and of [U; Pt V] (swizzled
@@ -94,7 +95,7 @@ constexpr int NTA = 256;
 constexpr uint32_t A_KQ = 0;                     // [K;Q] tile: two dk halves x 128 rows x 128 B
 constexpr uint32_t A_TBP = 32768;                // [Tb; P], later [Tb; Pt]: K-major, 128 rows x 64
 constexpr uint32_t A_V = 49152;                  // V tile: two 64-column halves x 64 rows
-constexpr uint32_t A_AW = 65536;                 // [Tbe 0; Ph -E]: two 16 KiB K atoms
+constexpr uint32_t A_AW = 65536;                 // [Tbe; Ph] (16 KiB K atom), then [-W; Qt] (32 KiB)
 constexpr uint32_t A_AF = A_AW;                  // fp32 A [64][AS] (dead before A_AW is written)
 constexpr uint32_t A_TF = A_AF + 64 * AS * 4;    // fp32 T [64][AS]; before it the decay table E
 constexpr uint32_t A_X = A_TF + 64 * AS * 4;     // fp32 scratch of the inverse, 1024 floats
@@ -261,6 +262,42 @@ __global__ void __launch_bounds__(NTA, 2)
       bv_n = __ldg(p.beta + (size_t)nxt.h * p.T + nxt.c0 + tid);
     }
 
+    __syncthreads();
+    // while the operands are copied: the decay table E[i][j] = e^{gamma_i -
+    // gamma_j} (j <= i; this thread: column j = tid % 64, rows 16 (tid / 64)
+    // .. +15), the record's vectors, and w * silu(z) straight into the record
+    // in the chain's tile layout (value block ch / 8, row r, swizzled chunk;
+    // a warp's stores fill whole 128-byte lines)
+    {
+      const int j = tid & 63, i0 = (tid >> 6) * 16;
+      const float gj = gam[j];
+#pragma unroll
+      for (int u2 = 0; u2 < 16; ++u2) {
+        const int i = i0 + u2;
+        if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
+      }
+    }
+    if (tid < 64) {
+      float* vec = reinterpret_cast<float*>(rec + R_VEC);
+      vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
+      if (tid == 0) vec[64] = eg[L - 1];
+    }
+    if (gated) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
+        uint4 res;
+        __half2* r2 = reinterpret_cast<__half2*>(&res);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 zf = __bfloat1622float2(z2[q]);
+          r2[q] = __floats2half2_rn(wsm[ch * 8 + 2 * q] * silu_tanh(zf.x), wsm[ch * 8 + 2 * q + 1] * silu_tanh(zf.y));
+        }
+        *reinterpret_cast<uint4*>(rec + R_ZW + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
+      }
+    }
+
     bool ok = mbar_wait(bar_load, par);
     if (!__syncthreads_or(!ok)) {
       if (tid == 0) {  // D1 = [K; Q] K^T (+ [K_lo; Q_lo] K^T + [K; Q] K_lo^T)
@@ -281,22 +318,6 @@ __global__ void __launch_bounds__(NTA, 2)
         }
         mma_commit(bar_m1);
         started_m1 = true;
-      }
-      // meanwhile: the decay table E[i][j] = e^{gamma_i - gamma_j} (j <= i) and
-      // the record's vectors; this thread: column j = tid % 64, rows 16 (tid / 64) .. +15
-      {
-        const int j = tid & 63, i0 = (tid >> 6) * 16;
-        const float gj = gam[j];
-#pragma unroll
-        for (int u2 = 0; u2 < 16; ++u2) {
-          const int i = i0 + u2;
-          if (j <= i) Ef[i * ES + j] = __expf(gam[i] - gj);
-        }
-      }
-      if (tid < 64) {
-        float* vec = reinterpret_cast<float*>(rec + R_VEC);
-        vec[tid] = tid < L ? __expf(gam[L - 1] - gam[tid]) : 0.f;
-        if (tid == 0) vec[64] = eg[L - 1];
       }
       ok = mbar_wait(bar_m1, par);
     }
@@ -359,18 +380,6 @@ __global__ void __launch_bounds__(NTA, 2)
         st_half8(smem + A_TBP, swz(i, qt * 2 + q), fb);  // Tb: A rows 0..63 and B block 0 of D2
         st_half8(smem + A_AW, swz(i, qt * 2 + q), fe);   // Tbe: AW rows 0..63 and B block 1 of D2
       }
-      // AW's second K atom: zero on rows 0..63, -E on rows 64..127
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = tid + NTA * k, r = e >> 3, ch = e & 7;
-        float f[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int ii = r - 64, j = ch * 8 + q;
-          f[q] = (r >= 64 && j == ii && ii < L) ? -eg[ii] : 0.f;
-        }
-        st_half8(smem + A_AW + 16384, swz(r, ch), f);
-      }
       fence_proxy_async();
       tc_fence_before();
       __syncthreads();
@@ -405,14 +414,13 @@ __global__ void __launch_bounds__(NTA, 2)
       __syncthreads();
       if (tid == 0) {
         tc_fence_after();
-        // D3 = [Tbe 0; Ph -E] [K; Q] = [W; -Qt]
+        // D3 = [Tbe; Ph] K = [W; P W]  (Qt = E Q - P W is completed at extraction)
         constexpr uint32_t id = idesc_f16(128, 128, false, true);
         const uint64_t da = sdesc_sw128(sb + A_AW, 16, 1024);
         const uint64_t db = sdesc_sw128(sb + A_KQ, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_f16(tmem + A_TM_D3, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(db, kk * 2048),
-                  id, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + A_TM_D3, sdesc_add(da, kk * 32), sdesc_add(db, kk * 2048), id, kk > 0);
         // D4 = [Tb; Pt] V = [U; Pt V]
         const uint64_t dt = sdesc_sw128(sb + A_TBP, 16, 1024);
         const uint64_t dv = sdesc_sw128(sb + A_V, TILE, 1024);
@@ -427,17 +435,33 @@ __global__ void __launch_bounds__(NTA, 2)
     if (!__syncthreads_or(!ok)) {
       tc_fence_after();
       // The record is assembled in shared memory regions the MMAs no longer
-      // read: [-W; Qt] over AW, [U; Pt V] over [K; Q], w * silu(z) over [Tb; Pt].
+      // read: [-W; Qt] over AW, [U; Pt V] over [K; Q] (w * silu(z) went
+      // straight to global memory at the start of the unit).
       // Row tl: [-W; Qt] dk atom wg and [U; Pt V] value block wg.  Each
       // warpgroup's part leaves by bulk copy as soon as that warpgroup has
       // written it (a named barrier per warpgroup), overlapping the rest.
       const bool wg_lead = tl == 0;
+      // rows 64.. take e^{gamma_i} q_i (fp32, from the Q rows of [K; Q]; 0 past the chunk)
+      const float eq = tl >= 64 && tl - 64 < L ? eg[tl - 64] : 0.f;
       float x[32];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(lane_base + A_TM_D3 + wg * 64 + hh * 32, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = -x[j];
+        if (tl >= 64) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u4 = *reinterpret_cast<const uint4*>(smem + A_KQ + wg * 16384 + swz(tl, hh * 4 + q));
+            const __half2* h2 = reinterpret_cast<const __half2*>(&u4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(h2[e]);
+              x[q * 8 + 2 * e] = fmaf(eq, f.x, x[q * 8 + 2 * e]);
+              x[q * 8 + 2 * e + 1] = fmaf(eq, f.y, x[q * 8 + 2 * e + 1]);
+            }
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) st_half8(smem + A_AW + wg * 16384, swz(tl, hh * 4 + q), x + q * 8);
       }
@@ -455,28 +479,6 @@ __global__ void __launch_bounds__(NTA, 2)
       if (wg_lead) {
         bulk_store(rec + R_UO + wg * 16384, sb + A_KQ + wg * 16384, 16384);
         bulk_commit();
-      }
-      // w * silu(z) in the chain's tile layout (value block ch / 8, row r, swizzled chunk)
-      if (gated) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = tid + NTA * k, r = e >> 4, ch = e & 15;
-          const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv[k]);
-          uint4 res;
-          __half2* r2 = reinterpret_cast<__half2*>(&res);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 zf = __bfloat1622float2(z2[q]);
-            r2[q] = __floats2half2_rn(wsm[ch * 8 + 2 * q] * silu_tanh(zf.x), wsm[ch * 8 + 2 * q + 1] * silu_tanh(zf.y));
-          }
-          *reinterpret_cast<uint4*>(smem + A_TBP + (ch >> 3) * 8192 + swz(r, ch & 7)) = res;
-        }
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
-          bulk_store(rec + R_ZW, sb + A_TBP, 16384);
-          bulk_commit();
-        }
       }
       if (wg_lead) bulk_wait_read();  // shared memory stays valid until the copies have read it
     }
