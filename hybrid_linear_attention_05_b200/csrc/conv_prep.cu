@@ -241,7 +241,7 @@ constexpr uint32_t KW = KR * 256;   // the head's conv taps (128 x 4 bf16) follo
 constexpr uint32_t KBUF = 18432;    // one box (67 x 256 B) and the taps (1 KiB), rounded up to 1 KiB
 constexpr int KST = 2;               // boxes in flight per CTA
 constexpr uint32_t KSMEM = KST * KBUF + 64 + 1024;
-constexpr int KCTAS_PER_SM = 4;
+constexpr int KCTAS_PER_SM = 5;
 
 __device__ int g_conv_error = 0;  // nonzero: a box of conv_tma_kernel never landed
 
@@ -319,20 +319,15 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
     const int c0 = ct * D + cg * 8;
     const int t0 = tt * KT + tg * 8;
     const bool is_qk = ct < 2 * p.Hk, is_q = ct < p.Hk;
-    // gate inputs of this thread's tokens (first thread of a value head's
-    // token group), requested before the wait so that their latency overlaps it
-    const bool gates = !is_qk && cg == 0;
+    // gate inputs: in a value head's token group, thread cg < 8 takes token
+    // t0 + cg; requested before the wait so that their latency overlaps it
     const int hh = ct - 2 * p.Hk;
-    float av[8], bv[8];
+    const int tgate = t0 + cg;
+    const bool gates = !is_qk && cg < 8 && tgate < p.T;
+    float av = 0.f, bv = 0.f;
     if (gates) {
-      const __nv_bfloat16* ap = static_cast<const __nv_bfloat16*>(p.a);
-      const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int t = min(t0 + kk, p.T - 1);
-        av[kk] = ld_f(ap + (size_t)t * p.Hv + hh);
-        bv[kk] = ld_f(bp + (size_t)t * p.Hv + hh);
-      }
+      av = ld_f(static_cast<const __nv_bfloat16*>(p.a) + (size_t)tgate * p.Hv + hh);
+      bv = ld_f(static_cast<const __nv_bfloat16*>(p.b) + (size_t)tgate * p.Hv + hh);
     }
     int n = seq_of_token(p.cu_seqlens, p.N, min(t0, p.T - 1));
     int bos = clampi(__ldg(p.cu_seqlens + n), 0, p.T);
@@ -477,16 +472,10 @@ __global__ void __launch_bounds__(KNT, KCTAS_PER_SM)
       store(t, y0, f0);
       if (has1) store(t + 1, y1, f1);
     }
-    if (gates) {
-      // gates of value head hh for this thread's tokens
+    if (gates) {  // gates of value head hh for token tgate
       const float eA = expf(__ldg(p.A_log + hh)), db = __ldg(p.dt_bias + hh);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int t = t0 + kk;
-        if (t >= p.T) break;
-        p.g[(size_t)hh * p.T + t] = -eA * softplus_f(av[kk] + db);
-        p.beta[(size_t)hh * p.T + t] = sigmoid_f(bv[kk]);
-      }
+      p.g[(size_t)hh * p.T + tgate] = -eA * softplus_f(av + db);
+      p.beta[(size_t)hh * p.T + tgate] = sigmoid_f(bv);
     }
     __syncthreads();  // this buffer is read; the next iteration's prefetch may refill it
   }
