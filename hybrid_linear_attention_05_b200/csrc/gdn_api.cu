@@ -499,7 +499,7 @@ const char* gdn_status_string(gdn_status s) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_DIMS: return "inconsistent or out-of-range sizes";
     case GDN_ERR_ALIGN: return "a pointer is not 16-byte aligned";
-    case GDN_ERR_UNSUPPORTED: return "shape or option not supported by this build";
+    case GDN_ERR_UNSUPPORTED: return "shape or option not supported by the library";
     case GDN_ERR_CUDA: return "a CUDA call failed";
     case GDN_ERR_WORKSPACE: return "workspace missing or too small";
     case GDN_ERR_ALIAS: return "buffers that must not overlap overlap";

@@ -69,7 +69,7 @@ typedef enum {
   GDN_ERR_NULL = -1,        /* a required pointer is NULL                       */
   GDN_ERR_DIMS = -2,        /* inconsistent or out-of-range sizes               */
   GDN_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned                 */
-  GDN_ERR_UNSUPPORTED = -4, /* valid, but not a shape this build supports       */
+  GDN_ERR_UNSUPPORTED = -4, /* valid, but not a shape the library supports     */
   GDN_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed (launch, ...)  */
   GDN_ERR_WORKSPACE = -6,   /* workspace missing or smaller than required       */
   GDN_ERR_ALIAS = -7,       /* buffers that must not overlap do overlap         */
@@ -356,7 +356,11 @@ gdn_status gdn_decode(const gdn_dims* dims, const gdn_decode_args* args, void* s
  *   Supported: K a positive multiple of 64; every out_cols[i] a positive
  *   multiple of 8 with the ranges summing to N; ldx, ldw >= K and out_ld[i] >=
  *   out_cols[i], all multiples of 8 elements; every pointer 16-byte aligned.
- *   GDN_ERR_UNSUPPORTED / GDN_ERR_DIMS / GDN_ERR_ALIGN / GDN_ERR_NULL otherwise.
+ *   GDN_ERR_UNSUPPORTED / GDN_ERR_DIMS / GDN_ERR_ALIGN / GDN_ERR_NULL otherwise,
+ *   before anything is launched.  M = 0 does nothing.  The caller owns every
+ *   buffer; the call is asynchronous on `stream` and allocates nothing; columns
+ *   of an output row past its range are not written.  A bounded wait of the
+ *   kernel that gives up is reported by gdn_device_error.
  */
 typedef struct {
   const void* x;               /* device [M, K] bf16, rows ldx elements apart   */
@@ -381,7 +385,13 @@ gdn_status gdn_linear(const gdn_linear_args* args, void* stream);
  * gdn_layer_workspace_size gives the bytes for both (0 for invalid sizes);
  * with gdn_layer_activation_bytes + gdn_prefill_workspace_size bytes the
  * mixer runs without records.  The other arguments mean what they mean for
- * gdn_prefill. */
+ * gdn_prefill.  Errors: GDN_ERR_UNSUPPORTED for d_model or Hv*dv not a
+ * multiple of 64 (or Hv not a multiple of 8), GDN_ERR_WORKSPACE for a
+ * workspace smaller than the activations, GDN_ERR_NULL / GDN_ERR_ALIGN for
+ * missing or misaligned buffers -- these before any launch -- and what
+ * gdn_prefill returns for the mixer's arguments, which it checks after
+ * in_proj has been queued (out_proj is then not launched).  Everything runs
+ * in order on `stream`: in_proj, the mixer, out_proj. */
 typedef struct {
   const void* hidden;          /* device [T_tot, d_model] bf16                   */
   const void* w_in;            /* device [Cc + Hv*dv + 2*Hv, d_model] bf16       */

@@ -39,6 +39,8 @@ def bf(x):
     (1000, [512], 4096),
     (129, [8192, 4096, 32, 32], 4096),    # the 9B in_proj columns (qkv | z | b | a)
     (256, [4096], 4096),                  # the 9B out_proj
+    (1, [256], 64),                       # one row, one K tile
+    (7, [24, 8], 192),                    # a few rows, ranges inside one column tile
 ])
 def test_linear_matches_fp64_product(M, splits, K):
     rng = np.random.default_rng(M + K)
@@ -114,3 +116,38 @@ def test_layer_unit_q_scale_and_no_records():
                        li.w_in[Cc + HVd + w.Hv:], li.w_in[Cc + HVd:Cc + HVd + w.Hv], li.w_out, m.conv_w, m.A_log,
                        m.dt_bias, m.norm_w, m.initial_state, m.conv_state_in, scale=w.scale)
     assert relerr(np64(bufs.y), ref.y) <= PREFILL_TOL
+
+
+def test_linear_strided_rows():
+    """X and W with row strides larger than K (a column slice of wider
+    tensors), and an output range with a row stride larger than its columns."""
+    rng = np.random.default_rng(9)
+    M, N, K = 300, 136, 256
+    xw = bf16_round(rng.standard_normal((M, K + 64)).astype(np.float32))
+    ww = bf16_round((rng.standard_normal((N, K + 128)) * K ** -0.5).astype(np.float32))
+    x_t, w_t = bf(xw), bf(ww)
+    y = torch.zeros((M, N + 8), dtype=torch.bfloat16, device="cuda")
+    gdn.gdn_linear(x=x_t, w=w_t, M=M, N=N, K=K, ldx=K + 64, ldw=K + 128, outs=[(y, N, N + 8)])
+    torch.cuda.synchronize()
+    ref = xw[:, :K].astype(np.float64) @ ww[:, :K].astype(np.float64).T
+    got = np64(y)
+    assert relerr_beyond_bf16(got[:, :N], ref) <= 1e-4
+    assert np.all(got[:, N:] == 0)  # the columns past the range are not written
+
+
+def test_layer_matches_oracle_397b():
+    """The whole layer at the 397B shapes (16 key / 64 value heads, d_model
+    4096): in_proj of 20 608 columns, two sequences with initial states."""
+    w = WORKLOADS["prefill_varlen8_T65536_Hk16_Hv64_d128"]
+    li = make_layer(w, 4096, seqlens=(130, 77))
+    dl = api.layer_to_device(li)
+    bufs = api.layer_prefill(dl)
+    torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0
+    m = li.mixer
+    Cc, HVd = w.Cc, w.Hv * w.d
+    ref = oracle.layer(w.Hk, w.Hv, w.d, w.d, m.cu_seqlens, li.hidden, li.w_in[:Cc], li.w_in[Cc:Cc + HVd],
+                       li.w_in[Cc + HVd + w.Hv:], li.w_in[Cc + HVd:Cc + HVd + w.Hv], li.w_out, m.conv_w, m.A_log,
+                       m.dt_bias, m.norm_w, m.initial_state, m.conv_state_in, scale=w.scale)
+    assert relerr(np64(bufs.y), ref.y) <= PREFILL_TOL
+    assert relerr(np64(bufs.final_state), ref.mixer.final_state) <= PREFILL_TOL
