@@ -344,14 +344,17 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (a->N == 0) return a->T_tot == 0 ? GDN_OK : GDN_ERR_DIMS;
   const int d = dims->dk;
-  // no record workspace here, hence no two-kernel path; AUTO takes the fused
-  // kernel only when given its chain-queue workspace
-  Path path = a->impl == GDN_IMPL_TC_SPLIT ? Path::None : pick_path(a->impl, d, a->chunk, a->dtype, false);
+  // AUTO takes the fused kernel only when given its chain-queue workspace; the
+  // two-kernel path runs when asked for and given room for its records
+  Path path = pick_path(a->impl, d, a->chunk, a->dtype, false);
   if (a->impl == GDN_IMPL_AUTO && path == Path::TcFused &&
       (!a->workspace || a->workspace_bytes < kFusedSchedBytes))
     path = Path::Tc;
   if (path == Path::None) return GDN_ERR_UNSUPPORTED;
   if (path == Path::TcFused && (!a->workspace || a->workspace_bytes < kFusedSchedBytes)) return GDN_ERR_WORKSPACE;
+  if (path == Path::TcSplit &&
+      (!a->workspace || a->workspace_bytes < chunk_tc_split_record_bytes(a->N, a->T_tot, dims->Hv)))
+    return GDN_ERR_WORKSPACE;
   if (!aligned16(a->workspace)) return GDN_ERR_ALIGN;
   if (!a->cu_seqlens) return GDN_ERR_NULL;
   if (a->T_tot > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o)) return GDN_ERR_NULL;
@@ -370,6 +373,10 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
   ch.eps_norm = dims->eps_norm;
   ch.nseg = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (path == Path::TcSplit) {
+    ch.rec = static_cast<uint8_t*>(a->workspace);
+    return from_cuda(launch_chunk_tc_split(ch, st));
+  }
   if (path == Path::TcFused) {
     int* sched = static_cast<int*>(a->workspace);
     s = from_cuda(launch_chunk_fused_order(ch, sched, st));
@@ -381,6 +388,12 @@ gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* a, void* st
 }
 
 size_t gdn_core_workspace_size(int N) { return N < 0 ? 0 : kFusedSchedBytes; }
+
+size_t gdn_core_workspace_size_split(const gdn_dims* dims, int N, int T_tot) {
+  if (check_dims(dims) != GDN_OK || N < 0 || T_tot < 0) return 0;
+  const size_t rec = chunk_tc_split_record_bytes(N, T_tot, dims->Hv);
+  return rec > kFusedSchedBytes ? rec : kFusedSchedBytes;
+}
 
 gdn_status gdn_linear(const gdn_linear_args* a, void* stream) {
   if (!a) return GDN_ERR_NULL;

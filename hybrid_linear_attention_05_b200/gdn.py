@@ -38,6 +38,7 @@ GDN_IMPL_TC_FUSED = 4
 EXPORTED = ["gdn_prefill_workspace_size", "gdn_prefill_workspace_size_n", "gdn_prefill",
             "gdn_prefill_auto_segments", "gdn_prefill_resolve_impl", "gdn_prefill_noalloc", "gdn_prefill_state_map",
             "gdn_state_fold", "gdn_decode", "gdn_chunk_core", "gdn_core_workspace_size",
+            "gdn_core_workspace_size_split",
             "gdn_linear", "gdn_layer_activation_bytes", "gdn_layer_workspace_size", "gdn_layer_prefill",
             "gdn_device_error", "gdn_selftest_bounded_wait", "gdn_status_string", "gdn_version"]
 
@@ -132,6 +133,8 @@ def lib():
         L.gdn_chunk_core.restype = ctypes.c_int
         L.gdn_core_workspace_size.argtypes = [ctypes.c_int]
         L.gdn_core_workspace_size.restype = ctypes.c_size_t
+        L.gdn_core_workspace_size_split.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
+        L.gdn_core_workspace_size_split.restype = ctypes.c_size_t
         L.gdn_linear.argtypes = [ctypes.POINTER(gdn_linear_args), _vp]
         L.gdn_linear.restype = ctypes.c_int
         L.gdn_layer_activation_bytes.argtypes = [ctypes.POINTER(gdn_dims), ctypes.c_int, ctypes.c_int]
@@ -289,6 +292,10 @@ def gdn_decode(dims: gdn_dims, *, mixed_qkv, conv_w, a, b, A_log, dt_bias, z, no
 
 def gdn_core_workspace_size(N: int) -> int:
     return int(lib().gdn_core_workspace_size(int(N)))
+
+
+def gdn_core_workspace_size_split(dims: gdn_dims, N: int, T_tot: int) -> int:
+    return int(lib().gdn_core_workspace_size_split(ctypes.byref(dims), int(N), int(T_tot)))
 
 
 def gdn_chunk_core(dims: gdn_dims, *, q, k, v, g, beta, cu_seqlens, N, T_tot, chunk, dtype, o,

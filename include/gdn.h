@@ -441,14 +441,20 @@ typedef struct {
   const float* initial_state;
   float* final_state;
   float* o;
-  void* workspace;             /* device scratch of gdn_core_workspace_size bytes
-                                  (GDN_IMPL_TC_FUSED only; may be NULL otherwise) */
+  void* workspace;             /* device scratch: gdn_core_workspace_size bytes for
+                                  GDN_IMPL_TC_FUSED, gdn_core_workspace_size_split
+                                  bytes for GDN_IMPL_TC_SPLIT (its records); may be
+                                  NULL otherwise */
   size_t workspace_bytes;
 } gdn_core_args;
 
 /* Bytes of workspace gdn_chunk_core needs for N sequences (the chain queue of
  * GDN_IMPL_TC_FUSED). */
 size_t gdn_core_workspace_size(int N);
+/* Bytes for GDN_IMPL_TC_SPLIT (the two-kernel path's per-(chunk, head) records,
+ * and at least gdn_core_workspace_size, so one buffer serves every path); 0
+ * for invalid sizes.  With less, GDN_IMPL_TC_SPLIT returns GDN_ERR_WORKSPACE. */
+size_t gdn_core_workspace_size_split(const gdn_dims* dims, int N, int T_tot);
 
 gdn_status gdn_chunk_core(const gdn_dims* dims, const gdn_core_args* args, void* stream);
 

@@ -168,6 +168,24 @@ def test_core_rejects_bad_args(L):
     assert gdn.gdn_chunk_core(dims, **{**kw, "chunk": 8}) == gdn.GDN_ERR_UNSUPPORTED
 
 
+def test_core_split_needs_its_record_workspace(L):
+    """The two-kernel core takes one 82 432-byte record per (chunk slot, value
+    head); with less workspace it is refused before anything is launched."""
+    dims = gdn.make_dims(2, 4, 128)
+    N, T = 3, 1000
+    need = gdn.gdn_core_workspace_size_split(dims, N, T)
+    slots = T // 64 + N + 1
+    assert need >= slots * 4 * 82432 and need < slots * 4 * 82432 + 4096
+    assert need >= gdn.gdn_core_workspace_size(N)
+    assert gdn.gdn_core_workspace_size_split(dims, -1, T) == 0
+    kw = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu_seqlens=FAKE, N=N, T_tot=T, chunk=64,
+              dtype=gdn.GDN_F16, o=FAKE, impl=gdn.GDN_IMPL_TC_SPLIT, stream=0, raise_on_error=False)
+    assert gdn.gdn_chunk_core(dims, workspace=FAKE, workspace_bytes=need - 256, **kw) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_chunk_core(dims, workspace=None, workspace_bytes=0, **kw) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_chunk_core(dims, workspace=FAKE, workspace_bytes=need, **{**kw, "chunk": 32}) == \
+        gdn.GDN_ERR_UNSUPPORTED  # the tensor-core paths take chunks of 64
+
+
 def map_kwargs(**over):
     kw = dict(mixed_qkv=FAKE, conv_w=FAKE, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, cu_seqlens=FAKE,
               N=1, T_tot=16, chunk=64, dtype=gdn.GDN_BF16, map_out=FAKE + (1 << 30),

@@ -520,7 +520,9 @@ def run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, impl, S0=None, dtype=torch.
     t = lambda x, dt=dtype: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev, dt)
     o = torch.empty((T, Hv, d), dtype=torch.float32, device=dev)
     S = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
-    ws = torch.empty(gdn.gdn_core_workspace_size(N), dtype=torch.uint8, device=dev)
+    # room for every path: the fused kernel's queue, the two-kernel path's records
+    ws = torch.empty(gdn.gdn_core_workspace_size_split(gdn.make_dims(Hk, Hv, d), N, T), dtype=torch.uint8,
+                     device=dev)
     status = gdn.gdn_chunk_core(
         gdn.make_dims(Hk, Hv, d, scale=1.0), q=t(q), k=t(k), v=t(v),
         g=t(np.ascontiguousarray(g.T), torch.float32), beta=t(np.ascontiguousarray(beta.T), torch.float32),
@@ -536,7 +538,7 @@ def run_core(q, k, v, g, beta, cu, Hk, Hv, d, chunk, impl, S0=None, dtype=torch.
 
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
     ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.float32),
-    ("tc", 128, 64, torch.float16), ("fused", 128, 64, torch.float16)])
+    ("tc", 128, 64, torch.float16), ("split", 128, 64, torch.float16), ("fused", 128, 64, torch.float16)])
 def test_core_orthonormal_overwrite(impl, d, chunk, dtype):
     """alpha = 1, beta = 1, orthonormal keys: S k_i = v_i after writing, and
     a rewritten key returns its new value (exact in real arithmetic)."""
@@ -567,7 +569,7 @@ def test_core_orthonormal_overwrite(impl, d, chunk, dtype):
 
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
     ("simt", 64, 32, torch.float32), ("tc", 128, 64, torch.float16),
-    ("fused", 128, 64, torch.float16)])
+    ("split", 128, 64, torch.float16), ("fused", 128, 64, torch.float16)])
 def test_core_beta_zero_only_decays(impl, d, chunk, dtype):
     code = IMPLS[impl][0]
     rng = np.random.default_rng(61)
@@ -589,7 +591,7 @@ def test_core_beta_zero_only_decays(impl, d, chunk, dtype):
 @pytest.mark.parametrize("impl,d,chunk,dtype", [
     ("simt", 32, 16, torch.float32), ("simt", 128, 32, torch.bfloat16),
     ("simt", 64, 64, torch.float16), ("tc", 128, 64, torch.float16),
-    ("fused", 128, 64, torch.float16)])
+    ("split", 128, 64, torch.float16), ("fused", 128, 64, torch.float16)])
 def test_core_matches_oracle(impl, d, chunk, dtype):
     code = IMPLS[impl][0]
     rng = np.random.default_rng(62)
