@@ -151,3 +151,31 @@ def test_layer_matches_oracle_397b():
                        m.dt_bias, m.norm_w, m.initial_state, m.conv_state_in, scale=w.scale)
     assert relerr(np64(bufs.y), ref.y) <= PREFILL_TOL
     assert relerr(np64(bufs.final_state), ref.mixer.final_state) <= PREFILL_TOL
+
+
+def test_layer_full_size_window_tails():
+    """The whole layer at the 9B workload's full size (4 x 8192 tokens, d_model
+    4096) in the launch the bench times.  The last 128 tokens of every
+    sequence are checked against the oracle's layer run on that sequence's
+    last 1024 tokens alone, from a zero state, with the projected inputs of
+    the three tokens before them as the conv history: the workloads' gates
+    decay the state by e^-45 or more per 64-token chunk, so the state at the
+    window's start cannot matter."""
+    w = WORKLOADS["prefill_4x8192_Hk16_Hv32_d128"]
+    li = make_layer(w, 4096)
+    dl = api.layer_to_device(li)
+    bufs = api.layer_prefill(dl)
+    torch.cuda.synchronize()
+    assert gdn.gdn_device_error(True) == 0
+    m = li.mixer
+    Cc, HVd = w.Cc, w.Hv * w.d
+    W_qkv = li.w_in[:Cc]
+    y = bufs.y
+    for n in range(m.N):
+        end = int(m.cu_seqlens[n + 1])
+        lo = end - 1024
+        hist = oracle.bf16(li.hidden[lo - 3:lo].astype(np.float64) @ W_qkv.astype(np.float64).T).T[None]
+        ref = oracle.layer(w.Hk, w.Hv, w.d, w.d, [0, 1024], li.hidden[lo:end], W_qkv, li.w_in[Cc:Cc + HVd],
+                           li.w_in[Cc + HVd + w.Hv:], li.w_in[Cc + HVd:Cc + HVd + w.Hv], li.w_out, m.conv_w,
+                           m.A_log, m.dt_bias, m.norm_w, None, hist, scale=w.scale)
+        assert relerr(np64(y[end - 128:end]), ref.y[-128:]) <= PREFILL_TOL, n
